@@ -1,0 +1,187 @@
+/*
+ * adamw4.h -- C ABI of the fused 4-bit AdamW optimizer step (ZIP-SR / ZE-EDEN)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method: AdamW keeps a first moment m and a second moment v per weight;
+ * both are stored in 4 bits with one fp32 scale per block of 128 values
+ * (1.0625 bytes per parameter), m in NF4, v in one of two codes:
+ *   - ZIP-SR: the zero-inclusive code {k/15 * s}, rounded stochastically so
+ *     that the preconditioner h(v) = 1/(sqrt(v/(1-b2^t)) + eps) is unbiased;
+ *   - ZE-EDEN: the zero-excluded code {(k+1)/16 * s}, rounded to nearest,
+ *     with the block scale multiplied by ||x||^2 / max(<x,Q(x)>, 1e-12 s^2).
+ * The LM-head first moment is rounded stochastically (in state space) over
+ * the final 10% of training; normalisation-layer tensors and tensors under
+ * 4096 elements keep fp32 state.
+ *
+ * Sources (page title -- section):
+ *   "ZIP-SR / ZE-EDEN: 4-bit AdamW state quantization" (daiwk.github.io)
+ *       -- Method flowchart (decode, update moments, update weights,
+ *          quantise, pack), Core equation (h(v), the ZIP-SR probability, the
+ *          ZE-EDEN scale, weights updated before the moments are quantised),
+ *          Local reproduction notes (uint8 nibble packing, fp32 block scales,
+ *          fp32 fallback below 4096 elements).
+ *   "ZIP-SR 4-bit AdamW -- Preconditioner-space stochastic rounding -- What
+ *    does it mean?" (learnaivisually.com)
+ *       -- memory paragraph (128-value blocks with one fp32 scale, 1.0625
+ *          B/param, normalisation-layer states in fp32), ZE-EDEN paragraph
+ *          (NF4 for m, LM-head stochastic rounding in the final 10%).
+ *   "A New Approach to 4-bit AdamW Optimizer Quantization: Rounding in
+ *    Preconditioner Space" (kongchang.com)
+ *       -- AdamW and optimizer states; Preconditioner; Two Complementary
+ *          Technical Approaches.
+ *
+ * Conventions for every entry point:
+ *   - Status codes are returned; nothing is thrown across the ABI.  On an
+ *     error the handle's state is unchanged (except where stated) and
+ *     adamw4_last_error() describes it.
+ *   - Device pointers are raw CUDA device addresses on the handle's device.
+ *     Host pointers are plain process memory.
+ *   - A handle is not thread-safe; one thread at a time may use it.
+ *   - Work is enqueued on the caller's CUDA stream (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream).  A device-side failure of an
+ *     earlier step surfaces as ADAMW4_ECUDA on a later call.
+ */
+#ifndef ADAMW4_H
+#define ADAMW4_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ADAMW4_OK = 0,
+    ADAMW4_EINVAL = -1,     /* bad argument, bad descriptor, unknown handle    */
+    ADAMW4_EALIGN = -2,     /* a device pointer is not 16-byte aligned         */
+    ADAMW4_ENOMEM = -3,     /* device or host allocation failed                */
+    ADAMW4_ECUDA = -4,      /* a CUDA runtime call or kernel launch failed     */
+    ADAMW4_ESTATE = -5,     /* state blob does not match this handle           */
+    ADAMW4_ERANGE = -6      /* size above a stated maximum                     */
+} adamw4_status;
+
+typedef enum {
+    ADAMW4_V_ZIPSR = 0,     /* zero-inclusive code, preconditioner-space SR    */
+    ADAMW4_V_ZEEDEN = 1     /* zero-excluded code, EDEN block rescale          */
+} adamw4_vcode;
+
+/* Per-tensor flags. */
+enum {
+    ADAMW4_T_NORM = 1u,       /* normalisation-layer tensor: fp32 state        */
+    ADAMW4_T_LM_HEAD = 2u,    /* LM head: m rounded stochastically in the final 10% */
+    ADAMW4_T_FP32_STATE = 4u  /* force fp32 state                              */
+};
+
+/* Tensors below this many elements keep fp32 state. */
+#define ADAMW4_MIN_QUANT_NUMEL 4096
+/* Values per quantisation block (one fp32 scale per block per moment). */
+#define ADAMW4_BLOCK 128
+
+/* One parameter tensor, flattened row-major.
+ *   param      device, fp32, numel elements, 16-byte aligned; updated in place
+ *   grad_bf16  device, bf16 bit patterns, numel elements, 16-byte aligned; read
+ *   tensor_id  unique within a handle; keys the random draws, so it must stay
+ *              the same across a checkpoint and resume
+ *   flags      ADAMW4_T_* bits
+ *   weight_decay  decoupled weight decay of this tensor (w <- w (1 - lr wd))
+ * Both buffers are borrowed: they stay owned by the caller, and must stay
+ * allocated and at the same address until adamw4_destroy. */
+typedef struct {
+    float *param;
+    const uint16_t *grad_bf16;
+    int64_t numel;
+    uint32_t tensor_id;
+    uint32_t flags;
+    float weight_decay;
+} adamw4_tensor;
+
+/* Optimizer configuration.
+ *   lr            default learning rate (each step passes its own lr)
+ *   beta1, beta2  in [0, 1); eps > 0
+ *   vcode         ADAMW4_V_ZIPSR or ADAMW4_V_ZEEDEN
+ *   seed          key of the counter-based random draws
+ *   total_steps   T for the final-10% LM-head phase (active when 10 t > 9 T);
+ *                 0 means the phase never starts */
+typedef struct {
+    float lr, beta1, beta2, eps;
+    int32_t vcode;
+    uint64_t seed;
+    int64_t total_steps;
+} adamw4_config;
+
+typedef struct adamw4_handle adamw4_handle;
+
+/* Creates an optimizer over n tensors on CUDA device `device`.
+ * Validates every descriptor on the host (non-NULL pointers, 16-byte
+ * alignment, numel > 0, unique tensor_id), classifies each tensor (fp32 state
+ * when numel < 4096 or flagged NORM/FP32_STATE, else 4-bit), allocates the
+ * packed state (owned by the handle) and zeroes it, which is the all-zero
+ * initial state m = v = 0.  The step counter starts at t = 0.
+ * Returns ADAMW4_EINVAL / EALIGN for bad input, ENOMEM, ECUDA.
+ * On success *out receives the handle. */
+int adamw4_create(const adamw4_config *cfg, const adamw4_tensor *tensors, int n, int device,
+                  adamw4_handle **out);
+
+/* One optimizer step over every tensor: t <- t + 1, then for each weight
+ * decode (m, v), m <- b1 m + (1-b1) g, v <- b2 v + (1-b2) g^2,
+ * w <- w (1 - lr wd) - lr/(1-b1^t) * m / (sqrt(v)/sqrt(1-b2^t) + eps),
+ * then requantise and pack m and v.  A single kernel launch on `cuda_stream`;
+ * the call returns without waiting.  Reads the grads, updates the params and
+ * the state in place. */
+int adamw4_step(adamw4_handle *h, float lr, void *cuda_stream);
+
+/* The same step with host buffers: for each tensor i, copies grads_host[i]
+ * (numel bf16) to the tensor's device grad buffer, runs adamw4_step, then
+ * copies the updated params back to params_host[i] (numel fp32), all on
+ * `cuda_stream`, and waits for the stream.  Pinned host memory gives
+ * asynchronous copies; pageable memory works but is slower.
+ * Either array may be NULL to skip that direction. */
+int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_host,
+                     float *const *params_host, void *cuda_stream);
+
+/* Frees the state and the handle.  Unknown or already destroyed handles
+ * return ADAMW4_EINVAL. */
+int adamw4_destroy(adamw4_handle *h);
+
+/* Step counter: the last completed step (0 before the first).  After
+ * adamw4_set_step(h, 999) the next step runs at t = 1000. */
+int adamw4_get_step(const adamw4_handle *h, int64_t *t);
+int adamw4_set_step(adamw4_handle *h, int64_t t);
+
+/* Persistent optimizer-state bytes: 136 per 128-value block of each 4-bit
+ * tensor (64 + 64 code bytes, two fp32 scales) plus 8 per element of each fp32
+ * tensor; 1.0625 bytes per quantised parameter when numel is a multiple of
+ * 128.  Alignment padding inside the allocation (at most 508 bytes per fp32
+ * tensor) is not counted.  Returns -1 for an unknown handle. */
+int64_t adamw4_state_bytes(const adamw4_handle *h);
+
+/* Checkpoint.  The blob (little-endian) is
+ *   char magic[8] = "ADAMW4S1"; uint32 n_tensors; uint32 vcode; int64 t;
+ *   uint64 seed; uint64 payload_bytes;                       (40 bytes)
+ * then per tensor, in creation order:
+ *   uint32 tensor_id; uint32 kind (0 = 4-bit, 1 = fp32); int64 numel;
+ *   4-bit: m codes [nb*64] u8, v codes [nb*64] u8, m scales [nb] f32,
+ *          v scales [nb] f32, nb = ceil(numel/128);
+ *   fp32:  m [numel] f32, v [numel] f32.
+ * adamw4_state_export writes it to host_buf (capacity cap bytes; *used gets
+ * the size, also when cap is too small, which returns ADAMW4_ERANGE;
+ * host_buf may be NULL to query).  adamw4_state_import reads such a blob into
+ * a handle created over the same tensor list (same ids, kinds, numels,
+ * vcode and seed, else ADAMW4_ESTATE) and sets t.  Both synchronise the device
+ * and copy with the CUDA runtime. */
+int adamw4_state_export(const adamw4_handle *h, void *host_buf, int64_t cap, int64_t *used);
+int adamw4_state_import(adamw4_handle *h, const void *host_buf, int64_t len);
+
+/* Launch geometry used by adamw4_step (filled at create): CUDA blocks, threads
+ * per block, and 128-value work units (4-bit blocks plus fp32 chunks). */
+int adamw4_launch_info(const adamw4_handle *h, int *grid, int *block, int64_t *units);
+
+/* Message of the last failed call on this handle, or of the last failed call
+ * on this thread when h is NULL.  Never NULL; valid until the next call. */
+const char *adamw4_last_error(const adamw4_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ADAMW4_H */

@@ -1,0 +1,186 @@
+"""Pins of the oracle's ZIP-SR second-moment rounding (CPU only).
+
+ZIP-SR keeps the lower of two code points a < b with probability
+[h(v)-h(b)]/[h(a)-h(b)], h(v) = 1/(sqrt(v/(1-b2^t)) + eps) ("ZIP-SR / ZE-EDEN:
+4-bit AdamW state quantization", Core equation), so E[h(Q(v))] = h(v).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+U_STEP = 2.0 ** -23
+N_U = 1 << 23
+
+
+def f32(x):
+    return float(np.float32(x))
+
+
+def p_low_exact(x, dv, R, eps):
+    """Fraction of the 2^23 uniforms for which the oracle keeps the lower code
+    point.  The decision is monotone in u; bisection finds the threshold."""
+    k_lo = oracle.zipsr_decide(x, dv, R, eps, 0.0)
+    k_hi = oracle.zipsr_decide(x, dv, R, eps, 1.0 - U_STEP)
+    if k_lo == k_hi:
+        return (1.0 if k_lo == oracle.zipsr_bracket(x) else 0.0), k_lo
+    lo, hi = 0, N_U
+    while lo < hi:
+        j = (lo + hi) // 2
+        if oracle.zipsr_decide(x, dv, R, eps, j * U_STEP) == k_lo:
+            lo = j + 1
+        else:
+            hi = j
+    return lo / N_U, k_lo
+
+
+def h64(v, rs_bc2, eps):
+    return 1.0 / (np.sqrt(v) * rs_bc2 + eps)
+
+
+def test_worked_example_near_zero_cell(golden_dir):
+    """The worked example of "ZIP-SR 4-bit AdamW -- Preconditioner-space
+    stochastic rounding" (quiet-gradient paragraph): v = 1e-12 between the
+    code points 0 and b = 4e-12, eps = 1e-8, beta2 = 0.95, bias correction
+    ignored.  Checked at the two significant figures the page prints."""
+    ex = json.load(open(os.path.join(golden_dir, "worked_example_near_zero.json")))
+    inp, pr = ex["inputs"], ex["printed"]
+    eps = f32(inp["eps"])
+    v = f32(inp["v"])
+    # block scale s with b = s/15; x = v/s lies in the zero cell
+    s = f32(15 * inp["b"])
+    _, _, vz, vzs = oracle.tables()
+    b = f32(np.float32(vz[1]) * np.float32(s))
+    assert abs(b - inp["b"]) / inp["b"] < 1e-6
+    rs_bc2 = 1.0
+    R = f32(np.float32(np.sqrt(np.float32(s))) * np.float32(rs_bc2))
+    dv = f32(np.float32(np.sqrt(np.float32(v))) * np.float32(rs_bc2) + np.float32(eps))
+    x = f32(np.float32(v) * (np.float32(1.0) / np.float32(s)))
+    assert oracle.zipsr_bracket(x) == 0
+
+    p_zero, k = p_low_exact(x, dv, R, eps)
+    assert k == 0
+    # page: "about 0.5%", closed form eps(1 - sqrt(v/b))/(sqrt(v) + eps)
+    closed = inp["eps"] * (1 - np.sqrt(inp["v"] / inp["b"])) / (np.sqrt(inp["v"]) + inp["eps"])
+    assert abs(p_zero - closed) < 1e-5
+    assert round(p_zero, 3) == pr["zipsr_p_zero"]
+
+    # next-step multipliers through the oracle's own update (g = 0, b2 = 0.95)
+    sc = oracle.make_scalars(1e-3, 0.9, 0.95, eps, t=100000)
+    assert sc.rs_bc2 == 1.0
+
+    def next_mult(v_stored):
+        den, _, _, _ = oracle.update_elem(sc, 1.0, 0.0, 0.0, v_stored, 0.0)
+        return 1.0 / den
+
+    m_exact, m_b, m_zero = next_mult(v), next_mult(b), next_mult(0.0)
+
+    def sig2(a, b_):
+        return abs(a - b_) <= 0.05 * abs(b_)
+    assert sig2(m_exact, pr["next_multiplier_exact_v"])
+    assert sig2(m_b, pr["next_multiplier_b_stored"])
+    assert m_zero == pytest.approx(pr["next_multiplier_zero_stored"], rel=1e-6)
+    # state-space rounding stores zero with probability (b - v)/b
+    p_ss = (b - v) / b
+    e_ss = p_ss * m_zero + (1 - p_ss) * m_b
+    assert p_ss == pytest.approx(pr["state_space_p_zero"], abs=1e-6)
+    assert sig2(e_ss, pr["state_space_expected_multiplier"])
+    assert round(e_ss / m_exact) == pr["state_space_overshoot_factor"]
+    # ZIP-SR's expected next multiplier is about the exact one
+    e_zip = p_zero * m_zero + (1 - p_zero) * m_b
+    assert sig2(e_zip, pr["zipsr_expected_multiplier"])
+    assert abs(e_zip - m_exact) / m_exact < 0.02
+
+
+CASES = []
+for s in [6e-11, 1e-8, 3e-7, 1e-4, 2.5e-2]:
+    for xv in [0.0, 1e-6, 0.003, 0.02, 1 / 15, 0.07, 0.2, 0.5, 0.81, 14 / 15, 0.99, 1.0]:
+        for rs in [1.0, 31.6]:
+            CASES.append((s, xv, rs))
+
+
+@pytest.mark.parametrize("s,xv,rs_bc2", CASES)
+def test_exact_expectation_of_h(s, xv, rs_bc2):
+    """Enumerating every uniform: the oracle's canonical binary32 probability
+    equals the pages' formula in binary64 within 1e-6 plus the binary32
+    conditioning of the cell, and the expected preconditioner
+    equals h(v) (the preconditioner-space unbiasedness ZIP-SR is built on)."""
+    eps = f32(1e-8)
+    s = f32(s)
+    rs_bc2 = f32(rs_bc2)
+    _, _, vz, vzs = oracle.tables()
+    v = f32(np.float32(xv) * np.float32(s))
+    inv = np.float32(1.0) / np.float32(s)
+    x = f32(np.float32(v) * inv)
+    R = f32(np.sqrt(np.float32(s)) * np.float32(rs_bc2))
+    dv = f32(np.float32(np.sqrt(np.float32(v))) * np.float32(rs_bc2) + np.float32(eps))
+    k = oracle.zipsr_bracket(x)
+    assert float(vz[k]) <= x and (k == 14 or x < float(vz[k + 1]))
+    p, _ = p_low_exact(x, dv, R, eps)
+    # the pages' probability in binary64 with the code points' d values
+    da = float(vzs[k]) * R + eps
+    db = float(vzs[k + 1]) * R + eps
+    if db == da:
+        return  # flat preconditioner: the state-space fallback applies
+    p_ref = (1 / dv - 1 / db) / (1 / da - 1 / db)
+    p_ref = min(max(p_ref, 0.0), 1.0)
+    # binary32 conditioning: da and db are each rounded once (half an ulp of
+    # d); p moves by that over (db - da).  Plus the draw granularity.
+    cond = 4 * 2.0 ** -24 * db / (db - da)
+    assert abs(p - p_ref) < 1e-6 + U_STEP + cond
+    # E[h(Q)] = h(v): with d-values of the code points, in binary64
+    e_h = p * (1 / da) + (1 - p) * (1 / db)
+    assert abs(e_h - 1 / dv) <= (1e-6 + U_STEP + cond) * abs(1 / da - 1 / db) + 1e-12 / dv
+
+
+def test_zero_and_top_are_deterministic():
+    eps = f32(1e-8)
+    R = f32(np.sqrt(np.float32(1e-6)))
+    assert oracle.zipsr_decide(0.0, eps, R, eps, 0.999) == 0
+    assert oracle.zipsr_decide(1.0, R + eps, R, eps, 0.0) == 15
+
+
+@pytest.mark.parametrize("v_frac", [0.004, 0.03, 0.5])
+def test_monte_carlo_unbiased_in_h(v_frac):
+    """10^6 draws through the oracle's whole block step: the mean of the
+    stored preconditioner 1/(sqrt(Q(v)) rs_bc2 + eps) matches h(v) within
+    4 sigma, while the state-space mean of the code point would not near zero.
+    One element carries the block maximum; 127 carry v."""
+    _, _, vz, vzs = oracle.tables()
+    b1, b2, eps = np.float32(0.9), np.float32(0.999), np.float32(1e-8)
+    # zero state: v1 = (1-b2) g^2 ; choose g so that v1 spans the near-zero cell
+    g_max = np.float32(3e-5)
+    g_small = np.float32(g_max * np.sqrt(np.float32(v_frac)))
+    from workloads import bf16_bits, bf16_to_f32
+    g = np.full(128, g_small, np.float32)
+    g[0] = g_max
+    gb = bf16_bits(g)
+    gf = bf16_to_f32(gb)
+    omb2 = np.float32(1.0) - b2
+    v1 = (omb2 * (gf * gf)).astype(np.float32)
+    hs, h_true = [], None
+    n_rep = 8000
+    for rep in range(n_rep):
+        sc = oracle.make_scalars(1e-3, b1, b2, eps, t=1, seed=rep)
+        w = np.zeros(128, np.float32)
+        mc = np.zeros(64, np.uint8)
+        vc = np.zeros(64, np.uint8)
+        ms = np.zeros(1, np.float32)
+        vs = np.zeros(1, np.float32)
+        oracle.lib().oracle_block4(sc, np.float32(1.0), 0, 0, 0, 0, 128, w, gb, mc, ms, vc, vs)
+        codes = np.empty(128, np.int64)
+        codes[0::2] = vc & 15
+        codes[1::2] = vc >> 4
+        rs = np.float64(sc.rs_bc2)
+        R = np.sqrt(np.float64(vs[0])) * rs
+        h_code = 1.0 / (np.sqrt(vz[codes[1:]].astype(np.float64)) * R + float(eps))
+        hs.append(h_code)
+        if h_true is None:
+            h_true = 1.0 / (np.sqrt(np.float64(v1[1])) * rs + float(eps))
+    hs = np.concatenate(hs)
+    assert hs.size >= 10 ** 6
+    mean, sd = hs.mean(), hs.std() / np.sqrt(hs.size)
+    assert abs(mean - h_true) < 4 * sd + 1e-6 * h_true
