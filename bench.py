@@ -1,0 +1,386 @@
+"""Benchmark of the fused 4-bit AdamW step (ZIP-SR / ZE-EDEN) on B200.
+
+One step = one pass of the whole path over the GPT-style 2.7B tensor list (32
+layers, d 2560, FFN 10,240, vocab 50,304, context 2048, untied head; 195
+4-bit tensors, 194 fp32-state tensors): decode, moment update, weight update,
+requantise and pack, as one kernel launch.  Inputs are synthetic and resident
+in HBM (19.7 GB > L2, so no L2 flush is needed between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--vcode zipsr|zeeden]
+                    [--impl ours|reference]
+
+With N > 1 (under torch.distributed.run) every rank steps its own replica of
+the workload on its own GPU: the path has no exchange step, so there is no
+data-path collective (weak scaling); the time is the max over ranks.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+WORKLOAD = "gpt-2.7b"        # the benchmark workload; --workload picks a profiling case
+METRIC = "fused 4-bit AdamW step Gparams/s; achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "bit_quantized_optimizer_b200", "csrc", "adamw4.cu")
+
+
+def is_fp32_state(numel, flags):
+    return numel < 4096 or bool(flags & (workloads.T_NORM | workloads.T_FP32_STATE))
+
+
+def algorithmic_bytes(ts):
+    """HBM bytes one step must move: per 4-bit value, w read+write (8), bf16
+    grad read (2); per 128-value block, m and v codes (64 B each) and scales
+    (4 B each), read and written; per fp32-state value 4+4+2+8+8."""
+    b = 0
+    for t in ts:
+        n = t["numel"]
+        if is_fp32_state(n, t["flags"]):
+            b += 26 * n
+        else:
+            b += 10 * n + 2 * 136 * ((n + 127) // 128)
+    return b
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sha():
+    return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+
+
+def traffic_record(vcode_name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", f"adamw4_step_{WORKLOAD}_{vcode_name}_traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    if d.get("kernel_source_sha256") != kernel_sha():
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    Q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5:
+            time.sleep(0.02)
+        self.skip = len(self.lines)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [l.split(",") for l in self.lines[max(self.skip - 1, 0):] if l.count(",") >= 6]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[3:7]):
+                if v.strip().lower() in ("active", "1", "yes"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].strip().replace(".", "").isdigit()
+                else None, "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(ts, params, grads, vcode, target_s=10.0, per_tensor_cap=1 << 18):
+    """The oracle on the host cores over a bounded sample of the workload: the
+    first up-to-256K values of every tensor of the list (about 40M params),
+    one step repeated until about `target_s` seconds have passed."""
+    import torch
+    import oracle
+    sub, ws, gs = [], [], []
+    for t, p, g in zip(ts, params, grads):
+        n = min(t["numel"], per_tensor_cap)
+        tt = dict(t)
+        tt["numel"] = n
+        sub.append(tt)
+        ws.append(p[:n].cpu().numpy().copy())
+        gs.append(g[:n].view(torch.int16).cpu().numpy().view(np.uint16).copy())
+    nthreads = max(1, oracle.max_threads())
+    o = oracle.OracleAdamW4(vcode=vcode, tensors=sub, nthreads=nthreads)
+    nparams = sum(t["numel"] for t in sub)
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        o.step(ws, gs)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= target_s:
+            break
+    return {"value": nparams * steps / el / 1e9, "unit": "Gparams/s", "cores": nthreads,
+            "kind": "oracle",
+            "sample": f"first <= {per_tensor_cap} values of each of the {len(sub)} tensors of the "
+                      f"{WORKLOAD} list ({nparams} params), {steps} step(s), {el:.1f} s, "
+                      f"{nthreads} OpenMP threads"}
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    vcode = 0 if args.vcode == "zipsr" else 1
+    ts = workloads.tensor_list(WORKLOAD)
+    # per step: the first up-to-64K values of every tensor (about 12M params);
+    # inputs from the host generator, state zero-initialised
+    cap = 1 << 16
+    sub = []
+    for t in ts:
+        tt = dict(t)
+        tt["numel"] = min(t["numel"], cap)
+        sub.append(tt)
+    wts = workloads.host_weights(WORKLOAD, sub)
+    grs = workloads.host_grads(WORKLOAD, sub, 1)
+    nthreads = max(1, oracle.max_threads())
+    o = oracle.OracleAdamW4(vcode=vcode, tensors=sub, nthreads=nthreads)
+    nparams = sum(t["numel"] for t in sub)
+    for _ in range(args.warmup):
+        o.step(wts, grs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        o.step(wts, grs)
+    el = time.perf_counter() - t0
+    value = nparams * args.steps / el / 1e9
+    sample = (f"first <= {cap} values of each of the {len(sub)} tensors of the {WORKLOAD} list "
+              f"({nparams} params) per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Gparams/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "vcode": args.vcode, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "Gparams/s", "cores": nthreads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "Gparams/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def e2e_run(B, opt, ts, grads, nparams, stream, ws_, args):
+    """Same metric through adamw4_step_host: every step copies the grads from
+    pinned host memory to the device, runs the step and copies the updated
+    params back to pinned host memory."""
+    import torch
+    e2e_steps = max(1, min(3, args.steps))
+    hg = torch.empty(nparams, dtype=torch.int16).pin_memory()
+    hp = torch.empty(nparams, dtype=torch.float32).pin_memory()
+    offs = np.cumsum([0] + [t["numel"] for t in ts])
+    gptrs = [hg.data_ptr() + 2 * int(o) for o in offs[:-1]]
+    pptrs = [hp.data_ptr() + 4 * int(o) for o in offs[:-1]]
+    for g, o, t in zip(grads, offs[:-1], ts):
+        hg[int(o):int(o) + t["numel"]].copy_(g.view(torch.int16).cpu())
+    B.adamw4_step_host(opt.handle, 1e-3, gptrs, pptrs, stream.cuda_stream)   # warm
+    barrier(ws_)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        B.adamw4_step_host(opt.handle, 1e-3, gptrs, pptrs, stream.cuda_stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws_)
+    h2d = 2 * nparams
+    d2h = 4 * nparams
+    del hg, hp
+    return {"value": ws_ * nparams / (e2e_ms * 1e-3) / 1e9, "unit": "Gparams/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+
+def run_ours(args):
+    import torch
+    ws_, rank, local = dist_setup(args.gpus)
+    import bit_quantized_optimizer_b200 as B
+    B.lib()  # fail loudly if the extension is missing
+    vcode = B.ADAMW4_V_ZIPSR if args.vcode == "zipsr" else B.ADAMW4_V_ZEEDEN
+    ts = workloads.tensor_list(WORKLOAD)
+    params, grads = workloads.device_inputs(WORKLOAD, ts, seed=rank)
+    torch.cuda.synchronize()
+    opt = B.AdamW4(params, grads, ts, lr=1e-3, vcode=vcode, seed=rank)
+    grid, block, units = B.adamw4_launch_info(opt.handle)
+    nparams = sum(t["numel"] for t in ts)
+    alg_bytes = algorithmic_bytes(ts)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        opt.step(stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(ws_)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        opt.step(stream=stream.cuda_stream)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws_)
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(total_ms, ws_)
+    avg_launch_ms = max_over_ranks(float(np.mean(launch_ms)), ws_)
+
+    # e2e through the C ABI with host buffers: grads H2D, step, params D2H
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_run(B, opt, ts, grads, nparams, stream, ws_, args)
+
+    cpu = None
+    if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(ts, params, grads, vcode)
+
+    if rank == 0:
+        peak, peak_kind = peaks()
+        achieved = alg_bytes / (avg_launch_ms * 1e-3) / 1e9
+        ms_per_step = total_ms / args.steps
+        line = {
+            "metric": METRIC,
+            "value": ws_ * nparams / (ms_per_step * 1e-3) / 1e9,
+            "unit": "Gparams/s",
+            "n_gpus": ws_,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "vcode": args.vcode, "params": nparams,
+                       "tensors": len(ts), "algorithmic_bytes_per_step": alg_bytes,
+                       "parallelism": f"replicas x{ws_} (no data-path collective)",
+                       "l2": "inputs 19.7 GB > 126 MB L2; no flush",
+                       "grid": grid, "block": block, "units": units},
+            "hbm_gbs": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": traffic_record(args.vcode)},
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if ws_ > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--vcode", choices=["zipsr", "zeeden"], default="zipsr")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["gpt-2.7b", "llama-1.1b", "gpt-130m"],
+                    help="tensor list (the benchmark is gpt-2.7b; the others are profiling cases)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)     # at least three untimed steps
+    globals()["WORKLOAD"] = args.workload
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

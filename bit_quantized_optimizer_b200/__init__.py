@@ -1,0 +1,216 @@
+"""Python binding of the fused 4-bit AdamW step (ZIP-SR / ZE-EDEN) for B200.
+
+Argument marshalling only: every step of the method runs in the CUDA kernels
+of ``libadamw4.so`` (built in-tree by ``build.py``).  There is no fallback: if
+the library is missing or cannot load, importing the functions raises.
+
+The functions carry the C ABI's names (``include/adamw4.h``); ``AdamW4``
+wraps them for torch tensors (fp32 params, bf16 grads on one CUDA device).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_T_NORM", "ADAMW4_T_LM_HEAD",
+           "ADAMW4_T_FP32_STATE", "AdamW4Error", "adamw4_tensor", "adamw4_config", "lib",
+           "adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
+           "adamw4_get_step", "adamw4_set_step", "adamw4_state_bytes", "adamw4_state_export",
+           "adamw4_state_import", "adamw4_launch_info", "adamw4_last_error", "AdamW4",
+           "is_fp32_state", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libadamw4.so")
+
+ADAMW4_OK = 0
+ADAMW4_V_ZIPSR = 0
+ADAMW4_V_ZEEDEN = 1
+ADAMW4_T_NORM = 1
+ADAMW4_T_LM_HEAD = 2
+ADAMW4_T_FP32_STATE = 4
+MIN_QUANT_NUMEL = 4096
+BLOCK = 128
+
+STATUS = {0: "ADAMW4_OK", -1: "ADAMW4_EINVAL", -2: "ADAMW4_EALIGN", -3: "ADAMW4_ENOMEM",
+          -4: "ADAMW4_ECUDA", -5: "ADAMW4_ESTATE", -6: "ADAMW4_ERANGE"}
+
+
+class AdamW4Error(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class adamw4_tensor(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("grad_bf16", ctypes.c_void_p),
+                ("numel", ctypes.c_int64), ("tensor_id", ctypes.c_uint32),
+                ("flags", ctypes.c_uint32), ("weight_decay", ctypes.c_float)]
+
+
+class adamw4_config(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("vcode", ctypes.c_int32), ("seed", ctypes.c_uint64),
+                ("total_steps", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libadamw4.so; raises if it is absent (build it with build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run bit_quantized_optimizer_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        H = c.c_void_p
+        L.adamw4_create.argtypes = [c.POINTER(adamw4_config), c.POINTER(adamw4_tensor), c.c_int,
+                                    c.c_int, c.POINTER(H)]
+        L.adamw4_step.argtypes = [H, c.c_float, c.c_void_p]
+        L.adamw4_step_host.argtypes = [H, c.c_float, c.POINTER(c.c_void_p),
+                                       c.POINTER(c.c_void_p), c.c_void_p]
+        L.adamw4_destroy.argtypes = [H]
+        L.adamw4_get_step.argtypes = [H, c.POINTER(c.c_int64)]
+        L.adamw4_set_step.argtypes = [H, c.c_int64]
+        L.adamw4_state_bytes.argtypes = [H]
+        L.adamw4_state_bytes.restype = c.c_int64
+        L.adamw4_state_export.argtypes = [H, c.c_void_p, c.c_int64, c.POINTER(c.c_int64)]
+        L.adamw4_state_import.argtypes = [H, c.c_void_p, c.c_int64]
+        L.adamw4_launch_info.argtypes = [H, c.POINTER(c.c_int), c.POINTER(c.c_int),
+                                         c.POINTER(c.c_int64)]
+        L.adamw4_last_error.argtypes = [H]
+        L.adamw4_last_error.restype = c.c_char_p
+        for f in ("adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
+                  "adamw4_get_step", "adamw4_set_step", "adamw4_state_export",
+                  "adamw4_state_import", "adamw4_launch_info"):
+            getattr(L, f).restype = c.c_int
+        _lib = L
+    return _lib
+
+
+def adamw4_last_error(h=None) -> str:
+    return lib().adamw4_last_error(h).decode()
+
+
+def _check(rc, h=None):
+    if rc != ADAMW4_OK:
+        raise AdamW4Error(rc, adamw4_last_error(h))
+
+
+def adamw4_create(cfg: adamw4_config, tensors, device: int = 0):
+    arr = (adamw4_tensor * max(len(tensors), 1))(*tensors)
+    h = ctypes.c_void_p()
+    _check(lib().adamw4_create(ctypes.byref(cfg), arr, len(tensors), device, ctypes.byref(h)))
+    return h
+
+
+def adamw4_step(h, lr: float, stream=None):
+    _check(lib().adamw4_step(h, lr, stream), h)
+
+
+def adamw4_step_host(h, lr: float, grads_host, params_host, stream=None):
+    """grads_host / params_host: sequences of host addresses (or None)."""
+    g = (ctypes.c_void_p * len(grads_host))(*grads_host) if grads_host is not None else None
+    p = (ctypes.c_void_p * len(params_host))(*params_host) if params_host is not None else None
+    _check(lib().adamw4_step_host(h, lr, g, p, stream), h)
+
+
+def adamw4_destroy(h):
+    _check(lib().adamw4_destroy(h))
+
+
+def adamw4_get_step(h) -> int:
+    t = ctypes.c_int64()
+    _check(lib().adamw4_get_step(h, ctypes.byref(t)), h)
+    return t.value
+
+
+def adamw4_set_step(h, t: int):
+    _check(lib().adamw4_set_step(h, t), h)
+
+
+def adamw4_state_bytes(h) -> int:
+    b = lib().adamw4_state_bytes(h)
+    if b < 0:
+        raise AdamW4Error(-1, "unknown handle")
+    return b
+
+
+def adamw4_state_export(h) -> bytes:
+    used = ctypes.c_int64()
+    _check(lib().adamw4_state_export(h, None, 0, ctypes.byref(used)), h)
+    buf = ctypes.create_string_buffer(used.value)
+    _check(lib().adamw4_state_export(h, buf, used.value, ctypes.byref(used)), h)
+    return buf.raw
+
+
+def adamw4_state_import(h, blob: bytes):
+    _check(lib().adamw4_state_import(h, blob, len(blob)), h)
+
+
+def adamw4_launch_info(h):
+    g, b, u = ctypes.c_int(), ctypes.c_int(), ctypes.c_int64()
+    _check(lib().adamw4_launch_info(h, ctypes.byref(g), ctypes.byref(b), ctypes.byref(u)), h)
+    return g.value, b.value, u.value
+
+
+def is_fp32_state(numel: int, flags: int) -> bool:
+    """The library's classification rule: fp32 state below 4096 elements or
+    for NORM / FP32_STATE tensors."""
+    return numel < MIN_QUANT_NUMEL or bool(flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE))
+
+
+class AdamW4:
+    """Optimizer over torch tensors: fp32 params and bf16 grads (contiguous,
+    16-byte aligned, on one CUDA device).  ``specs`` is a list of dicts with
+    tensor_id, flags and weight_decay, parallel to ``params``."""
+
+    def __init__(self, params, grads, specs, lr=1e-3, betas=(0.9, 0.999), eps=1e-8,
+                 vcode=ADAMW4_V_ZIPSR, seed=0, total_steps=0):
+        import torch
+        self.params, self.grads = list(params), list(grads)
+        dev = self.params[0].device.index if self.params else 0
+        ts = []
+        for p, g, s in zip(self.params, self.grads, specs):
+            if p.dtype != torch.float32 or g.dtype != torch.bfloat16:
+                raise TypeError("params must be float32 and grads bfloat16")
+            if not (p.is_contiguous() and g.is_contiguous()) or p.numel() != g.numel():
+                raise ValueError("params and grads must be contiguous and of equal size")
+            ts.append(adamw4_tensor(p.data_ptr(), g.data_ptr(), p.numel(), s["tensor_id"],
+                                    s.get("flags", 0), s.get("weight_decay", 0.0)))
+        self.cfg = adamw4_config(lr, betas[0], betas[1], eps, vcode, seed, total_steps)
+        self.lr = lr
+        self.handle = adamw4_create(self.cfg, ts, dev)
+
+    def step(self, lr=None, stream=None):
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+        adamw4_step(self.handle, self.lr if lr is None else lr, s)
+
+    @property
+    def t(self) -> int:
+        return adamw4_get_step(self.handle)
+
+    @t.setter
+    def t(self, value: int):
+        adamw4_set_step(self.handle, value)
+
+    def state_bytes(self) -> int:
+        return adamw4_state_bytes(self.handle)
+
+    def state_dict_blob(self) -> bytes:
+        return adamw4_state_export(self.handle)
+
+    def load_state_blob(self, blob: bytes):
+        adamw4_state_import(self.handle, blob)
+
+    def close(self):
+        if self.handle is not None:
+            adamw4_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,49 @@
+"""Builds libadamw4.so in-tree with nvcc for sm_100a.
+
+Flags that matter for the results: -fmad=false (no implicit multiply-add
+contraction), IEEE division and square root, denormals kept.  The kernel names
+every fused multiply-add it wants explicitly, so the result does not depend on
+the compiler's contraction choices.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "csrc", "adamw4.cu")
+OUT = os.path.join(HERE, "libadamw4.so")
+DEPS = [SRC, os.path.join(HERE, "csrc", "nf4_table.h"),
+        os.path.join(os.path.dirname(HERE), "include", "adamw4.h")]
+
+
+def nvcc():
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def flags():
+    return ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+            "-fmad=false", "-prec-div=true", "-prec-sqrt=true", "-ftz=false",
+            "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "-shared", "-Xptxas", "-v"]
+
+
+def build(force=False, verbose=False):
+    if not force and os.path.exists(OUT) and all(
+            os.path.getmtime(OUT) >= os.path.getmtime(d) for d in DEPS):
+        return OUT
+    tmp = OUT + f".tmp{os.getpid()}"
+    cmd = [nvcc()] + flags() + [SRC, "-o", tmp]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
+    if verbose:
+        sys.stderr.write(r.stderr)
+    os.replace(tmp, OUT)
+    return OUT
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose=True))

@@ -260,11 +260,17 @@ class OracleAdamW4:
     def m_sr(self, ts: TensorState, s: Scalars) -> int:
         return int(bool(ts.flags & T_LM_HEAD) and s.lm_sr_active)
 
-    def step(self, params, grads, lr=None):
+    def step(self, params, grads, lr=None, only=None, advance=True):
+        """One step over every tensor, or over the tensors listed in `only`
+        (then params/grads hold just those, in that order).  With
+        advance=False the step counter is not incremented first."""
         L = lib()
-        self.t += 1
+        if advance:
+            self.t += 1
         s = self.scalars(self.lr if lr is None else lr)
-        for ts, w, g in zip(self.tensors, params, grads):
+        idx = range(len(self.tensors)) if only is None else list(only)
+        for i, w, g in zip(idx, params, grads):
+            ts = self.tensors[i]
             assert w.dtype == np.float32 and g.dtype == np.uint16 and w.size == ts.numel
             if ts.fp32:
                 L.oracle_step_fp32(ctypes.byref(s), ts.weight_decay, ts.numel, w, g, ts.m, ts.v)

@@ -1,0 +1,117 @@
+"""The C ABI library: builds, loads, exports every declared entry point, and
+rejects bad input on the host before touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_quantized_optimizer_b200 as B
+from bit_quantized_optimizer_b200 import build as B_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B_build.build()
+    return B.lib()
+
+
+def declared_functions():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(adamw4_[a-z_0-9]+)\s*\(", txt))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert "adamw4_create" in names and "adamw4_step" in names and "adamw4_destroy" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def _cfg(**kw):
+    c = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, vcode=0, seed=0, total_steps=0)
+    c.update(kw)
+    return B.adamw4_config(c["lr"], c["beta1"], c["beta2"], c["eps"], c["vcode"], c["seed"],
+                           c["total_steps"])
+
+
+def _create(cfg, ts):
+    arr = (B.adamw4_tensor * max(len(ts), 1))(*ts)
+    h = ctypes.c_void_p()
+    rc = B.lib().adamw4_create(ctypes.byref(cfg), arr, len(ts), 0, ctypes.byref(h))
+    return rc, h
+
+
+P0 = 0x7F0000000000   # fake, aligned device addresses: validation never dereferences them
+
+
+@pytest.mark.parametrize("kw,code", [(dict(beta1=1.0), -1), (dict(beta2=-0.1), -1),
+                                     (dict(eps=0.0), -1), (dict(vcode=2), -1),
+                                     (dict(total_steps=-1), -1), (dict(lr=float("nan")), -1)])
+def test_bad_config(L, kw, code):
+    rc, _ = _create(_cfg(**kw), [B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, 0.0)])
+    assert rc == code
+    assert B.adamw4_last_error()
+
+
+@pytest.mark.parametrize("t,code,msg", [
+    (B.adamw4_tensor(0, P0, 4096, 0, 0, 0.0), -1, "NULL"),
+    (B.adamw4_tensor(P0, 0, 4096, 0, 0, 0.0), -1, "NULL"),
+    (B.adamw4_tensor(P0 + 4, P0 + (1 << 30), 4096, 0, 0, 0.0), -2, "aligned"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30) + 8, 4096, 0, 0, 0.0), -2, "aligned"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 0, 0, 0, 0.0), -1, "numel"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), -5, 0, 0, 0.0), -1, "numel"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, float("inf")), -1, "weight_decay"),
+])
+def test_bad_tensor(L, t, code, msg):
+    rc, _ = _create(_cfg(), [t])
+    assert rc == code
+    assert msg in B.adamw4_last_error()
+
+
+def test_duplicate_ids_and_overlaps(L):
+    a = B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 7, 0, 0.0)
+    b = B.adamw4_tensor(P0 + (1 << 20), P0 + (1 << 31), 4096, 7, 0, 0.0)
+    rc, _ = _create(_cfg(), [a, b])
+    assert rc == -1 and "duplicate" in B.adamw4_last_error()
+    # param of b inside param of a
+    b = B.adamw4_tensor(P0 + 1024, P0 + (1 << 31), 4096, 8, 0, 0.0)
+    rc, _ = _create(_cfg(), [a, b])
+    assert rc == -1 and "overlaps" in B.adamw4_last_error()
+    # grad of b inside param of a
+    b = B.adamw4_tensor(P0 + (1 << 20), P0 + 4096, 4096, 8, 0, 0.0)
+    rc, _ = _create(_cfg(), [a, b])
+    assert rc == -1 and "overlaps" in B.adamw4_last_error()
+    # grads may alias each other (read only)
+    b = B.adamw4_tensor(P0 + (1 << 20), P0 + (1 << 30), 4096, 8, 0, 0.0)
+    os.environ["ADAMW4_FAIL_ALLOC"] = "1"
+    try:
+        rc, _ = _create(_cfg(), [a, b])
+    finally:
+        del os.environ["ADAMW4_FAIL_ALLOC"]
+    assert rc == -3 and "injected" in B.adamw4_last_error()
+
+
+def test_unknown_handles_are_rejected(L):
+    bogus = ctypes.c_void_p(0x1234)
+    assert L.adamw4_step(bogus, 1e-3, None) == -1
+    assert L.adamw4_destroy(bogus) == -1
+    assert L.adamw4_destroy(None) == -1
+    assert L.adamw4_state_bytes(bogus) == -1
+    t = ctypes.c_int64()
+    assert L.adamw4_get_step(bogus, ctypes.byref(t)) == -1
+    assert L.adamw4_set_step(bogus, 3) == -1
+    assert L.adamw4_state_import(bogus, b"x", 1) == -1
+
+
+def test_null_out_pointer(L):
+    cfg = _cfg()
+    arr = (B.adamw4_tensor * 1)(B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, 0.0))
+    assert L.adamw4_create(ctypes.byref(cfg), arr, 1, 0, None) == -1
