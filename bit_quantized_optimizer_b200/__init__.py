@@ -16,7 +16,8 @@ __all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_T_NORM", "ADAMW4_T_LM_HE
            "ADAMW4_T_FP32_STATE", "AdamW4Error", "adamw4_tensor", "adamw4_config", "lib",
            "adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
            "adamw4_get_step", "adamw4_set_step", "adamw4_state_bytes", "adamw4_state_export",
-           "adamw4_state_import", "adamw4_launch_info", "adamw4_last_error", "AdamW4",
+           "adamw4_state_import", "adamw4_launch_info", "adamw4_last_error", "adamw4_sync",
+           "adamw4_inject_fault", "ADAMW4_ETIMEOUT", "ADAMW4_FAULT_STALL_PIPELINE", "AdamW4",
            "is_fp32_state", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libadamw4.so")
@@ -30,8 +31,11 @@ ADAMW4_T_FP32_STATE = 4
 MIN_QUANT_NUMEL = 4096
 BLOCK = 128
 
+ADAMW4_ETIMEOUT = -7
+ADAMW4_FAULT_STALL_PIPELINE = 1
+
 STATUS = {0: "ADAMW4_OK", -1: "ADAMW4_EINVAL", -2: "ADAMW4_EALIGN", -3: "ADAMW4_ENOMEM",
-          -4: "ADAMW4_ECUDA", -5: "ADAMW4_ESTATE", -6: "ADAMW4_ERANGE"}
+          -4: "ADAMW4_ECUDA", -5: "ADAMW4_ESTATE", -6: "ADAMW4_ERANGE", -7: "ADAMW4_ETIMEOUT"}
 
 
 class AdamW4Error(RuntimeError):
@@ -78,11 +82,14 @@ def lib() -> ctypes.CDLL:
         L.adamw4_state_import.argtypes = [H, c.c_void_p, c.c_int64]
         L.adamw4_launch_info.argtypes = [H, c.POINTER(c.c_int), c.POINTER(c.c_int),
                                          c.POINTER(c.c_int64)]
+        L.adamw4_sync.argtypes = [H, c.c_void_p]
+        L.adamw4_inject_fault.argtypes = [H, c.c_int]
         L.adamw4_last_error.argtypes = [H]
         L.adamw4_last_error.restype = c.c_char_p
         for f in ("adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
                   "adamw4_get_step", "adamw4_set_step", "adamw4_state_export",
-                  "adamw4_state_import", "adamw4_launch_info"):
+                  "adamw4_state_import", "adamw4_launch_info", "adamw4_sync",
+                  "adamw4_inject_fault"):
             getattr(L, f).restype = c.c_int
         _lib = L
     return _lib
@@ -148,6 +155,14 @@ def adamw4_state_import(h, blob: bytes):
     _check(lib().adamw4_state_import(h, blob, len(blob)), h)
 
 
+def adamw4_sync(h, stream=None):
+    _check(lib().adamw4_sync(h, stream), h)
+
+
+def adamw4_inject_fault(h, fault: int):
+    _check(lib().adamw4_inject_fault(h, fault), h)
+
+
 def adamw4_launch_info(h):
     g, b, u = ctypes.c_int(), ctypes.c_int(), ctypes.c_int64()
     _check(lib().adamw4_launch_info(h, ctypes.byref(g), ctypes.byref(b), ctypes.byref(u)), h)
@@ -197,6 +212,13 @@ class AdamW4:
 
     def state_bytes(self) -> int:
         return adamw4_state_bytes(self.handle)
+
+    def sync(self, stream=None):
+        """Waits for the stream; raises AdamW4Error(ADAMW4_ETIMEOUT) if a step
+        kernel on it stopped on a pipeline wait."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+        adamw4_sync(self.handle, s)
 
     def state_dict_blob(self) -> bytes:
         return adamw4_state_export(self.handle)

@@ -4,11 +4,20 @@
 // One kernel launch per step covers every parameter tensor.  The work is a flat
 // list of 128-value units: each block of a 4-bit tensor is one unit, and each
 // fp32-state tensor is cut into 128-element chunks.  A half-warp owns one unit
-// (16 lanes x 8 contiguous values), so a lane moves two 16-byte fp32 weight
-// vectors, one 16-byte bf16 gradient vector and one 32-bit word of codes per
-// moment.  The grid is persistent (SM count x resident CTAs) and half-warps
-// stride through the unit list, which keeps all SMs streaming one contiguous
-// window of HBM.
+// at a time (16 lanes x 8 contiguous values).  The grid is persistent (SM count
+// x resident CTAs) and half-warps stride through the unit list, so all SMs
+// stream one contiguous window of HBM.
+//
+// Memory pipeline: every half-warp keeps kStages units in flight in its own
+// shared-memory ring.  Lane 0 fills a stage with TMA bulk copies
+// (cp.async.bulk: 512 B of fp32 weights, 256 B of bf16 grads, 64 + 64 B of
+// codes) plus two 4-byte cp.async copies of the block scales, all completing on
+// the stage's mbarrier.  The half-warp waits on the barrier (bounded by a
+// timer; on expiry the kernel records an error in a status word and leaves),
+// computes from shared memory, stores the results straight to global memory,
+// and refills the stage with the unit kStages ahead.  Units that are not whole
+// 4-bit blocks (a ragged last block, fp32-state chunks) take a direct path with
+// plain guarded loads.
 //
 // Per unit, following the method flowchart of "ZIP-SR / ZE-EDEN: 4-bit AdamW
 // state quantization" (daiwk.github.io, Method): decode the prior moments,
@@ -18,11 +27,13 @@
 //
 // Arithmetic follows one fixed binary32 evaluation order with IEEE division
 // and square root (__fdiv_rn, __fsqrt_rn) and fused multiply-add only where
-// __fmaf_rn is written; the file is built with -fmad=false so nothing else is
-// contracted.  With that, codes, scales and weights are reproducible bit for bit
-// by any IEEE implementation of the same order.
+// written (__fmaf_rn, or __ffma2_rn on value pairs, which rounds each lane like
+// __fmaf_rn); the file is built with -fmad=false so nothing else is contracted.
+// With that, codes, scales and weights are reproducible bit for bit by any
+// IEEE implementation of the same order.
 //
-// No tensor cores: the step is a streaming codec, bound by HBM bandwidth.
+// No tensor cores: the step is a streaming codec, bound by HBM bandwidth.  No
+// TMA multicast: every copy is this GPU's global memory into its own CTA.
 
 #include <cuda_runtime.h>
 
@@ -47,11 +58,21 @@ constexpr int kBlock = ADAMW4_BLOCK;        // values per quantisation block
 constexpr int kLanesPerUnit = 16;           // a half-warp per block
 constexpr int kPerLane = kBlock / kLanesPerUnit;  // 8 values per lane
 constexpr int kThreads = 256;               // threads per CTA
+constexpr int kHalves = kThreads / kLanesPerUnit; // half-warps per CTA
+constexpr int kStages = 4;                  // units in flight per half-warp
+// Stage layout: w 512 B | g 256 B | m codes 64 B | v codes 64 B | m scale | v scale
+constexpr int kOffW = 0, kOffG = 512, kOffMC = 768, kOffVC = 832, kOffMS = 896, kOffVS = 900;
+constexpr int kStageBytes = 912;            // 16-byte multiple
+constexpr uint32_t kStageTx = 896;          // bytes delivered by the bulk copies
+constexpr int kSmemStages = kHalves * kStages * kStageBytes;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per stage wait
+constexpr uint64_t kDrainLimitNs = 10000000ull;    // 10 ms per stage when draining
 constexpr int kVZip = ADAMW4_V_ZIPSR;
 constexpr int kVZe = ADAMW4_V_ZEEDEN;
 constexpr uint32_t kKindFp32 = 1u << 16;    // internal flag: fp32-state tensor
 constexpr uint32_t kStreamV = 0u;           // Philox stream of the v draw
 constexpr uint32_t kStreamM = 1u;           // Philox stream of the LM-head m draw
+constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23: adding it rounds to an integer
 
 // Philox4x32-10 round multipliers and key increments (Salmon et al., SC'11).
 constexpr uint32_t kPhiloxM0 = 0xD2511F53u;
@@ -82,6 +103,8 @@ struct StepArgs {
   uint32_t key0, key1;   // Philox key = seed
   uint32_t t_lo;         // step, low word (Philox counter word 2)
   int lm_sr_active;      // final-10% LM-head phase
+  uint32_t* status;      // device status word (bit 0: a pipeline wait timed out)
+  int fault_stall;       // test hook: mark stages pending without filling them
 };
 
 // Code tables, passed by value and staged in shared memory by each CTA.
@@ -90,7 +113,7 @@ struct CodeTables {
   float nf4_gap[16];    // nf4[j+1] - nf4[j]
   float vz[16];         // ZIP-SR code points k/15
   float vz_sqrt[16];    // sqrt(k/15)
-  float2 rtn[65];       // NF4 nearest-level buckets: .x threshold, .y base code (int bits)
+  float2 rtn[128];      // NF4 nearest-level buckets: .x threshold, .y base code (int bits)
 };
 
 struct StateArena {
@@ -103,7 +126,71 @@ struct StateArena {
 };
 
 // ---------------------------------------------------------------------------
-// Device helpers
+// PTX wrappers: mbarrier, bulk copies, timer
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for a barrier phase; false if `limit_ns` passed first.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Arithmetic helpers
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
@@ -113,9 +200,10 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
       k0 += kPhiloxW0;
       k1 += kPhiloxW1;
     }
-    const uint32_t hi0 = __umulhi(kPhiloxM0, c.x), lo0 = kPhiloxM0 * c.x;
-    const uint32_t hi1 = __umulhi(kPhiloxM1, c.z), lo1 = kPhiloxM1 * c.z;
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    const uint64_t p0 = (uint64_t)kPhiloxM0 * c.x;
+    const uint64_t p1 = (uint64_t)kPhiloxM1 * c.z;
+    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1,
+                   (uint32_t)p0);
   }
   return c;
 }
@@ -125,7 +213,7 @@ __device__ __forceinline__ float uniform23(uint32_t w) {
   return __fsub_rn(__uint_as_float((w >> 9) | 0x3F800000u), 1.0f);
 }
 
-// The eight draws of one lane: elements q*4 .. q*4+7 (q = first quad).
+// The eight draws of one lane: elements 4*quad .. 4*quad + 7.
 __device__ __forceinline__ void draws8(const StepArgs& a, uint32_t tensor_id, uint32_t stream,
                                        uint64_t quad, float u[8]) {
   const uint32_t c3 = tensor_id * 2u + stream;
@@ -140,27 +228,30 @@ __device__ __forceinline__ void draws8(const StepArgs& a, uint32_t tensor_id, ui
 
 __device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
-__device__ __forceinline__ float hmax16(float v, unsigned mask) {
+// Max of non-negative binary32 values over a half-warp: their bit patterns
+// order like the values, so an integer reduction gives the exact maximum.
+__device__ __forceinline__ float hmax16_nonneg(float v, unsigned mask) {
+  return __uint_as_float(__reduce_max_sync(mask, __float_as_uint(v)));
+}
+
+// Balanced pairwise sum of (x, y) pairs over the half-warp: partner offsets 1,
+// 2, 4, 8 join adjacent 8-value groups in index order (IEEE addition is
+// commutative, so both partners hold the same bits).
+__device__ __forceinline__ float2 hsum16_tree2(float2 v, unsigned mask) {
 #pragma unroll
-  for (int off = 8; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(mask, v, off));
+  for (int off = 1; off < 16; off <<= 1) {
+    const float2 o = make_float2(__shfl_xor_sync(mask, v.x, off), __shfl_xor_sync(mask, v.y, off));
+    v = __fadd2_rn(v, o);
+  }
   return v;
 }
 
-// Balanced pairwise sum over the half-warp: partner offsets 1, 2, 4, 8 join
-// adjacent 8-value groups in index order (IEEE addition is commutative, so
-// both partners hold the same bits).
-__device__ __forceinline__ float hsum16_tree(float v, unsigned mask) {
-#pragma unroll
-  for (int off = 1; off < 16; off <<= 1) v = __fadd_rn(v, __shfl_xor_sync(mask, v, off));
-  return v;
-}
-
-// NF4 nearest level: #{j : x > mid[j]} through 65 uniform buckets of x.
-__device__ __forceinline__ uint32_t nf4_rtn(float x, const float2* rtn) {
-  int b = __float_as_int(__fmaf_rn(x, 32.0f, 12582944.0f)) - 0x4B400000;
-  b = min(max(b, 0), 64);
-  const float2 e = rtn[b];
+// NF4 nearest level: #{j : x > mid[j]}.  Bucket round(32 x + 32) holds at most
+// one threshold; the table has 128 entries so any 7-bit index stays inside.
+__device__ __forceinline__ uint32_t nf4_rtn_bucket(float x, float bucket_sum, const float2* rtn) {
+  const float2 e = rtn[__float_as_uint(bucket_sum) & 127u];
   return (uint32_t)(__float_as_int(e.y) + (x > e.x ? 1 : 0));
 }
 
@@ -173,247 +264,376 @@ __device__ __forceinline__ uint32_t nf4_sr(float x, float u, const float* nf4, c
   return lower ? (uint32_t)j : (uint32_t)(j + 1);
 }
 
+// Shared tables of one CTA.
+struct SmemTables {
+  float nf4[16];
+  float gap[16];
+  float vq[16];        // decoded v code points: k/15 (ZIP-SR) or (k+1)/16 (ZE-EDEN)
+  float vz[16];        // ZIP-SR code points k/15
+  float2 sqp[16];      // {sqrt(k/15), sqrt((k+1)/15)}
+  float2 vzp[16];      // {k/15, (k+1)/15}
+  float2 rtn[128];
+};
+
+// Per-tensor values a half-warp keeps while it walks the unit list.
+struct Cursor {
+  int ti;
+  int64_t begin, end, numel, soff;
+  float* param;
+  const uint16_t* grad;
+  uint32_t id, flags;
+  float wd;
+};
+
+__device__ __forceinline__ void cursor_seek(Cursor& c, const DevTensor* __restrict__ T,
+                                            int64_t u) {
+  if (u < c.end) return;
+  do {
+    ++c.ti;
+    c.end = __ldg(&T[c.ti].unit_end);
+  } while (u >= c.end);
+  const DevTensor* d = &T[c.ti];
+  c.begin = __ldg(&d->unit_begin);
+  c.numel = __ldg(&d->numel);
+  c.soff = __ldg(&d->state_off);
+  c.param = d->param;
+  c.grad = d->grad;
+  c.id = __ldg(&d->tensor_id);
+  c.flags = __ldg(&d->flags);
+  c.wd = __ldg(&d->weight_decay);
+}
+
+// ---------------------------------------------------------------------------
+// Requantisation of one 4-bit block held by a half-warp (8 values per lane).
+// FULL: all 128 values valid.  Otherwise `myn` values of this lane are valid.
+// ---------------------------------------------------------------------------
+template <int VCODE, bool FULL>
+__device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTables& S,
+                                              const Cursor& c, int64_t e0, int lane, int myn,
+                                              unsigned hmask, const float (&m1)[kPerLane],
+                                              const float (&v1)[kPerLane],
+                                              const float (&den)[kPerLane], uint32_t* mcw,
+                                              uint32_t* vcw, float* msp, float* vsp) {
+  float am = 0.0f, av = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    if (FULL || i < myn) {
+      am = fmaxf(am, fabsf(m1[i]));
+      av = fmaxf(av, fabsf(v1[i]));
+    }
+  }
+  am = hmax16_nonneg(am, hmask);
+  av = hmax16_nonneg(av, hmask);
+
+  // ---- first moment: absmax scale, NF4 codes ----
+  uint32_t mco = 0;
+  float mso = 0.0f;
+  if (am >= FLT_MIN) {
+    const float inv = __fdiv_rn(1.0f, am);
+    if ((c.flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
+      float ud[kPerLane];
+      draws8(a, c.id, kStreamM, (uint64_t)(e0 + lane * kPerLane) >> 2, ud);
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i)
+        if (FULL || i < myn) mco |= nf4_sr(__fmul_rn(m1[i], inv), ud[i], S.nf4, S.gap) << (4 * i);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPerLane / 2; ++j) {
+        const float2 x = __fmul2_rn(make_float2(m1[2 * j], m1[2 * j + 1]), f2(inv));
+        const float2 b = __ffma2_rn(x, f2(32.0f), f2(kMagic + 32.0f));
+        const uint32_t c0 = nf4_rtn_bucket(x.x, b.x, S.rtn);
+        const uint32_t c1 = nf4_rtn_bucket(x.y, b.y, S.rtn);
+        if (FULL || 2 * j < myn) mco |= c0 << (8 * j);
+        if (FULL || 2 * j + 1 < myn) mco |= c1 << (8 * j + 4);
+      }
+    }
+    mso = am;
+  }
+
+  // ---- second moment ----
+  uint32_t vco = 0;
+  float vso = 0.0f;
+  if (av >= FLT_MIN) {
+    const float inv = __fdiv_rn(1.0f, av);
+    if (VCODE == kVZip) {
+      // ZIP-SR ("ZIP-SR / ZE-EDEN", Core equation): keep the lower code point
+      // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
+      // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
+      const float R = __fmul_rn(__fsqrt_rn(av), a.rs_bc2);
+      float ud[kPerLane];
+      draws8(a, c.id, kStreamV, (uint64_t)(e0 + lane * kPerLane) >> 2, ud);
+#pragma unroll
+      for (int j = 0; j < kPerLane / 2; ++j) {
+        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+        const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = 2 * j + h;
+          const float x = h ? x2.y : x2.x;
+          // nearest of 15x is the bracket or one above it; step down if needed
+          int k = (int)(__float_as_uint(h ? t2.y : t2.x) & 31u);
+          k -= (x < S.vz[k]) ? 1 : 0;
+          k = min(k, 14);
+          const float2 sq = S.sqp[k];
+          const float2 dd = __ffma2_rn(sq, f2(R), f2(a.eps));        // (da, db)
+          const float2 ad = __fadd2_rn(f2(dd.y), make_float2(-dd.x, -den[i]));  // (db-da, db-dv)
+          const float2 pr = __fmul2_rn(ad, make_float2(den[i], dd.x));          // (..*dv, ..*da)
+          bool lower = __fmul_rn(ud[i], pr.x) < pr.y;
+          if (dd.x == dd.y) {
+            const float2 z = S.vzp[k];
+            lower = __fmul_rn(ud[i], __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
+          }
+          if (FULL || i < myn) vco |= (uint32_t)(k + (lower ? 0 : 1)) << (4 * i);
+        }
+      }
+      vso = av;
+    } else {
+      // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
+      // code point, scale times ||x||^2 / max(<x,Q(x)>, 1e-12 s^2) on x = v/s.
+      float2 l1[kPerLane / 2];
+#pragma unroll
+      for (int j = 0; j < kPerLane / 2; ++j) {
+        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+        const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
+        const float2 c2 = __fadd2_rn(t2, f2(-kMagic));             // rint(16x), exact
+        const float2 q2 = __fmul2_rn(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)),
+                                     f2(0.0625f));                 // (k+1)/16
+        const uint32_t k0 = max(__float_as_uint(t2.x) & 31u, 1u) - 1u;
+        const uint32_t k1 = max(__float_as_uint(t2.y) & 31u, 1u) - 1u;
+        float2 xx = __fmul2_rn(x2, x2);
+        float2 xq = __fmul2_rn(x2, q2);
+        if (!FULL) {
+          if (2 * j >= myn) { xx.x = 0.0f; xq.x = 0.0f; }
+          if (2 * j + 1 >= myn) { xx.y = 0.0f; xq.y = 0.0f; }
+        }
+        if (FULL || 2 * j < myn) vco |= k0 << (8 * j);
+        if (FULL || 2 * j + 1 < myn) vco |= k1 << (8 * j + 4);
+        // first tree level: (x0^2 + x1^2, x0 q0 + x1 q1)
+        l1[j] = __fadd2_rn(make_float2(xx.x, xq.x), make_float2(xx.y, xq.y));
+      }
+      const float2 l2a = __fadd2_rn(l1[0], l1[1]);
+      const float2 l2b = __fadd2_rn(l1[2], l1[3]);
+      const float2 s = hsum16_tree2(__fadd2_rn(l2a, l2b), hmask);    // (sum x^2, sum x q)
+      vso = __fmul_rn(av, __fdiv_rn(s.x, fmaxf(s.y, 1e-12f)));
+    }
+  }
+
+  *mcw = mco;
+  *vcw = vco;
+  if (lane == 0) {
+    *msp = mso;
+    *vsp = vso;
+  }
+}
+
+// Decode + moment update + weight update for 8 values of a 4-bit block.
+template <bool FULL>
+__device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, float decay,
+                                        float (&w)[kPerLane], const float (&g)[kPerLane],
+                                        uint32_t mc, uint32_t vc, float sm, float sv,
+                                        float (&m1)[kPerLane], float (&v1)[kPerLane],
+                                        float (&den)[kPerLane]) {
+#pragma unroll
+  for (int j = 0; j < kPerLane / 2; ++j) {
+    const float2 m0 = __fmul2_rn(
+        make_float2(S.nf4[(mc >> (8 * j)) & 15u], S.nf4[(mc >> (8 * j + 4)) & 15u]), f2(sm));
+    const float2 v0 = __fmul2_rn(
+        make_float2(S.vq[(vc >> (8 * j)) & 15u], S.vq[(vc >> (8 * j + 4)) & 15u]), f2(sv));
+    const float2 gg = make_float2(g[2 * j], g[2 * j + 1]);
+    const float2 mm = __ffma2_rn(f2(a.b1), m0, __fmul2_rn(f2(a.omb1), gg));
+    const float2 vv = __ffma2_rn(f2(a.b2), v0, __fmul2_rn(f2(a.omb2), __fmul2_rn(gg, gg)));
+    const float2 dd = __ffma2_rn(make_float2(__fsqrt_rn(vv.x), __fsqrt_rn(vv.y)), f2(a.rs_bc2),
+                                 f2(a.eps));
+    const float2 qq = make_float2(__fdiv_rn(mm.x, dd.x), __fdiv_rn(mm.y, dd.y));
+    const float2 ww = __ffma2_rn(f2(-a.step_size), qq,
+                                 __fmul2_rn(make_float2(w[2 * j], w[2 * j + 1]), f2(decay)));
+    w[2 * j] = ww.x; w[2 * j + 1] = ww.y;
+    m1[2 * j] = mm.x; m1[2 * j + 1] = mm.y;
+    v1[2 * j] = vv.x; v1[2 * j + 1] = vv.y;
+    den[2 * j] = dd.x; den[2 * j + 1] = dd.y;
+  }
+}
+
+// A unit read straight from global memory: a ragged last 4-bit block or a
+// chunk of an fp32-state tensor.
+template <int VCODE>
+__device__ __noinline__ void process_direct(const StepArgs& a, const SmemTables& S,
+                                            const StateArena& st, const Cursor& c, float decay,
+                                            int64_t u, int lane, unsigned hmask) {
+  const int64_t ub = u - c.begin;
+  const int64_t e0 = ub * kBlock;
+  const int nvalid = (int)min((int64_t)kBlock, c.numel - e0);
+  const int my0 = lane * kPerLane;
+  const int myn = min(max(nvalid - my0, 0), kPerLane);
+  float* wp = c.param + e0 + my0;
+  const uint16_t* gp = c.grad + e0 + my0;
+  float w[kPerLane], g[kPerLane];
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    w[i] = (i < myn) ? wp[i] : 0.0f;
+    g[i] = (i < myn) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
+  }
+  if (c.flags & kKindFp32) {
+    float* mp = st.fm + c.soff + e0 + my0;
+    float* vp = st.fv + c.soff + e0 + my0;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      if (i < myn) {
+        const float m1 = __fmaf_rn(a.b1, mp[i], __fmul_rn(a.omb1, g[i]));
+        const float v1 = __fmaf_rn(a.b2, vp[i], __fmul_rn(a.omb2, __fmul_rn(g[i], g[i])));
+        const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
+        wp[i] = __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay));
+        mp[i] = m1;
+        vp[i] = v1;
+      }
+    }
+    return;
+  }
+  const int64_t blk = c.soff + ub;
+  uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
+  uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
+  float m1[kPerLane], v1[kPerLane], den[kPerLane];
+  update8<false>(a, S, decay, w, g, *mcw, *vcw, st.mscale[blk], st.vscale[blk], m1, v1, den);
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i)
+    if (i < myn) wp[i] = w[i];
+  requant_store<VCODE, false>(a, S, c, e0, lane, myn, hmask, m1, v1, den, mcw, vcw,
+                              st.mscale + blk, st.vscale + blk);
+}
+
 // ---------------------------------------------------------------------------
 // The step kernel
 // ---------------------------------------------------------------------------
 
 template <int VCODE>
-__global__ void __launch_bounds__(kThreads)
-adamw4_step_kernel(const DevTensor* __restrict__ tensors, int64_t nunits, StepArgs a,
-                   CodeTables tabs, StateArena st) {
-  __shared__ float s_nf4[16], s_gap[16], s_vz[16], s_vzs[16];
-  __shared__ float2 s_rtn[65];
+__global__ void __launch_bounds__(kThreads, 2)
+adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, CodeTables tabs,
+                   StateArena st) {
+  extern __shared__ __align__(128) uint8_t s_stage[];
+  __shared__ __align__(8) uint64_t s_bar[kHalves * kStages];
+  __shared__ SmemTables S;
+
   if (threadIdx.x < 16) {
-    s_nf4[threadIdx.x] = tabs.nf4[threadIdx.x];
-    s_gap[threadIdx.x] = tabs.nf4_gap[threadIdx.x];
-    s_vz[threadIdx.x] = tabs.vz[threadIdx.x];
-    s_vzs[threadIdx.x] = tabs.vz_sqrt[threadIdx.x];
+    const int k = threadIdx.x;
+    S.nf4[k] = tabs.nf4[k];
+    S.gap[k] = tabs.nf4_gap[k];
+    S.vz[k] = tabs.vz[k];
+    S.vq[k] = (VCODE == kVZip) ? tabs.vz[k] : __fmul_rn((float)(k + 1), 0.0625f);
+    S.sqp[k] = make_float2(tabs.vz_sqrt[k], tabs.vz_sqrt[min(k + 1, 15)]);
+    S.vzp[k] = make_float2(tabs.vz[k], tabs.vz[min(k + 1, 15)]);
   }
-  if (threadIdx.x < 65) s_rtn[threadIdx.x] = tabs.rtn[threadIdx.x];
-  __syncthreads();
+  if (threadIdx.x < 128) S.rtn[threadIdx.x] = tabs.rtn[threadIdx.x];
 
   const int lane = threadIdx.x & 15;
+  const int half = threadIdx.x >> 4;
   const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
-  const int64_t H = (int64_t)gridDim.x * (kThreads / kLanesPerUnit);
-  int64_t u = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kLanesPerUnit;
+  const uint32_t stage0 = smem_addr(s_stage) + (uint32_t)(half * kStages * kStageBytes);
+  const uint32_t bar0 = smem_addr(&s_bar[half * kStages]);
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8u * s, 2);
+    fence_mbar_init();
+  }
+  __syncthreads();
 
-  // Cached descriptor of the current tensor; half-warps move forward only.
-  int ti = -1;
-  int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0;
-  float* t_param = nullptr;
-  const uint16_t* t_grad = nullptr;
-  uint32_t t_id = 0, t_flags = 0;
+  const int64_t H = (int64_t)gridDim.x * kHalves;
+  const int64_t hw = (int64_t)blockIdx.x * kHalves + half;
+
+  // Issue side: fills stage s with unit ui if it is a whole 4-bit block.
+  Cursor ic{-1, 0, 0, 0, 0, nullptr, nullptr, 0, 0, 0.0f};
+  auto issue = [&](int64_t ui, int s) -> bool {
+    if (ui >= nunits) return false;
+    cursor_seek(ic, T, ui);
+    if (ic.flags & kKindFp32) return false;
+    const int64_t ub = ui - ic.begin;
+    const int64_t e0 = ub * kBlock;
+    if (ic.numel - e0 < kBlock) return false;
+    if (lane == 0) {
+      const uint32_t dst = stage0 + (uint32_t)(s * kStageBytes);
+      const uint32_t bar = bar0 + 8u * s;
+      if (a.fault_stall) return true;      // test hook: nothing will arrive
+      const int64_t blk = ic.soff + ub;
+      mbar_arrive_expect_tx(bar, kStageTx);
+      bulk_g2s(dst + kOffW, ic.param + e0, 512, bar);
+      bulk_g2s(dst + kOffG, ic.grad + e0, 256, bar);
+      bulk_g2s(dst + kOffMC, st.mcodes + blk * (kBlock / 2), 64, bar);
+      bulk_g2s(dst + kOffVC, st.vcodes + blk * (kBlock / 2), 64, bar);
+      cp_async4(dst + kOffMS, st.mscale + blk);
+      cp_async4(dst + kOffVS, st.vscale + blk);
+      cp_async_arrive_noinc(bar);
+    }
+    return true;
+  };
+
+  uint32_t pend = 0, phase = 0;
+  int64_t ui = hw;
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) {
+    if (issue(ui, s)) pend |= 1u << s;
+    ui += H;
+  }
+
+  Cursor cc{-1, 0, 0, 0, 0, nullptr, nullptr, 0, 0, 0.0f};
   float decay = 1.0f;
-
-  for (; u < nunits; u += H) {
-    if (u >= t_end) {
-      do {
-        ++ti;
-        t_end = __ldg(&tensors[ti].unit_end);
-      } while (u >= t_end);
-      const DevTensor* d = &tensors[ti];
-      t_begin = __ldg(&d->unit_begin);
-      t_numel = __ldg(&d->numel);
-      t_soff = __ldg(&d->state_off);
-      t_param = d->param;
-      t_grad = d->grad;
-      t_id = __ldg(&d->tensor_id);
-      t_flags = __ldg(&d->flags);
-      decay = (float)(1.0 - (double)a.lr * (double)__ldg(&d->weight_decay));
+  int s = 0;
+  for (int64_t u = hw; u < nunits; u += H) {
+    if (u >= cc.end) {
+      cursor_seek(cc, T, u);
+      decay = (float)(1.0 - (double)a.lr * (double)cc.wd);
     }
-    const int64_t ub = u - t_begin;               // unit within the tensor
-    const int64_t e0 = ub * kBlock;               // its first element
-    const int nvalid = (int)min((int64_t)kBlock, t_numel - e0);
-    const int my0 = lane * kPerLane;
-    const int myn = min(max(nvalid - my0, 0), kPerLane);
-    float* wp = t_param + e0 + my0;
-    const uint16_t* gp = t_grad + e0 + my0;
+    if ((pend >> s) & 1u) {
+      const uint32_t bar = bar0 + 8u * s;
+      const bool ok = __all_sync(hmask, wait_phase(bar, (phase >> s) & 1u, kWaitLimitNs));
+      if (!ok) {
+        // Leave cleanly: record the failure, let copies still in flight land.
+        if (lane == 0) atomicOr(a.status, 1u);
+        pend &= ~(1u << s);
+        for (int s2 = 0; s2 < kStages; ++s2)
+          if ((pend >> s2) & 1u) wait_phase(bar0 + 8u * s2, (phase >> s2) & 1u, kDrainLimitNs);
+        __syncwarp(hmask);
+        return;
+      }
+      phase ^= 1u << s;
+      const uint8_t* sp = s_stage + (half * kStages + s) * kStageBytes;
+      const int64_t ub = u - cc.begin;
+      const int64_t e0 = ub * kBlock;
+      const int64_t blk = cc.soff + ub;
+      float w[kPerLane], g[kPerLane];
+      {
+        const float4 wa = *reinterpret_cast<const float4*>(sp + kOffW + lane * 32);
+        const float4 wb = *reinterpret_cast<const float4*>(sp + kOffW + lane * 32 + 16);
+        const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + lane * 16);
+        w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
+        w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
+        g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
+        g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
+      }
+      const uint32_t mc = *reinterpret_cast<const uint32_t*>(sp + kOffMC + lane * 4);
+      const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + lane * 4);
+      const float sm = *reinterpret_cast<const float*>(sp + kOffMS);
+      const float sv = *reinterpret_cast<const float*>(sp + kOffVS);
+      // every read of the stage is done: hand it back to the async proxy
+      fence_proxy_async_smem();
+      __syncwarp(hmask);
+      pend &= ~(1u << s);
+      if (issue(ui, s)) pend |= 1u << s;
+      ui += H;
 
-    // ---- load weights and gradients ----
-    float w[kPerLane];
-    float g[kPerLane];
-    if (myn == kPerLane) {
-      const float4 wa = *reinterpret_cast<const float4*>(wp);
-      const float4 wb = *reinterpret_cast<const float4*>(wp + 4);
-      const uint4 gg = *reinterpret_cast<const uint4*>(gp);
-      w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
-      w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
-      g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
-      g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
-    } else {
-#pragma unroll
-      for (int i = 0; i < kPerLane; ++i) {
-        w[i] = (i < myn) ? wp[i] : 0.0f;
-        g[i] = (i < myn) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
-      }
-    }
-
-    if (t_flags & kKindFp32) {
-      // ---- fp32-state AdamW chunk ----
-      float* mp = st.fm + t_soff + e0 + my0;
-      float* vp = st.fv + t_soff + e0 + my0;
-      float m[kPerLane], v[kPerLane];
-      if (myn == kPerLane) {
-        const float4 ma = *reinterpret_cast<const float4*>(mp);
-        const float4 mb = *reinterpret_cast<const float4*>(mp + 4);
-        const float4 va = *reinterpret_cast<const float4*>(vp);
-        const float4 vb = *reinterpret_cast<const float4*>(vp + 4);
-        m[0] = ma.x; m[1] = ma.y; m[2] = ma.z; m[3] = ma.w;
-        m[4] = mb.x; m[5] = mb.y; m[6] = mb.z; m[7] = mb.w;
-        v[0] = va.x; v[1] = va.y; v[2] = va.z; v[3] = va.w;
-        v[4] = vb.x; v[5] = vb.y; v[6] = vb.z; v[7] = vb.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-          m[i] = (i < myn) ? mp[i] : 0.0f;
-          v[i] = (i < myn) ? vp[i] : 0.0f;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < kPerLane; ++i) {
-        const float m1 = __fmaf_rn(a.b1, m[i], __fmul_rn(a.omb1, g[i]));
-        const float v1 = __fmaf_rn(a.b2, v[i], __fmul_rn(a.omb2, __fmul_rn(g[i], g[i])));
-        const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
-        w[i] = __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay));
-        m[i] = m1;
-        v[i] = v1;
-      }
-      if (myn == kPerLane) {
-        *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
-        *reinterpret_cast<float4*>(mp) = make_float4(m[0], m[1], m[2], m[3]);
-        *reinterpret_cast<float4*>(mp + 4) = make_float4(m[4], m[5], m[6], m[7]);
-        *reinterpret_cast<float4*>(vp) = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4*>(vp + 4) = make_float4(v[4], v[5], v[6], v[7]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i)
-          if (i < myn) { wp[i] = w[i]; mp[i] = m[i]; vp[i] = v[i]; }
-      }
-      continue;
-    }
-
-    // ---- 4-bit block: load codes and scales ----
-    const int64_t blk = t_soff + ub;
-    uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
-    uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
-    const uint32_t mc = *mcw;
-    const uint32_t vc = *vcw;
-    const float sm = st.mscale[blk];
-    const float sv = st.vscale[blk];
-
-    // ---- decode, moment update, weight update ----
-    float m1[kPerLane], v1[kPerLane], den[kPerLane];
-    float am = 0.0f, av = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i) {
-      const float m0 = __fmul_rn(s_nf4[(mc >> (4 * i)) & 15u], sm);
-      const uint32_t cv = (vc >> (4 * i)) & 15u;
-      const float q0 = (VCODE == kVZip) ? s_vz[cv] : __fmul_rn((float)(cv + 1), 0.0625f);
-      const float v0 = __fmul_rn(q0, sv);
-      m1[i] = __fmaf_rn(a.b1, m0, __fmul_rn(a.omb1, g[i]));
-      v1[i] = __fmaf_rn(a.b2, v0, __fmul_rn(a.omb2, __fmul_rn(g[i], g[i])));
-      den[i] = __fmaf_rn(__fsqrt_rn(v1[i]), a.rs_bc2, a.eps);
-      w[i] = __fmaf_rn(-a.step_size, __fdiv_rn(m1[i], den[i]), __fmul_rn(w[i], decay));
-      if (i < myn) {
-        am = fmaxf(am, fabsf(m1[i]));
-        av = fmaxf(av, v1[i]);
-      }
-    }
-    if (myn == kPerLane) {
+      float m1[kPerLane], v1[kPerLane], den[kPerLane];
+      update8<true>(a, S, decay, w, g, mc, vc, sm, sv, m1, v1, den);
+      float* wp = cc.param + e0 + lane * kPerLane;
       *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
       *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
+      uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
+      uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
+      requant_store<VCODE, true>(a, S, cc, e0, lane, kPerLane, hmask, m1, v1, den, mcw, vcw,
+                                 st.mscale + blk, st.vscale + blk);
     } else {
-#pragma unroll
-      for (int i = 0; i < kPerLane; ++i)
-        if (i < myn) wp[i] = w[i];
+      process_direct<VCODE>(a, S, st, cc, decay, u, lane, hmask);
+      if (issue(ui, s)) pend |= 1u << s;
+      ui += H;
     }
-    am = hmax16(am, hmask);
-    av = hmax16(av, hmask);
-
-    // ---- first moment: absmax scale, NF4 codes ----
-    uint32_t mco = 0;
-    float mso = 0.0f;
-    if (am >= FLT_MIN) {
-      const float inv = __fdiv_rn(1.0f, am);
-      if ((t_flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
-        float ud[kPerLane];
-        draws8(a, t_id, kStreamM, (uint64_t)(e0 + my0) >> 2, ud);
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i)
-          if (i < myn) mco |= nf4_sr(__fmul_rn(m1[i], inv), ud[i], s_nf4, s_gap) << (4 * i);
-      } else {
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i)
-          if (i < myn) mco |= nf4_rtn(__fmul_rn(m1[i], inv), s_rtn) << (4 * i);
-      }
-      mso = am;
-    }
-
-    // ---- second moment ----
-    uint32_t vco = 0;
-    float vso = 0.0f;
-    if (av >= FLT_MIN) {
-      const float inv = __fdiv_rn(1.0f, av);
-      if (VCODE == kVZip) {
-        // ZIP-SR ("ZIP-SR / ZE-EDEN", Core equation): keep the lower code point
-        // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
-        // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
-        const float R = __fmul_rn(__fsqrt_rn(av), a.rs_bc2);
-        float ud[kPerLane];
-        draws8(a, t_id, kStreamV, (uint64_t)(e0 + my0) >> 2, ud);
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-          if (i < myn) {
-            const float x = __fmul_rn(v1[i], inv);
-            int k = min(__float2int_rz(__fmul_rn(x, 15.0f)), 14);
-            if (x < s_vz[k]) --k;
-            else if (k < 14 && x >= s_vz[k + 1]) ++k;
-            const float da = __fmaf_rn(s_vzs[k], R, a.eps);
-            const float db = __fmaf_rn(s_vzs[k + 1], R, a.eps);
-            bool lower;
-            if (da == db) {
-              lower = __fmul_rn(ud[i], __fsub_rn(s_vz[k + 1], s_vz[k])) < __fsub_rn(s_vz[k + 1], x);
-            } else {
-              lower = __fmul_rn(ud[i], __fmul_rn(__fsub_rn(db, da), den[i])) <
-                      __fmul_rn(__fsub_rn(db, den[i]), da);
-            }
-            vco |= (uint32_t)(lower ? k : k + 1) << (4 * i);
-          }
-        }
-        vso = av;
-      } else {
-        // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
-        // code point, scale times ||x||^2 / max(<x,Q(x)>, 1e-12 s^2) on x = v/s.
-        float xx[kPerLane], xq[kPerLane];
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-          const float x = __fmul_rn(v1[i], inv);
-          int k = __float2int_rz(rintf(__fmul_rn(x, 16.0f))) - 1;
-          k = min(max(k, 0), 15);
-          const float q = __fmul_rn((float)(k + 1), 0.0625f);
-          const bool ok = i < myn;
-          xx[i] = ok ? __fmul_rn(x, x) : 0.0f;
-          xq[i] = ok ? __fmul_rn(x, q) : 0.0f;
-          if (ok) vco |= (uint32_t)k << (4 * i);
-        }
-        float sxx = __fadd_rn(__fadd_rn(__fadd_rn(xx[0], xx[1]), __fadd_rn(xx[2], xx[3])),
-                              __fadd_rn(__fadd_rn(xx[4], xx[5]), __fadd_rn(xx[6], xx[7])));
-        float sxq = __fadd_rn(__fadd_rn(__fadd_rn(xq[0], xq[1]), __fadd_rn(xq[2], xq[3])),
-                              __fadd_rn(__fadd_rn(xq[4], xq[5]), __fadd_rn(xq[6], xq[7])));
-        sxx = hsum16_tree(sxx, hmask);
-        sxq = hsum16_tree(sxq, hmask);
-        vso = __fmul_rn(av, __fdiv_rn(sxx, fmaxf(sxq, 1e-12f)));
-      }
-    }
-
-    // ---- pack and store ----
-    *mcw = mco;
-    *vcw = vco;
-    if (lane == 0) {
-      st.mscale[blk] = mso;
-      st.vscale[blk] = vso;
-    }
+    s = (s + 1 == kStages) ? 0 : s + 1;
   }
 }
 
@@ -443,6 +663,8 @@ struct adamw4_handle {
   int64_t nfp32 = 0;          // fp32 arena elements (with alignment)
   int64_t nunits = 0;
   int grid = 0;
+  uint32_t* d_status = nullptr;   // device status word (in the arena)
+  int fault_stall = 0;            // test hook for the next step
   CodeTables tabs{};
   std::string err;
 };
@@ -497,9 +719,9 @@ void build_tables(CodeTables* T) {
   float mid[15];
   for (int j = 0; j < 15; ++j)
     mid[j] = (float)(((double)kNF4Levels[j] + (double)kNF4Levels[j + 1]) * 0.5);
-  // Bucket b of x is round(32 x + 32) clamped to [0, 64] (monotone in x).  A
-  // bucket holds at most one midpoint, so the nearest level is the count of
-  // midpoints in lower buckets plus one comparison.
+  // Bucket b of x is round(32 x + 32), in [0, 64] for |x| <= 1 + 2^-23 and
+  // monotone in x.  A bucket holds at most one midpoint, so the nearest level
+  // is the count of midpoints in lower buckets plus one comparison.
   int bucket_of[15];
   for (int j = 0; j < 15; ++j) {
     const float y = std::fma(mid[j], 32.0f, 12582944.0f);
@@ -507,7 +729,8 @@ void build_tables(CodeTables* T) {
     std::memcpy(&bits, &y, 4);
     bucket_of[j] = std::min(std::max(bits - 0x4B400000, 0), 64);
   }
-  for (int b = 0; b < 65; ++b) {
+  // Indices 65..127 never occur for |x| <= 1 + 2^-23; they hold "above all".
+  for (int b = 0; b < 128; ++b) {
     int base = 0;
     float thr = INFINITY;
     for (int j = 0; j < 15; ++j) {
@@ -551,6 +774,8 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.key1 = (uint32_t)(c.seed >> 32);
   a.t_lo = (uint32_t)t;
   a.lm_sr_active = (c.total_steps > 0) && (10 * t > 9 * c.total_steps);
+  a.status = nullptr;
+  a.fault_stall = 0;
   return a;
 }
 
@@ -615,21 +840,30 @@ int occupancy_grid(int device, int* grid) {
   int sms = 0, per_sm = 0;
   cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
   if (e != cudaSuccess) return (int)e;
+  // The stage rings live in dynamic shared memory above the 48 KB default.
+  e = cudaFuncSetAttribute(adamw4_step_kernel<VCODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemStages);
+  if (e != cudaSuccess) return (int)e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adamw4_step_kernel<VCODE>,
-                                                    kThreads, 0);
+                                                    kThreads, kSmemStages);
   if (e != cudaSuccess) return (int)e;
   *grid = sms * std::max(per_sm, 1);
   return 0;
 }
 
-int launch(adamw4_handle* h, const StepArgs& a, cudaStream_t s) {
+int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
   if (h->nunits == 0) return ADAMW4_OK;
-  const int64_t need = (h->nunits + (kThreads / kLanesPerUnit) - 1) / (kThreads / kLanesPerUnit);
+  const int64_t need = (h->nunits + kHalves - 1) / kHalves;
   const int grid = (int)std::min<int64_t>(h->grid, need);
+  a.status = h->d_status;
+  a.fault_stall = h->fault_stall;
+  h->fault_stall = 0;
   if (h->cfg.vcode == kVZip)
-    adamw4_step_kernel<kVZip><<<grid, kThreads, 0, s>>>(h->d_tensors, h->nunits, a, h->tabs, h->st);
+    adamw4_step_kernel<kVZip><<<grid, kThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
+                                                                  h->tabs, h->st);
   else
-    adamw4_step_kernel<kVZe><<<grid, kThreads, 0, s>>>(h->d_tensors, h->nunits, a, h->tabs, h->st);
+    adamw4_step_kernel<kVZe><<<grid, kThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
+                                                                 h->tabs, h->st);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(h, e, "step kernel launch");
   return ADAMW4_OK;
@@ -723,7 +957,8 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
   const size_t o_vs = off; off = align_up(off + scales, 256);
   const size_t o_fm = off; off = align_up(off + fp, 256);
   const size_t o_fv = off; off = align_up(off + fp, 256);
-  h->arena_bytes = std::max<size_t>(off, 256);
+  const size_t o_st = off; off = align_up(off + sizeof(uint32_t), 256);
+  h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->d_arena, h->arena_bytes);
   if (e != cudaSuccess) {
     delete h;
@@ -742,6 +977,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
   h->st.vscale = reinterpret_cast<float*>(base + o_vs);
   h->st.fm = reinterpret_cast<float*>(base + o_fm);
   h->st.fv = reinterpret_cast<float*>(base + o_fv);
+  h->d_status = reinterpret_cast<uint32_t*>(base + o_st);
   if ((e = cudaMemset(h->d_arena, 0, h->arena_bytes)) != cudaSuccess ||
       (e = cudaMemcpy(h->d_tensors, dev.data(), sizeof(DevTensor) * dev.size(),
                       cudaMemcpyHostToDevice)) != cudaSuccess) {
@@ -971,9 +1207,36 @@ extern "C" int adamw4_state_import(adamw4_handle* h, const void* host_buf, int64
   return ADAMW4_OK;
 }
 
+extern "C" int adamw4_sync(adamw4_handle* h, void* cuda_stream) {
+  if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return cuda_fail(h, dg.err, "selecting the device");
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "synchronising the stream");
+  uint32_t status = 0;
+  e = cudaMemcpy(&status, h->d_status, sizeof status, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "reading the status word");
+  if (status != 0) {
+    e = cudaMemset(h->d_status, 0, sizeof status);
+    if (e != cudaSuccess) return cuda_fail(h, e, "clearing the status word");
+    return fail(h, ADAMW4_ETIMEOUT,
+                "a stage wait in the step kernel ran out of time; the step is incomplete");
+  }
+  return ADAMW4_OK;
+}
+
+extern "C" int adamw4_inject_fault(adamw4_handle* h, int fault) {
+  if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
+  if (fault != 0 && fault != ADAMW4_FAULT_STALL_PIPELINE)
+    return fail(h, ADAMW4_EINVAL, "unknown fault");
+  h->fault_stall = (fault == ADAMW4_FAULT_STALL_PIPELINE);
+  return ADAMW4_OK;
+}
+
 extern "C" int adamw4_launch_info(const adamw4_handle* h, int* grid, int* block, int64_t* units) {
   if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
-  const int64_t need = (h->nunits + (kThreads / kLanesPerUnit) - 1) / (kThreads / kLanesPerUnit);
+  const int64_t need = (h->nunits + kHalves - 1) / kHalves;
   if (grid) *grid = (int)std::min<int64_t>(h->grid, need);
   if (block) *block = kThreads;
   if (units) *units = h->nunits;

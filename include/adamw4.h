@@ -57,8 +57,14 @@ typedef enum {
     ADAMW4_ENOMEM = -3,     /* device or host allocation failed                */
     ADAMW4_ECUDA = -4,      /* a CUDA runtime call or kernel launch failed     */
     ADAMW4_ESTATE = -5,     /* state blob does not match this handle           */
-    ADAMW4_ERANGE = -6      /* size above a stated maximum                     */
+    ADAMW4_ERANGE = -6,     /* size above a stated maximum                     */
+    ADAMW4_ETIMEOUT = -7    /* a bounded wait inside the step kernel ran out   */
 } adamw4_status;
+
+/* Faults adamw4_inject_fault can arm (test hooks; no GPU fault is raised). */
+enum {
+    ADAMW4_FAULT_STALL_PIPELINE = 1  /* next step: stages marked pending, never filled */
+};
 
 typedef enum {
     ADAMW4_V_ZIPSR = 0,     /* zero-inclusive code, preconditioner-space SR    */
@@ -138,6 +144,21 @@ int adamw4_step(adamw4_handle *h, float lr, void *cuda_stream);
  * Either array may be NULL to skip that direction. */
 int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_host,
                      float *const *params_host, void *cuda_stream);
+
+/* Waits for `cuda_stream` and reports whether the steps enqueued on it so far
+ * completed.  The step kernel bounds every wait on its shared-memory pipeline
+ * (about one second); when a wait runs out, the kernel records it in a device
+ * status word and its half-warp stops, leaving that step incomplete.  This
+ * call reads and clears the word: ADAMW4_ETIMEOUT if it was set, ADAMW4_ECUDA
+ * on a CUDA error, else ADAMW4_OK.  The CUDA context stays usable. */
+int adamw4_sync(adamw4_handle *h, void *cuda_stream);
+
+/* Test hook: arms `fault` (ADAMW4_FAULT_STALL_PIPELINE, or 0 to disarm) for
+ * the next adamw4_step only.  With the stall armed the kernel marks its
+ * pipeline stages as filled without issuing the copies, so every stage wait
+ * runs out after its time limit and adamw4_sync then returns ADAMW4_ETIMEOUT.
+ * Nothing faults; the handle's state after that step is unspecified. */
+int adamw4_inject_fault(adamw4_handle *h, int fault);
 
 /* Frees the state and the handle.  Unknown or already destroyed handles
  * return ADAMW4_EINVAL. */

@@ -165,3 +165,27 @@ def test_host_buffer_step_matches_device_step():
     for x, y in zip(hp, wa):
         assert np.array_equal(x.numpy(), y)
     b.close()
+
+
+def test_pipeline_wait_timeout_is_reported_and_context_survives():
+    """Failure detection without a GPU fault: the test hook marks the kernel's
+    pipeline stages as filled without issuing copies, so every stage wait runs
+    out after its one-second limit; adamw4_sync reports ADAMW4_ETIMEOUT and the
+    next step on the same handle and context completes normally."""
+    import torch
+    B = binding()
+    ts = workloads.tensor_list("single-65k")
+    ws = workloads.host_weights("single-65k", ts)
+    g = GpuRun(ts, ws)
+    try:
+        B.adamw4_inject_fault(g.opt.handle, B.ADAMW4_FAULT_STALL_PIPELINE)
+        g.step(workloads.host_grads("single-65k", ts, 1))
+        with pytest.raises(B.AdamW4Error) as err:
+            g.opt.sync()
+        assert err.value.code == B.ADAMW4_ETIMEOUT
+        g.opt.sync()                      # the status word was cleared
+        g.step(workloads.host_grads("single-65k", ts, 2))
+        g.opt.sync()
+        assert all(np.isfinite(w).all() for w in g.weights())
+    finally:
+        g.close()
