@@ -69,52 +69,91 @@ _u32p = np.ctypeslib.ndpointer(np.uint32, flags="C_CONTIGUOUS")
 _i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
 
 
+def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
+    S = ctypes.POINTER(Scalars)
+    c = ctypes
+    L.oracle_philox4x32_10.argtypes = [_u32p, _u32p, _u32p]
+    L.oracle_draw_word.restype = c.c_uint32
+    L.oracle_draw_word.argtypes = [c.c_uint64, c.c_int64, c.c_uint32, c.c_uint32, c.c_uint64]
+    L.oracle_uniform.restype = c.c_float
+    L.oracle_uniform.argtypes = [c.c_uint32]
+    L.oracle_nf4_levels_f64.argtypes = [_f64p]
+    L.oracle_tables.argtypes = [_f32p, _f32p, _f32p, _f32p]
+    L.oracle_make_scalars.argtypes = [c.c_float, c.c_float, c.c_float, c.c_float,
+                                      c.c_int64, c.c_int64, c.c_uint64, S]
+    L.oracle_decay.restype = c.c_float
+    L.oracle_decay.argtypes = [c.c_float, c.c_float]
+    L.oracle_update_elem.restype = c.c_float
+    L.oracle_update_elem.argtypes = [S, c.c_float, c.c_float, c.c_float, c.c_float,
+                                     c.POINTER(c.c_float), c.POINTER(c.c_float),
+                                     c.POINTER(c.c_float)]
+    L.oracle_nf4_rtn.restype = c.c_int
+    L.oracle_nf4_rtn.argtypes = [c.c_float]
+    L.oracle_nf4_sr.restype = c.c_int
+    L.oracle_nf4_sr.argtypes = [c.c_float, c.c_float]
+    L.oracle_zipsr_bracket.restype = c.c_int
+    L.oracle_zipsr_bracket.argtypes = [c.c_float]
+    L.oracle_zipsr_decide.restype = c.c_int
+    L.oracle_zipsr_decide.argtypes = [c.c_float] * 5
+    L.oracle_zeeden_code.restype = c.c_int
+    L.oracle_zeeden_code.argtypes = [c.c_float]
+    L.oracle_zeeden_factor.restype = c.c_float
+    L.oracle_zeeden_factor.argtypes = [_f32p, _f32p]
+    L.oracle_block4.argtypes = [S, c.c_float, c.c_int, c.c_int, c.c_uint32, c.c_uint64,
+                                c.c_int, _f32p, _u16p, _u8p, _f32p, _u8p, _f32p]
+    L.oracle_step_tensor4.argtypes = [S, c.c_float, c.c_int, c.c_int, c.c_uint32,
+                                      c.c_int64, _f32p, _u16p, _u8p, _f32p, _u8p,
+                                      _f32p, c.c_int]
+    L.oracle_step_blocks4.argtypes = [S, c.c_float, c.c_int, c.c_int, c.c_uint32,
+                                      c.c_int64, c.c_int64, _i64p, _f32p, _u16p, _u8p,
+                                      _f32p, _u8p, _f32p]
+    L.oracle_step_fp32.argtypes = [S, c.c_float, c.c_int64, _f32p, _u16p, _f32p, _f32p]
+    L.oracle_max_threads.restype = c.c_int
+    return L
+
+
 def lib() -> ctypes.CDLL:
     global _lib
     with _lock:
         if _lib is None:
-            L = ctypes.CDLL(build())
-            S = ctypes.POINTER(Scalars)
-            c = ctypes
-            L.oracle_philox4x32_10.argtypes = [_u32p, _u32p, _u32p]
-            L.oracle_draw_word.restype = c.c_uint32
-            L.oracle_draw_word.argtypes = [c.c_uint64, c.c_int64, c.c_uint32, c.c_uint32, c.c_uint64]
-            L.oracle_uniform.restype = c.c_float
-            L.oracle_uniform.argtypes = [c.c_uint32]
-            L.oracle_nf4_levels_f64.argtypes = [_f64p]
-            L.oracle_tables.argtypes = [_f32p, _f32p, _f32p, _f32p]
-            L.oracle_make_scalars.argtypes = [c.c_float, c.c_float, c.c_float, c.c_float,
-                                              c.c_int64, c.c_int64, c.c_uint64, S]
-            L.oracle_decay.restype = c.c_float
-            L.oracle_decay.argtypes = [c.c_float, c.c_float]
-            L.oracle_update_elem.restype = c.c_float
-            L.oracle_update_elem.argtypes = [S, c.c_float, c.c_float, c.c_float, c.c_float,
-                                             c.POINTER(c.c_float), c.POINTER(c.c_float),
-                                             c.POINTER(c.c_float)]
-            L.oracle_nf4_rtn.restype = c.c_int
-            L.oracle_nf4_rtn.argtypes = [c.c_float]
-            L.oracle_nf4_sr.restype = c.c_int
-            L.oracle_nf4_sr.argtypes = [c.c_float, c.c_float]
-            L.oracle_zipsr_bracket.restype = c.c_int
-            L.oracle_zipsr_bracket.argtypes = [c.c_float]
-            L.oracle_zipsr_decide.restype = c.c_int
-            L.oracle_zipsr_decide.argtypes = [c.c_float] * 5
-            L.oracle_zeeden_code.restype = c.c_int
-            L.oracle_zeeden_code.argtypes = [c.c_float]
-            L.oracle_zeeden_factor.restype = c.c_float
-            L.oracle_zeeden_factor.argtypes = [_f32p, _f32p]
-            L.oracle_block4.argtypes = [S, c.c_float, c.c_int, c.c_int, c.c_uint32, c.c_uint64,
-                                        c.c_int, _f32p, _u16p, _u8p, _f32p, _u8p, _f32p]
-            L.oracle_step_tensor4.argtypes = [S, c.c_float, c.c_int, c.c_int, c.c_uint32,
-                                              c.c_int64, _f32p, _u16p, _u8p, _f32p, _u8p,
-                                              _f32p, c.c_int]
-            L.oracle_step_blocks4.argtypes = [S, c.c_float, c.c_int, c.c_int, c.c_uint32,
-                                              c.c_int64, c.c_int64, _i64p, _f32p, _u16p, _u8p,
-                                              _f32p, _u8p, _f32p]
-            L.oracle_step_fp32.argtypes = [S, c.c_float, c.c_int64, _f32p, _u16p, _f32p, _f32p]
-            L.oracle_max_threads.restype = c.c_int
-            _lib = L
+            _lib = _bind(ctypes.CDLL(build()))
     return _lib
+
+
+def build_variant(source_text: str, out_path: str) -> str:
+    """Compiles a modified copy of the oracle source (used by the tests that
+    plant mistakes in the oracle to show that the pins catch them)."""
+    src = out_path + ".c"
+    with open(src, "w") as f:
+        f.write(source_text)
+    cmd = ["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+           "-fopenmp", src, "-o", out_path, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True)
+    return out_path
+
+
+class use_library:
+    """Context manager: route every oracle call to the library at `path`."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        lib()
+        self.saved = _lib
+        _lib = _bind(ctypes.CDLL(self.path))
+        return _lib
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
+
+
+def source() -> str:
+    with open(_SRC) as f:
+        return f.read()
 
 
 # ----------------------------------------------------------------------------

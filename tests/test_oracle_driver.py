@@ -92,3 +92,22 @@ def test_lm_head_phase_changes_only_the_head_m_codes():
     assert not np.array_equal(a.tensors[0].mcodes, b.tensors[0].mcodes)
     assert np.array_equal(a.tensors[0].vcodes, b.tensors[0].vcodes)
     assert np.array_equal(a.tensors[1].mcodes, b.tensors[1].mcodes)
+
+
+def test_nibble_layout_of_the_codes():
+    """Element 2i sits in the low nibble of byte i and 2i+1 in the high one
+    (the checkpoint layout).  A block whose only nonzero first moment is
+    element 1 (byte 0 = 0xF7: element 0 on the NF4 zero level, element 1 on
+    +1) moves weight 1 and leaves weight 0 alone when the gradients are zero."""
+    s = oracle.make_scalars(1e-3, 0.9, 0.999, 1e-8, t=5)
+    w0 = np.full(128, 0.25, np.float32)
+    w = w0.copy()
+    g = np.zeros(128, np.uint16)
+    mc = np.full(64, 0x77, np.uint8)
+    mc[0] = 0xF7
+    vc = np.zeros(64, np.uint8)
+    ms = np.ones(1, np.float32)
+    vs = np.zeros(1, np.float32)
+    oracle.lib().oracle_block4(s, np.float32(1.0), 0, 0, 0, 0, 128, w, g, mc, ms, vc, vs)
+    assert w[0] == w0[0] and np.all(w[2:] == w0[2:])
+    assert w[1] < w0[1] - 1.0

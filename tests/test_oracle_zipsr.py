@@ -184,3 +184,14 @@ def test_monte_carlo_unbiased_in_h(v_frac):
     assert hs.size >= 10 ** 6
     mean, sd = hs.mean(), hs.std() / np.sqrt(hs.size)
     assert abs(mean - h_true) < 4 * sd + 1e-6 * h_true
+
+
+def test_bracket_at_and_below_code_points():
+    """The ZIP-SR bracket of a value exactly on code point k is [k, k+1] (k
+    for the top one, 14), and one binary32 step below it is [k-1, k]."""
+    _, _, vz, _ = oracle.tables()
+    for k in range(1, 16):
+        assert oracle.zipsr_bracket(float(vz[k])) == min(k, 14)
+        below = float(np.nextafter(vz[k], np.float32(-1)))
+        assert oracle.zipsr_bracket(below) == k - 1
+    assert oracle.zipsr_bracket(0.0) == 0
