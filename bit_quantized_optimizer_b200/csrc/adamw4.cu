@@ -3,21 +3,24 @@
 //
 // One kernel launch per step covers every parameter tensor.  The work is a flat
 // list of 128-value units: each block of a 4-bit tensor is one unit, and each
-// fp32-state tensor is cut into 128-element chunks.  A half-warp owns one unit
-// at a time (16 lanes x 8 contiguous values).  The grid is persistent (SM count
-// x resident CTAs) and half-warps stride through the unit list, so all SMs
-// stream one contiguous window of HBM.
+// fp32-state tensor is cut into 128-element chunks.  The grid is persistent
+// (SM count x resident CTAs) and the units are dealt out round-robin, so all
+// SMs stream one contiguous window of HBM.
 //
-// Memory pipeline: every half-warp keeps kStages units in flight in its own
-// shared-memory ring.  Lane 0 fills a stage with TMA bulk copies
-// (cp.async.bulk: 512 B of fp32 weights, 256 B of bf16 grads, 64 + 64 B of
-// codes) plus two 4-byte cp.async copies of the block scales, all completing on
-// the stage's mbarrier.  The half-warp waits on the barrier (bounded by a
-// timer; on expiry the kernel records an error in a status word and leaves),
-// computes from shared memory, stores the results straight to global memory,
-// and refills the stage with the unit kStages ahead.  Units that are not whole
-// 4-bit blocks (a ragged last block, fp32-state chunks) take a direct path with
-// plain guarded loads.
+// A CTA has one producer warp and eight consumer warps.  Each consumer
+// half-warp owns a ring of kStages shared-memory stages; producer lane j feeds
+// the ring of half-warp j.  For every unit the producer writes a 64-byte header
+// (addresses, block index, tensor id, flags, decay) into the stage and, for a
+// whole 4-bit block, fills the stage with TMA bulk copies (cp.async.bulk: 512 B
+// of fp32 weights, 256 B of bf16 grads, 64 + 64 B of codes) plus two 4-byte
+// cp.async copies of the block scales, all completing on the stage's "full"
+// mbarrier.  The consumer half-warp waits on it, computes from the stage,
+// stores the results straight to global memory and hands the stage back on
+// its "empty" mbarrier.  Units that are not whole
+// 4-bit blocks (a ragged last block, fp32-state chunks) carry only the header
+// and are read from global memory by the consumer.  Every wait is bounded by
+// a timer; on expiry the kernel records the failure in a status word and the
+// waiting warp leaves.
 //
 // Per unit, following the method flowchart of "ZIP-SR / ZE-EDEN: 4-bit AdamW
 // state quantization" (daiwk.github.io, Method): decode the prior moments,
@@ -54,27 +57,32 @@
 
 namespace {
 
-constexpr int kBlock = ADAMW4_BLOCK;        // values per quantisation block
-constexpr int kLanesPerUnit = 16;           // a half-warp per block
+constexpr int kBlock = ADAMW4_BLOCK;              // values per quantisation block
+constexpr int kLanesPerUnit = 16;                 // a half-warp per block
 constexpr int kPerLane = kBlock / kLanesPerUnit;  // 8 values per lane
-constexpr int kThreads = 256;               // threads per CTA
-constexpr int kHalves = kThreads / kLanesPerUnit; // half-warps per CTA
-constexpr int kStages = 4;                  // units in flight per half-warp
-// Stage layout: w 512 B | g 256 B | m codes 64 B | v codes 64 B | m scale | v scale
-constexpr int kOffW = 0, kOffG = 512, kOffMC = 768, kOffVC = 832, kOffMS = 896, kOffVS = 900;
-constexpr int kStageBytes = 912;            // 16-byte multiple
-constexpr uint32_t kStageTx = 896;          // bytes delivered by the bulk copies
+constexpr int kConsumerThreads = 256;             // eight consumer warps
+constexpr int kCtaThreads = kConsumerThreads + 32;  // plus the producer warp
+constexpr int kHalves = kConsumerThreads / kLanesPerUnit;  // consumer half-warps per CTA
+constexpr int kProducerWarp = kConsumerThreads / 32;
+constexpr int kStages = 4;                        // units in flight per half-warp
+// Stage layout: header 64 B | w 512 B | g 256 B | m codes 64 B | v codes 64 B |
+// m scale 4 B | v scale 4 B
+constexpr int kOffHdr = 0, kOffW = 64, kOffG = 576, kOffMC = 832, kOffVC = 896, kOffMS = 960,
+              kOffVS = 964;
+constexpr int kStageBytes = 976;                  // 16-byte multiple
+constexpr uint32_t kStageTx = 896;                // bytes delivered by the bulk copies
 constexpr int kSmemStages = kHalves * kStages * kStageBytes;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per stage wait
-constexpr uint64_t kDrainLimitNs = 10000000ull;    // 10 ms per stage when draining
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr int kVZip = ADAMW4_V_ZIPSR;
 constexpr int kVZe = ADAMW4_V_ZEEDEN;
-constexpr uint32_t kKindFp32 = 1u << 16;    // internal flag: fp32-state tensor
-constexpr uint32_t kStreamV = 0u;           // Philox stream of the v draw
-constexpr uint32_t kStreamM = 1u;           // Philox stream of the LM-head m draw
-constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23: adding it rounds to an integer
+constexpr uint32_t kKindFp32 = 1u << 16;          // internal flag: fp32-state tensor
+constexpr uint32_t kStaged = 1u << 17;            // internal flag: unit data is in the stage
+constexpr uint32_t kStreamV = 0u;                 // Philox stream of the v draw
+constexpr uint32_t kStreamM = 1u;                 // Philox stream of the LM-head m draw
+constexpr float kMagic = 12582912.0f;             // 1.5 * 2^23: adding it rounds to an integer
 
-// Philox4x32-10 round multipliers and key increments (Salmon et al., SC'11).
+// Philox4x32-10 round multipliers (Salmon et al., SC'11).  The per-round keys
+// (key + r * Weyl constants) are formed on the host.
 constexpr uint32_t kPhiloxM0 = 0xD2511F53u;
 constexpr uint32_t kPhiloxM1 = 0xCD9E8D57u;
 constexpr uint32_t kPhiloxW0 = 0x9E3779B9u;
@@ -100,11 +108,11 @@ struct StepArgs {
   float step_size;   // lr / (1 - b1^t)
   float rs_bc2;      // 1 / sqrt(1 - b2^t)
   float b1, omb1, b2, omb2, eps, lr;
-  uint32_t key0, key1;   // Philox key = seed
+  uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   uint32_t t_lo;         // step, low word (Philox counter word 2)
   int lm_sr_active;      // final-10% LM-head phase
   uint32_t* status;      // device status word (bit 0: a pipeline wait timed out)
-  int fault_stall;       // test hook: mark stages pending without filling them
+  int fault_stall;       // test hook: mark stages filled without filling them
 };
 
 // Code tables, passed by value and staged in shared memory by each CTA.
@@ -125,6 +133,20 @@ struct StateArena {
   float* fv;
 };
 
+// What the producer tells the consumer about one unit (64 bytes).
+struct __align__(16) UnitHeader {
+  float* w;              // the unit's first weight
+  const uint16_t* g;     // its first gradient
+  uint64_t e0;           // index of that element within its tensor
+  uint64_t state;        // 4-bit: block index in the code arena; fp32: element index
+  uint32_t tensor_id;
+  uint32_t flags;        // ADAMW4_T_* | kKindFp32 | kStaged
+  float decay;           // 1 - lr * weight_decay of the tensor
+  int32_t nvalid;        // values in the unit (1..128)
+  uint32_t pad_[4];
+};
+static_assert(sizeof(UnitHeader) == 64, "UnitHeader layout");
+
 // ---------------------------------------------------------------------------
 // PTX wrappers: mbarrier, bulk copies, timer
 // ---------------------------------------------------------------------------
@@ -142,8 +164,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+__device__ __forceinline__ void mbar_arrive(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -170,6 +192,9 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -179,12 +204,27 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Waits for a barrier phase; false if `limit_ns` passed first.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for a barrier phase; false if `limit_ns` passed first.  The timer is
+// read once per 64 polls.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (global_ns() - t0 > limit_ns) return false;
   }
 }
@@ -193,17 +233,13 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint64
 // Arithmetic helpers
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const StepArgs& a) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += kPhiloxW0;
-      k1 += kPhiloxW1;
-    }
     const uint64_t p0 = (uint64_t)kPhiloxM0 * c.x;
     const uint64_t p1 = (uint64_t)kPhiloxM1 * c.z;
-    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1,
-                   (uint32_t)p0);
+    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ a.rk0[r], (uint32_t)p1,
+                   (uint32_t)(p0 >> 32) ^ c.w ^ a.rk1[r], (uint32_t)p0);
   }
   return c;
 }
@@ -217,11 +253,9 @@ __device__ __forceinline__ float uniform23(uint32_t w) {
 __device__ __forceinline__ void draws8(const StepArgs& a, uint32_t tensor_id, uint32_t stream,
                                        uint64_t quad, float u[8]) {
   const uint32_t c3 = tensor_id * 2u + stream;
-  const uint4 r0 = philox4x32_10(make_uint4((uint32_t)quad, (uint32_t)(quad >> 32), a.t_lo, c3),
-                                 a.key0, a.key1);
+  const uint4 r0 = philox4x32_10(make_uint4((uint32_t)quad, (uint32_t)(quad >> 32), a.t_lo, c3), a);
   const uint64_t q1 = quad + 1;
-  const uint4 r1 = philox4x32_10(make_uint4((uint32_t)q1, (uint32_t)(q1 >> 32), a.t_lo, c3),
-                                 a.key0, a.key1);
+  const uint4 r1 = philox4x32_10(make_uint4((uint32_t)q1, (uint32_t)(q1 >> 32), a.t_lo, c3), a);
   u[0] = uniform23(r0.x); u[1] = uniform23(r0.y); u[2] = uniform23(r0.z); u[3] = uniform23(r0.w);
   u[4] = uniform23(r1.x); u[5] = uniform23(r1.y); u[6] = uniform23(r1.z); u[7] = uniform23(r1.w);
 }
@@ -266,51 +300,62 @@ __device__ __forceinline__ uint32_t nf4_sr(float x, float u, const float* nf4, c
 
 // Shared tables of one CTA.
 struct SmemTables {
+  float2 mpair[256];   // byte of two m codes -> their two NF4 levels
+  float2 vpair[256];   // byte of two v codes -> their two code points
+  float2 rtn[128];
   float nf4[16];
   float gap[16];
-  float vq[16];        // decoded v code points: k/15 (ZIP-SR) or (k+1)/16 (ZE-EDEN)
   float vz[16];        // ZIP-SR code points k/15
   float2 sqp[16];      // {sqrt(k/15), sqrt((k+1)/15)}
   float2 vzp[16];      // {k/15, (k+1)/15}
-  float2 rtn[128];
 };
-
-// Per-tensor values a half-warp keeps while it walks the unit list.
-struct Cursor {
-  int ti;
-  int64_t begin, end, numel, soff;
-  float* param;
-  const uint16_t* grad;
-  uint32_t id, flags;
-  float wd;
-};
-
-__device__ __forceinline__ void cursor_seek(Cursor& c, const DevTensor* __restrict__ T,
-                                            int64_t u) {
-  if (u < c.end) return;
-  do {
-    ++c.ti;
-    c.end = __ldg(&T[c.ti].unit_end);
-  } while (u >= c.end);
-  const DevTensor* d = &T[c.ti];
-  c.begin = __ldg(&d->unit_begin);
-  c.numel = __ldg(&d->numel);
-  c.soff = __ldg(&d->state_off);
-  c.param = d->param;
-  c.grad = d->grad;
-  c.id = __ldg(&d->tensor_id);
-  c.flags = __ldg(&d->flags);
-  c.wd = __ldg(&d->weight_decay);
-}
 
 // ---------------------------------------------------------------------------
 // Requantisation of one 4-bit block held by a half-warp (8 values per lane).
 // FULL: all 128 values valid.  Otherwise `myn` values of this lane are valid.
 // ---------------------------------------------------------------------------
+
+// ZIP-SR codes of 8 values.  FLAT: also test for d(a) == d(b), which needs the
+// state-space fallback; callers skip it when the block's R makes that
+// impossible.
+template <bool FULL, bool FLAT>
+__device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
+                                                 const float (&v1)[kPerLane],
+                                                 const float (&den)[kPerLane],
+                                                 const float (&ud)[kPerLane], float inv, float R,
+                                                 int myn) {
+  uint32_t vco = 0;
+#pragma unroll
+  for (int j = 0; j < kPerLane / 2; ++j) {
+    const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+    const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 2 * j + h;
+      const float x = h ? x2.y : x2.x;
+      // the nearest integer to 15x is the bracket or one above it
+      int k = (int)(__float_as_uint(h ? t2.y : t2.x) & 31u);
+      k -= (x < S.vz[k]) ? 1 : 0;
+      k = min(k, 14);
+      const float2 dd = __ffma2_rn(S.sqp[k], f2(R), f2(a.eps));               // (da, db)
+      const float2 ad = __fadd2_rn(f2(dd.y), make_float2(-dd.x, -den[i]));   // (db-da, db-dv)
+      const float2 pr = __fmul2_rn(ad, make_float2(den[i], dd.x));           // (.*dv, .*da)
+      bool lower = __fmul_rn(ud[i], pr.x) < pr.y;
+      if (FLAT && dd.x == dd.y) {
+        const float2 z = S.vzp[k];
+        lower = __fmul_rn(ud[i], __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
+      }
+      if (FULL || i < myn) vco |= (uint32_t)(k + (lower ? 0 : 1)) << (4 * i);
+    }
+  }
+  return vco;
+}
+
 template <int VCODE, bool FULL>
 __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTables& S,
-                                              const Cursor& c, int64_t e0, int lane, int myn,
-                                              unsigned hmask, const float (&m1)[kPerLane],
+                                              uint32_t tensor_id, uint32_t flags, uint64_t e0,
+                                              int lane, int myn, unsigned hmask,
+                                              const float (&m1)[kPerLane],
                                               const float (&v1)[kPerLane],
                                               const float (&den)[kPerLane], uint32_t* mcw,
                                               uint32_t* vcw, float* msp, float* vsp) {
@@ -330,9 +375,9 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   float mso = 0.0f;
   if (am >= FLT_MIN) {
     const float inv = __fdiv_rn(1.0f, am);
-    if ((c.flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
+    if ((flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
       float ud[kPerLane];
-      draws8(a, c.id, kStreamM, (uint64_t)(e0 + lane * kPerLane) >> 2, ud);
+      draws8(a, tensor_id, kStreamM, (e0 + (uint64_t)(lane * kPerLane)) >> 2, ud);
 #pragma unroll
       for (int i = 0; i < kPerLane; ++i)
         if (FULL || i < myn) mco |= nf4_sr(__fmul_rn(m1[i], inv), ud[i], S.nf4, S.gap) << (4 * i);
@@ -361,31 +406,13 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
       const float R = __fmul_rn(__fsqrt_rn(av), a.rs_bc2);
       float ud[kPerLane];
-      draws8(a, c.id, kStreamV, (uint64_t)(e0 + lane * kPerLane) >> 2, ud);
-#pragma unroll
-      for (int j = 0; j < kPerLane / 2; ++j) {
-        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
-        const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int i = 2 * j + h;
-          const float x = h ? x2.y : x2.x;
-          // nearest of 15x is the bracket or one above it; step down if needed
-          int k = (int)(__float_as_uint(h ? t2.y : t2.x) & 31u);
-          k -= (x < S.vz[k]) ? 1 : 0;
-          k = min(k, 14);
-          const float2 sq = S.sqp[k];
-          const float2 dd = __ffma2_rn(sq, f2(R), f2(a.eps));        // (da, db)
-          const float2 ad = __fadd2_rn(f2(dd.y), make_float2(-dd.x, -den[i]));  // (db-da, db-dv)
-          const float2 pr = __fmul2_rn(ad, make_float2(den[i], dd.x));          // (..*dv, ..*da)
-          bool lower = __fmul_rn(ud[i], pr.x) < pr.y;
-          if (dd.x == dd.y) {
-            const float2 z = S.vzp[k];
-            lower = __fmul_rn(ud[i], __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
-          }
-          if (FULL || i < myn) vco |= (uint32_t)(k + (lower ? 0 : 1)) << (4 * i);
-        }
-      }
+      draws8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, ud);
+      // d(a) == d(b) needs (sqrt(k+1/15) - sqrt(k/15)) R below two ulps of
+      // R + eps; the smallest gap is 0.0339, so R > 1e-5 eps rules it out.
+      if (R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN)
+        vco = zipsr_codes8<FULL, false>(a, S, v1, den, ud, inv, R, myn);
+      else
+        vco = zipsr_codes8<FULL, true>(a, S, v1, den, ud, inv, R, myn);
       vso = av;
     } else {
       // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
@@ -427,7 +454,6 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
 }
 
 // Decode + moment update + weight update for 8 values of a 4-bit block.
-template <bool FULL>
 __device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, float decay,
                                         float (&w)[kPerLane], const float (&g)[kPerLane],
                                         uint32_t mc, uint32_t vc, float sm, float sv,
@@ -435,10 +461,9 @@ __device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, 
                                         float (&den)[kPerLane]) {
 #pragma unroll
   for (int j = 0; j < kPerLane / 2; ++j) {
-    const float2 m0 = __fmul2_rn(
-        make_float2(S.nf4[(mc >> (8 * j)) & 15u], S.nf4[(mc >> (8 * j + 4)) & 15u]), f2(sm));
-    const float2 v0 = __fmul2_rn(
-        make_float2(S.vq[(vc >> (8 * j)) & 15u], S.vq[(vc >> (8 * j + 4)) & 15u]), f2(sv));
+    // one byte holds the codes of values 2j (low nibble) and 2j+1 (high nibble)
+    const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], f2(sm));
+    const float2 v0 = __fmul2_rn(S.vpair[__byte_perm(vc, 0, 0x4440 + j)], f2(sv));
     const float2 gg = make_float2(g[2 * j], g[2 * j + 1]);
     const float2 mm = __ffma2_rn(f2(a.b1), m0, __fmul2_rn(f2(a.omb1), gg));
     const float2 vv = __ffma2_rn(f2(a.b2), v0, __fmul2_rn(f2(a.omb2), __fmul2_rn(gg, gg)));
@@ -457,25 +482,25 @@ __device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, 
 // A unit read straight from global memory: a ragged last 4-bit block or a
 // chunk of an fp32-state tensor.
 template <int VCODE>
-__device__ __noinline__ void process_direct(const StepArgs& a, const SmemTables& S,
-                                            const StateArena& st, const Cursor& c, float decay,
-                                            int64_t u, int lane, unsigned hmask) {
-  const int64_t ub = u - c.begin;
-  const int64_t e0 = ub * kBlock;
-  const int nvalid = (int)min((int64_t)kBlock, c.numel - e0);
+__device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTables& S,
+                                            const StateArena& st, const UnitHeader* hdp,
+                                            int lane, unsigned hmask) {
   const int my0 = lane * kPerLane;
-  const int myn = min(max(nvalid - my0, 0), kPerLane);
-  float* wp = c.param + e0 + my0;
-  const uint16_t* gp = c.grad + e0 + my0;
+  const int myn = min(max(hdp->nvalid - my0, 0), kPerLane);
+  const uint32_t flags = hdp->flags;
+  const float decay = hdp->decay;
+  const uint64_t state = hdp->state;
+  float* wp = hdp->w + my0;
+  const uint16_t* gp = hdp->g + my0;
   float w[kPerLane], g[kPerLane];
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
     w[i] = (i < myn) ? wp[i] : 0.0f;
     g[i] = (i < myn) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
   }
-  if (c.flags & kKindFp32) {
-    float* mp = st.fm + c.soff + e0 + my0;
-    float* vp = st.fv + c.soff + e0 + my0;
+  if (flags & kKindFp32) {
+    float* mp = st.fm + state + my0;
+    float* vp = st.fv + state + my0;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
       if (i < myn) {
@@ -489,16 +514,108 @@ __device__ __noinline__ void process_direct(const StepArgs& a, const SmemTables&
     }
     return;
   }
-  const int64_t blk = c.soff + ub;
+  const uint64_t blk = state;
   uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
   uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
   float m1[kPerLane], v1[kPerLane], den[kPerLane];
-  update8<false>(a, S, decay, w, g, *mcw, *vcw, st.mscale[blk], st.vscale[blk], m1, v1, den);
+  update8(a, S, decay, w, g, *mcw, *vcw, st.mscale[blk], st.vscale[blk], m1, v1, den);
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i)
     if (i < myn) wp[i] = w[i];
-  requant_store<VCODE, false>(a, S, c, e0, lane, myn, hmask, m1, v1, den, mcw, vcw,
-                              st.mscale + blk, st.vscale + blk);
+  requant_store<VCODE, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask, m1, v1,
+                              den, mcw, vcw, st.mscale + blk, st.vscale + blk);
+}
+
+// ---------------------------------------------------------------------------
+// Producer: lane j fills the stage ring of consumer half-warp j.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t nunits,
+                                        const StepArgs& a, const StateArena& st, uint8_t* stages,
+                                        uint32_t full0, uint32_t empty0, int j) {
+  const int64_t H = (int64_t)gridDim.x * kHalves;
+  int ti = -1;
+  int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0;
+  float* t_param = nullptr;
+  const uint16_t* t_grad = nullptr;
+  uint32_t t_id = 0, t_flags = 0;
+  float t_decay = 1.0f;
+  uint8_t* my = stages + j * (kStages * kStageBytes);
+  const uint32_t my_s = smem_addr(my);
+  int s = 0;
+  uint32_t round = 0;     // completed passes over the ring
+  uint64_t stalled_since = 0;
+  // Each lane refills its own ring as soon as its consumer hands a stage back,
+  // independently of the other lanes; the warp naps only when no lane could
+  // make progress.
+  for (int64_t u = (int64_t)blockIdx.x * kHalves + j; u < nunits;) {
+    const uint32_t full = full0 + 8u * (j * kStages + s);
+    const bool ready =
+        round == 0 || mbar_test_wait(empty0 + 8u * (j * kStages + s), (round - 1) & 1u);
+    const bool any_ready = __any_sync(__activemask(), ready);
+    if (!ready) {
+      const uint64_t now = global_ns();
+      if (stalled_since == 0) {
+        stalled_since = now;
+      } else if (now - stalled_since > kWaitLimitNs) {
+        atomicOr(a.status, 1u);
+        break;
+      }
+      // consumers spend microseconds per unit: when no stage is free, nap
+      // instead of taking issue slots from them
+      if (!any_ready) __nanosleep(1000);
+      continue;
+    }
+    stalled_since = 0;
+    if (u >= t_end) {
+      do {
+        ++ti;
+        t_end = __ldg(&T[ti].unit_end);
+      } while (u >= t_end);
+      const DevTensor* d = &T[ti];
+      t_begin = __ldg(&d->unit_begin);
+      t_numel = __ldg(&d->numel);
+      t_soff = __ldg(&d->state_off);
+      t_param = d->param;
+      t_grad = d->grad;
+      t_id = __ldg(&d->tensor_id);
+      t_flags = __ldg(&d->flags);
+      t_decay = (float)(1.0 - (double)a.lr * (double)__ldg(&d->weight_decay));
+    }
+    const int64_t ub = u - t_begin;
+    const int64_t e0 = ub * kBlock;
+    const int nvalid = (int)min((int64_t)kBlock, t_numel - e0);
+    const bool staged = !(t_flags & kKindFp32) && nvalid == kBlock;
+    UnitHeader* hd = reinterpret_cast<UnitHeader*>(my + s * kStageBytes + kOffHdr);
+    hd->w = t_param + e0;
+    hd->g = t_grad + e0;
+    hd->e0 = (uint64_t)e0;
+    hd->state = (t_flags & kKindFp32) ? (uint64_t)(t_soff + e0) : (uint64_t)(t_soff + ub);
+    hd->tensor_id = t_id;
+    hd->flags = t_flags | (staged ? kStaged : 0u);
+    hd->decay = t_decay;
+    hd->nvalid = nvalid;
+    if (staged && !a.fault_stall) {
+      const uint32_t dst = my_s + (uint32_t)(s * kStageBytes);
+      const int64_t blk = t_soff + ub;
+      mbar_arrive_expect_tx(full, kStageTx);
+      bulk_g2s(dst + kOffW, t_param + e0, 512, full);
+      bulk_g2s(dst + kOffG, t_grad + e0, 256, full);
+      bulk_g2s(dst + kOffMC, st.mcodes + blk * (kBlock / 2), 64, full);
+      bulk_g2s(dst + kOffVC, st.vcodes + blk * (kBlock / 2), 64, full);
+      cp_async4(dst + kOffMS, st.mscale + blk);
+      cp_async4(dst + kOffVS, st.vscale + blk);
+      cp_async_arrive_noinc(full);
+    } else if (!staged) {
+      mbar_arrive(full, 2);          // header only: complete the phase now
+    }
+    // (test hook: a staged unit with the stall armed never completes)
+    u += H;
+    if (++s == kStages) {
+      s = 0;
+      ++round;
+    }
+  }
+  cp_async_wait_all();               // this thread's 4-byte copies have landed
 }
 
 // ---------------------------------------------------------------------------
@@ -506,98 +623,65 @@ __device__ __noinline__ void process_direct(const StepArgs& a, const SmemTables&
 // ---------------------------------------------------------------------------
 
 template <int VCODE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kCtaThreads, 3)
 adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, CodeTables tabs,
                    StateArena st) {
   extern __shared__ __align__(128) uint8_t s_stage[];
-  __shared__ __align__(8) uint64_t s_bar[kHalves * kStages];
+  __shared__ __align__(8) uint64_t s_full[kHalves * kStages];
+  __shared__ __align__(8) uint64_t s_empty[kHalves * kStages];
   __shared__ SmemTables S;
 
-  if (threadIdx.x < 16) {
-    const int k = threadIdx.x;
-    S.nf4[k] = tabs.nf4[k];
-    S.gap[k] = tabs.nf4_gap[k];
-    S.vz[k] = tabs.vz[k];
-    S.vq[k] = (VCODE == kVZip) ? tabs.vz[k] : __fmul_rn((float)(k + 1), 0.0625f);
-    S.sqp[k] = make_float2(tabs.vz_sqrt[k], tabs.vz_sqrt[min(k + 1, 15)]);
-    S.vzp[k] = make_float2(tabs.vz[k], tabs.vz[min(k + 1, 15)]);
-  }
-  if (threadIdx.x < 128) S.rtn[threadIdx.x] = tabs.rtn[threadIdx.x];
-
-  const int lane = threadIdx.x & 15;
-  const int half = threadIdx.x >> 4;
-  const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
-  const uint32_t stage0 = smem_addr(s_stage) + (uint32_t)(half * kStages * kStageBytes);
-  const uint32_t bar0 = smem_addr(&s_bar[half * kStages]);
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8u * s, 2);
+  {
+    const int t = threadIdx.x;
+    if (t < 256) {
+      S.mpair[t] = make_float2(tabs.nf4[t & 15], tabs.nf4[t >> 4]);
+      const float lo = (VCODE == kVZip) ? tabs.vz[t & 15] : __fmul_rn((float)((t & 15) + 1), 0.0625f);
+      const float hi = (VCODE == kVZip) ? tabs.vz[t >> 4] : __fmul_rn((float)((t >> 4) + 1), 0.0625f);
+      S.vpair[t] = make_float2(lo, hi);
+    }
+    if (t < 128) S.rtn[t] = tabs.rtn[t];
+    if (t < 16) {
+      S.nf4[t] = tabs.nf4[t];
+      S.gap[t] = tabs.nf4_gap[t];
+      S.vz[t] = tabs.vz[t];
+      S.sqp[t] = make_float2(tabs.vz_sqrt[t], tabs.vz_sqrt[min(t + 1, 15)]);
+      S.vzp[t] = make_float2(tabs.vz[t], tabs.vz[min(t + 1, 15)]);
+    }
+    if (t < kHalves * kStages) {
+      mbar_init(smem_addr(&s_full[t]), 2);    // producer arrive + the scales' cp.async arrive
+      mbar_init(smem_addr(&s_empty[t]), 1);   // the consumer half-warp's release
+    }
     fence_mbar_init();
   }
   __syncthreads();
 
-  const int64_t H = (int64_t)gridDim.x * kHalves;
-  const int64_t hw = (int64_t)blockIdx.x * kHalves + half;
-
-  // Issue side: fills stage s with unit ui if it is a whole 4-bit block.
-  Cursor ic{-1, 0, 0, 0, 0, nullptr, nullptr, 0, 0, 0.0f};
-  auto issue = [&](int64_t ui, int s) -> bool {
-    if (ui >= nunits) return false;
-    cursor_seek(ic, T, ui);
-    if (ic.flags & kKindFp32) return false;
-    const int64_t ub = ui - ic.begin;
-    const int64_t e0 = ub * kBlock;
-    if (ic.numel - e0 < kBlock) return false;
-    if (lane == 0) {
-      const uint32_t dst = stage0 + (uint32_t)(s * kStageBytes);
-      const uint32_t bar = bar0 + 8u * s;
-      if (a.fault_stall) return true;      // test hook: nothing will arrive
-      const int64_t blk = ic.soff + ub;
-      mbar_arrive_expect_tx(bar, kStageTx);
-      bulk_g2s(dst + kOffW, ic.param + e0, 512, bar);
-      bulk_g2s(dst + kOffG, ic.grad + e0, 256, bar);
-      bulk_g2s(dst + kOffMC, st.mcodes + blk * (kBlock / 2), 64, bar);
-      bulk_g2s(dst + kOffVC, st.vcodes + blk * (kBlock / 2), 64, bar);
-      cp_async4(dst + kOffMS, st.mscale + blk);
-      cp_async4(dst + kOffVS, st.vscale + blk);
-      cp_async_arrive_noinc(bar);
-    }
-    return true;
-  };
-
-  uint32_t pend = 0, phase = 0;
-  int64_t ui = hw;
-#pragma unroll
-  for (int s = 0; s < kStages; ++s) {
-    if (issue(ui, s)) pend |= 1u << s;
-    ui += H;
+  const uint32_t full0 = smem_addr(&s_full[0]);
+  const uint32_t empty0 = smem_addr(&s_empty[0]);
+  const int warp = threadIdx.x >> 5;
+  if (warp == kProducerWarp) {
+    const int j = threadIdx.x & 31;
+    if (j < kHalves) produce(T, nunits, a, st, s_stage, full0, empty0, j);
+    return;
   }
 
-  Cursor cc{-1, 0, 0, 0, 0, nullptr, nullptr, 0, 0, 0.0f};
-  float decay = 1.0f;
+  // ---- consumers ----
+  const int lane = threadIdx.x & 15;
+  const int half = threadIdx.x >> 4;
+  const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
+  const int64_t H = (int64_t)gridDim.x * kHalves;
+  const uint8_t* ring = s_stage + half * (kStages * kStageBytes);
   int s = 0;
-  for (int64_t u = hw; u < nunits; u += H) {
-    if (u >= cc.end) {
-      cursor_seek(cc, T, u);
-      decay = (float)(1.0 - (double)a.lr * (double)cc.wd);
+  uint32_t parity = 0;
+  for (int64_t u = (int64_t)blockIdx.x * kHalves + half; u < nunits; u += H) {
+    const uint32_t full = full0 + 8u * (half * kStages + s);
+    const uint32_t empty = empty0 + 8u * (half * kStages + s);
+    if (!__all_sync(hmask, wait_phase(full, parity, kWaitLimitNs))) {
+      if (lane == 0) atomicOr(a.status, 1u);
+      return;
     }
-    if ((pend >> s) & 1u) {
-      const uint32_t bar = bar0 + 8u * s;
-      const bool ok = __all_sync(hmask, wait_phase(bar, (phase >> s) & 1u, kWaitLimitNs));
-      if (!ok) {
-        // Leave cleanly: record the failure, let copies still in flight land.
-        if (lane == 0) atomicOr(a.status, 1u);
-        pend &= ~(1u << s);
-        for (int s2 = 0; s2 < kStages; ++s2)
-          if ((pend >> s2) & 1u) wait_phase(bar0 + 8u * s2, (phase >> s2) & 1u, kDrainLimitNs);
-        __syncwarp(hmask);
-        return;
-      }
-      phase ^= 1u << s;
-      const uint8_t* sp = s_stage + (half * kStages + s) * kStageBytes;
-      const int64_t ub = u - cc.begin;
-      const int64_t e0 = ub * kBlock;
-      const int64_t blk = cc.soff + ub;
+    const uint8_t* sp = ring + s * kStageBytes;
+    const UnitHeader* hdp = reinterpret_cast<const UnitHeader*>(sp + kOffHdr);
+    if (hdp->flags & kStaged) {
       float w[kPerLane], g[kPerLane];
       {
         const float4 wa = *reinterpret_cast<const float4*>(sp + kOffW + lane * 32);
@@ -612,28 +696,28 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
       const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + lane * 4);
       const float sm = *reinterpret_cast<const float*>(sp + kOffMS);
       const float sv = *reinterpret_cast<const float*>(sp + kOffVS);
-      // every read of the stage is done: hand it back to the async proxy
-      fence_proxy_async_smem();
-      __syncwarp(hmask);
-      pend &= ~(1u << s);
-      if (issue(ui, s)) pend |= 1u << s;
-      ui += H;
 
       float m1[kPerLane], v1[kPerLane], den[kPerLane];
-      update8<true>(a, S, decay, w, g, mc, vc, sm, sv, m1, v1, den);
-      float* wp = cc.param + e0 + lane * kPerLane;
+      update8(a, S, hdp->decay, w, g, mc, vc, sm, sv, m1, v1, den);
+      float* wp = hdp->w + lane * kPerLane;
       *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
       *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
+      const uint64_t blk = hdp->state;
       uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
       uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
-      requant_store<VCODE, true>(a, S, cc, e0, lane, kPerLane, hmask, m1, v1, den, mcw, vcw,
-                                 st.mscale + blk, st.vscale + blk);
+      requant_store<VCODE, true>(a, S, hdp->tensor_id, hdp->flags, hdp->e0, lane, kPerLane, hmask,
+                                 m1, v1, den, mcw, vcw, st.mscale + blk, st.vscale + blk);
     } else {
-      process_direct<VCODE>(a, S, st, cc, decay, u, lane, hmask);
-      if (issue(ui, s)) pend |= 1u << s;
-      ui += H;
+      process_direct<VCODE>(a, S, st, hdp, lane, hmask);
     }
-    s = (s + 1 == kStages) ? 0 : s + 1;
+    // every read of the stage (header included) is done: hand it back
+    fence_proxy_async_smem();
+    __syncwarp(hmask);
+    if (lane == 0) mbar_arrive(empty, 1);
+    if (++s == kStages) {
+      s = 0;
+      parity ^= 1u;
+    }
   }
 }
 
@@ -770,8 +854,12 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.omb2 = (float)(1.0 - (double)c.beta2);
   a.eps = c.eps;
   a.lr = lr;
-  a.key0 = (uint32_t)c.seed;
-  a.key1 = (uint32_t)(c.seed >> 32);
+  // Philox round keys: round r uses the seed words plus r times the Weyl
+  // constants (mod 2^32).
+  for (int r = 0; r < 10; ++r) {
+    a.rk0[r] = (uint32_t)c.seed + (uint32_t)r * kPhiloxW0;
+    a.rk1[r] = (uint32_t)(c.seed >> 32) + (uint32_t)r * kPhiloxW1;
+  }
   a.t_lo = (uint32_t)t;
   a.lm_sr_active = (c.total_steps > 0) && (10 * t > 9 * c.total_steps);
   a.status = nullptr;
@@ -845,7 +933,7 @@ int occupancy_grid(int device, int* grid) {
                            kSmemStages);
   if (e != cudaSuccess) return (int)e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adamw4_step_kernel<VCODE>,
-                                                    kThreads, kSmemStages);
+                                                    kCtaThreads, kSmemStages);
   if (e != cudaSuccess) return (int)e;
   *grid = sms * std::max(per_sm, 1);
   return 0;
@@ -859,11 +947,11 @@ int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
   a.fault_stall = h->fault_stall;
   h->fault_stall = 0;
   if (h->cfg.vcode == kVZip)
-    adamw4_step_kernel<kVZip><<<grid, kThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
-                                                                  h->tabs, h->st);
+    adamw4_step_kernel<kVZip><<<grid, kCtaThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
+                                                                     h->tabs, h->st);
   else
-    adamw4_step_kernel<kVZe><<<grid, kThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
-                                                                 h->tabs, h->st);
+    adamw4_step_kernel<kVZe><<<grid, kCtaThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
+                                                                    h->tabs, h->st);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(h, e, "step kernel launch");
   return ADAMW4_OK;
@@ -1238,7 +1326,7 @@ extern "C" int adamw4_launch_info(const adamw4_handle* h, int* grid, int* block,
   if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
   const int64_t need = (h->nunits + kHalves - 1) / kHalves;
   if (grid) *grid = (int)std::min<int64_t>(h->grid, need);
-  if (block) *block = kThreads;
+  if (block) *block = kCtaThreads;
   if (units) *units = h->nunits;
   return ADAMW4_OK;
 }
