@@ -18,6 +18,7 @@ __all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_T_NORM", "ADAMW4_T_LM_HE
            "adamw4_get_step", "adamw4_set_step", "adamw4_state_bytes", "adamw4_state_export",
            "adamw4_state_import", "adamw4_launch_info", "adamw4_last_error", "adamw4_sync",
            "adamw4_inject_fault", "ADAMW4_ETIMEOUT", "ADAMW4_FAULT_STALL_PIPELINE", "AdamW4",
+           "adamw4_state_buffers", "adamw4_step_noalloc", "ADAMW4_NOALLOC_MAX_TENSORS",
            "is_fp32_state", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libadamw4.so")
@@ -32,6 +33,7 @@ MIN_QUANT_NUMEL = 4096
 BLOCK = 128
 
 ADAMW4_ETIMEOUT = -7
+ADAMW4_NOALLOC_MAX_TENSORS = 1024
 ADAMW4_FAULT_STALL_PIPELINE = 1
 
 STATUS = {0: "ADAMW4_OK", -1: "ADAMW4_EINVAL", -2: "ADAMW4_EALIGN", -3: "ADAMW4_ENOMEM",
@@ -48,6 +50,13 @@ class adamw4_tensor(ctypes.Structure):
     _fields_ = [("param", ctypes.c_void_p), ("grad_bf16", ctypes.c_void_p),
                 ("numel", ctypes.c_int64), ("tensor_id", ctypes.c_uint32),
                 ("flags", ctypes.c_uint32), ("weight_decay", ctypes.c_float)]
+
+
+class adamw4_state_buffers(ctypes.Structure):
+    """Caller-owned device buffers of the packed state (allocation-free step)."""
+    _fields_ = [("mcodes", ctypes.c_void_p), ("vcodes", ctypes.c_void_p),
+                ("mscale", ctypes.c_void_p), ("vscale", ctypes.c_void_p),
+                ("m32", ctypes.c_void_p), ("v32", ctypes.c_void_p)]
 
 
 class adamw4_config(ctypes.Structure):
@@ -84,12 +93,15 @@ def lib() -> ctypes.CDLL:
                                          c.POINTER(c.c_int64)]
         L.adamw4_sync.argtypes = [H, c.c_void_p]
         L.adamw4_inject_fault.argtypes = [H, c.c_int]
+        L.adamw4_step_noalloc.argtypes = [c.POINTER(adamw4_config), c.POINTER(adamw4_tensor),
+                                          c.c_int, c.POINTER(adamw4_state_buffers), c.c_int64,
+                                          c.c_float, c.c_int, c.c_void_p]
         L.adamw4_last_error.argtypes = [H]
         L.adamw4_last_error.restype = c.c_char_p
         for f in ("adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
                   "adamw4_get_step", "adamw4_set_step", "adamw4_state_export",
                   "adamw4_state_import", "adamw4_launch_info", "adamw4_sync",
-                  "adamw4_inject_fault"):
+                  "adamw4_inject_fault", "adamw4_step_noalloc"):
             getattr(L, f).restype = c.c_int
         _lib = L
     return _lib
@@ -161,6 +173,17 @@ def adamw4_sync(h, stream=None):
 
 def adamw4_inject_fault(h, fault: int):
     _check(lib().adamw4_inject_fault(h, fault), h)
+
+
+def adamw4_step_noalloc(cfg: adamw4_config, tensors, state: adamw4_state_buffers, t: int,
+                        lr: float, device: int = 0, stream=None):
+    """The allocation-free step (see include/adamw4.h): no handle, caller-owned
+    state buffers, step number t.  Raises AdamW4Error with the status code."""
+    arr = (adamw4_tensor * max(len(tensors), 1))(*tensors)
+    rc = lib().adamw4_step_noalloc(ctypes.byref(cfg), arr, len(tensors), ctypes.byref(state), t,
+                                   lr, device, stream)
+    if rc != ADAMW4_OK:
+        raise AdamW4Error(rc, "adamw4_step_noalloc failed")
 
 
 def adamw4_launch_info(h):

@@ -1335,3 +1335,150 @@ extern "C" const char* adamw4_last_error(const adamw4_handle* h) {
   if (h != nullptr && live(h)) return h->err.c_str();
   return t_err.c_str();
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free step
+//
+// adamw4_step_noalloc runs the same step kernel without allocating device
+// memory.  The kernel's own scratch -- the per-tensor descriptor table it walks
+// and the status word its bounded waits report to -- lives in the file-scope
+// array below: kNoAllocScratchBytes (about 64.3 KB) on every GPU that loads
+// this library, held until the process exits.  The caller passes the inputs
+// and outputs (params, grads, and the packed state buffers).
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoAllocMaxTensors = ADAMW4_NOALLOC_MAX_TENSORS;
+constexpr size_t kNoAllocStatusBytes = 256;   // status word, padded to keep the table aligned
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocStatusBytes + sizeof(DevTensor) * (size_t)kNoAllocMaxTensors;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocDevice {
+  bool ready;
+  unsigned char* scratch;   // device address of g_noalloc_scratch on this device
+  int grid_zip, grid_ze;
+};
+
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+DevTensor g_noalloc_table[kNoAllocMaxTensors];   // host staging of the table
+
+bool na_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// The checks adamw4_create makes, written without containers so that nothing
+// is allocated (duplicate ids and overlaps by pairwise comparison).
+int na_validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n,
+                const adamw4_state_buffers* sb, int64_t t, float lr) {
+  if (cfg == nullptr || sb == nullptr) return ADAMW4_EINVAL;
+  if (!(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) || !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f))
+    return ADAMW4_EINVAL;
+  if (!(cfg->eps > 0.0f) || !std::isfinite(cfg->eps)) return ADAMW4_EINVAL;
+  if (cfg->vcode != ADAMW4_V_ZIPSR && cfg->vcode != ADAMW4_V_ZEEDEN) return ADAMW4_EINVAL;
+  if (cfg->total_steps < 0 || t < 1) return ADAMW4_EINVAL;
+  if (!(lr >= 0.0f) || !std::isfinite(lr)) return ADAMW4_EINVAL;
+  if (n < 0 || (n > 0 && ts == nullptr)) return ADAMW4_EINVAL;
+  if (n > kNoAllocMaxTensors) return ADAMW4_ERANGE;
+  if (!na_aligned(sb->mcodes, 16) || !na_aligned(sb->vcodes, 16) || !na_aligned(sb->mscale, 4) ||
+      !na_aligned(sb->vscale, 4) || !na_aligned(sb->m32, 16) || !na_aligned(sb->v32, 16))
+    return ADAMW4_EALIGN;
+  for (int i = 0; i < n; ++i) {
+    const adamw4_tensor& x = ts[i];
+    if (x.param == nullptr || x.grad_bf16 == nullptr || x.numel <= 0 ||
+        x.numel > ((int64_t)1 << 40) || !std::isfinite(x.weight_decay))
+      return ADAMW4_EINVAL;
+    if (!na_aligned(x.param, 16) || !na_aligned(x.grad_bf16, 16)) return ADAMW4_EALIGN;
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(x.param), p1 = p0 + (uintptr_t)x.numel * 4u;
+    const uintptr_t g0 = reinterpret_cast<uintptr_t>(x.grad_bf16), g1 = g0 + (uintptr_t)x.numel * 2u;
+    if (p0 < g1 && g0 < p1) return ADAMW4_EINVAL;                 // own grad
+    for (int k = 0; k < i; ++k) {
+      const adamw4_tensor& y = ts[k];
+      if (y.tensor_id == x.tensor_id) return ADAMW4_EINVAL;
+      const uintptr_t q0 = reinterpret_cast<uintptr_t>(y.param), q1 = q0 + (uintptr_t)y.numel * 4u;
+      const uintptr_t h0 = reinterpret_cast<uintptr_t>(y.grad_bf16), h1 = h0 + (uintptr_t)y.numel * 2u;
+      if ((p0 < q1 && q0 < p1) || (p0 < h1 && h0 < p1) || (q0 < g1 && g0 < q1))
+        return ADAMW4_EINVAL;                                     // a param overlaps
+    }
+  }
+  return ADAMW4_OK;
+}
+
+}  // namespace
+
+extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor* tensors, int n,
+                                   const adamw4_state_buffers* state, int64_t t, float lr,
+                                   int device, void* cuda_stream) {
+  const int rc = na_validate(cfg, tensors, n, state, t, lr);
+  if (rc != ADAMW4_OK) return rc;
+  if (device < 0 || device >= kNoAllocMaxDevices) return ADAMW4_EINVAL;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  DeviceGuard dg(device);
+  if (!dg.ok) return ADAMW4_ECUDA;
+  NoAllocDevice& nd = g_noalloc_dev[device];
+  if (!nd.ready) {
+    // Once per device, with that device current: the device address of the
+    // scratch array (its host-side name is only a stand-in), and the launch
+    // geometry.
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&nd.scratch), g_noalloc_scratch) !=
+        cudaSuccess)
+      return ADAMW4_ECUDA;
+    if (occupancy_grid<kVZip>(device, &nd.grid_zip) != 0 ||
+        occupancy_grid<kVZe>(device, &nd.grid_ze) != 0)
+      return ADAMW4_ECUDA;
+    nd.ready = true;
+  }
+  // The table adamw4_create would build, in the same order and layout.
+  int64_t unit = 0, blocks4 = 0, elems32 = 0;
+  for (int i = 0; i < n; ++i) {
+    const adamw4_tensor& x = tensors[i];
+    const bool fp32 = x.numel < ADAMW4_MIN_QUANT_NUMEL ||
+                      (x.flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE)) != 0;
+    const int64_t nb = (x.numel + kBlock - 1) / kBlock;
+    DevTensor& d = g_noalloc_table[i];
+    d.param = x.param;
+    d.grad = x.grad_bf16;
+    d.numel = x.numel;
+    d.unit_begin = unit;
+    d.unit_end = unit + nb;
+    d.state_off = fp32 ? elems32 : blocks4;
+    d.tensor_id = x.tensor_id;
+    d.flags = x.flags | (fp32 ? kKindFp32 : 0u);
+    d.weight_decay = x.weight_decay;
+    d.pad_ = 0;
+    if (fp32) elems32 += nb * kBlock; else blocks4 += nb;
+    unit += nb;
+  }
+  if (unit == 0) return ADAMW4_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(nd.scratch);
+  DevTensor* table = reinterpret_cast<DevTensor*>(nd.scratch + kNoAllocStatusBytes);
+  // The array keeps the previous call's contents: clear the status word and
+  // overwrite the table.  The copy is from pageable memory, so the staging
+  // buffer is free again when the call returns.
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return ADAMW4_ECUDA;
+  if (cudaMemcpyAsync(table, g_noalloc_table, sizeof(DevTensor) * (size_t)n,
+                      cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return ADAMW4_ECUDA;
+  CodeTables tabs;
+  build_tables(&tabs);
+  StepArgs a = make_args(*cfg, lr, t);
+  a.status = status;
+  a.fault_stall = 0;
+  StateArena st;
+  st.mcodes = state->mcodes;
+  st.vcodes = state->vcodes;
+  st.mscale = state->mscale;
+  st.vscale = state->vscale;
+  st.fm = state->m32;
+  st.fv = state->v32;
+  const int64_t need = (unit + kHalves - 1) / kHalves;
+  if (cfg->vcode == kVZip)
+    adamw4_step_kernel<kVZip><<<(int)std::min<int64_t>(nd.grid_zip, need), kCtaThreads,
+                                kSmemStages, s>>>(table, unit, a, tabs, st);
+  else
+    adamw4_step_kernel<kVZe><<<(int)std::min<int64_t>(nd.grid_ze, need), kCtaThreads,
+                               kSmemStages, s>>>(table, unit, a, tabs, st);
+  return cudaGetLastError() == cudaSuccess ? ADAMW4_OK : ADAMW4_ECUDA;
+}

@@ -197,6 +197,57 @@ int adamw4_state_import(adamw4_handle *h, const void *host_buf, int64_t len);
  * per block, and 128-value work units (4-bit blocks plus fp32 chunks). */
 int adamw4_launch_info(const adamw4_handle *h, int *grid, int *block, int64_t *units);
 
+/* ---------------------------------------------------------------------------
+ * Allocation-free step.  The paper has no counterpart: this entry point exists
+ * for callers that must not allocate device memory.  Examples are code running
+ * while a CUDA graph is being captured, where an allocation would be refused or
+ * frozen into the graph; programs whose device memory belongs to a pooling
+ * allocator or a fixed arena sized at start-up, which has to account for every
+ * byte; and tight training loops, where cudaMalloc and cudaFree can
+ * synchronise the device and stall other streams.
+ *
+ * It runs the same step as adamw4_step, without a handle.  The caller passes
+ * the tensors, the packed state buffers below, the step number t (1-based)
+ * and lr; nothing is allocated.  The step kernel's own scratch (its table of
+ * tensor descriptors and the status word of its bounded waits) lives in one
+ * static device array of 256 + 64 * ADAMW4_NOALLOC_MAX_TENSORS bytes (about
+ * 64 KB) that every GPU which loads this library holds until the process exits.
+ *   - More than ADAMW4_NOALLOC_MAX_TENSORS tensors: ADAMW4_ERANGE, nothing runs.
+ *   - Bad arguments: ADAMW4_EINVAL / ADAMW4_EALIGN, checked on the host first.
+ *     The status code is the whole report: this call records no message for
+ *     adamw4_last_error.
+ *   - The first call on a device looks up the array's device address and the
+ *     launch geometry for that device; make that first call before any stream
+ *     capture.
+ *   - All calls share the one array and each overwrites it: calls whose work
+ *     overlaps on the GPU (different streams, or different host threads without
+ *     ordering) race.  Calls on one stream are ordered and safe.
+ *   - A pipeline wait that runs out ends the kernel early like in adamw4_step;
+ *     this entry point has no handle to report it, so only launch errors are
+ *     returned (ADAMW4_ECUDA).
+ * Results equal adamw4_step's for the same inputs, state and t.
+ * ------------------------------------------------------------------------- */
+#define ADAMW4_NOALLOC_MAX_TENSORS 1024
+
+/* Packed optimizer state in caller-owned device memory, in the order of the
+ * tensor list.  4-bit tensors (see adamw4_create for the classification) own
+ * ceil(numel/128) consecutive blocks each; fp32-state tensors own consecutive
+ * ranges of m32/v32, each starting at a multiple of 128 elements.
+ *   mcodes, vcodes  64 bytes per block (element 2i in the low nibble of byte
+ *                   i), 16-byte aligned
+ *   mscale, vscale  one float per block, 4-byte aligned
+ *   m32, v32        floats, 16-byte aligned
+ * All-zero buffers are the initial state m = v = 0. */
+typedef struct {
+    uint8_t *mcodes, *vcodes;
+    float *mscale, *vscale;
+    float *m32, *v32;
+} adamw4_state_buffers;
+
+int adamw4_step_noalloc(const adamw4_config *cfg, const adamw4_tensor *tensors, int n,
+                        const adamw4_state_buffers *state, int64_t t, float lr, int device,
+                        void *cuda_stream);
+
 /* Message of the last failed call on this handle, or of the last failed call
  * on this thread when h is NULL.  Never NULL; valid until the next call. */
 const char *adamw4_last_error(const adamw4_handle *h);

@@ -1,0 +1,124 @@
+"""The allocation-free step, for callers that must not allocate device memory
+(code inside CUDA graph capture, programs whose memory belongs to a pooling
+allocator or a fixed arena, loops where cudaMalloc's device synchronisation is
+not acceptable).  It keeps the step kernel's scratch -- the descriptor table
+and the status word -- in a static device array instead of allocating it.
+
+Checked through the C ABI against the handle-based step: two calls in a row on
+the same inputs must give the same weights and packed state, within the
+tolerances the other parity tests use.  This file is collected last so that a
+run stopping at the first failure has already run every other test.
+"""
+import numpy as np
+import pytest
+
+import workloads
+from gpu_common import assert_state_equal, assert_weights_close, binding, parse_blob
+
+pytestmark = pytest.mark.gpu
+
+
+def _layout(ts):
+    """Byte sizes of the caller-owned state buffers, as the header describes."""
+    nb4, n32 = 0, 0
+    for t in ts:
+        nb = (t["numel"] + 127) // 128
+        if t["numel"] < 4096 or t["flags"] & (workloads.T_NORM | workloads.T_FP32_STATE):
+            n32 += nb * 128
+        else:
+            nb4 += nb
+    return nb4, n32
+
+
+def _blob_from_buffers(ts, bufs, t, vcode, seed):
+    """The checkpoint-layout view of caller-owned buffers (host copies)."""
+    import struct
+    mc, vc, ms, vs, m32, v32 = (b.cpu().numpy() for b in bufs)
+    parts, b4, e32 = [], 0, 0
+    for tt in ts:
+        n = tt["numel"]
+        nb = (n + 127) // 128
+        if n < 4096 or tt["flags"] & (workloads.T_NORM | workloads.T_FP32_STATE):
+            parts += [struct.pack("<IIq", tt["tensor_id"], 1, n), m32[e32:e32 + n].tobytes(),
+                      v32[e32:e32 + n].tobytes()]
+            e32 += nb * 128
+        else:
+            parts += [struct.pack("<IIq", tt["tensor_id"], 0, n),
+                      mc[b4 * 64:(b4 + nb) * 64].tobytes(), vc[b4 * 64:(b4 + nb) * 64].tobytes(),
+                      ms[b4:b4 + nb].tobytes(), vs[b4:b4 + nb].tobytes()]
+            b4 += nb
+    payload = b"".join(parts)
+    return b"ADAMW4S1" + struct.pack("<IIqQQ", len(ts), vcode, t, seed, len(payload)) + payload
+
+
+@pytest.mark.parametrize("vcode", [0, 1])
+def test_noalloc_step_matches_handle_step_twice(vcode):
+    import torch
+    B = binding()
+    ts = [dict(numel=65536, tensor_id=0, flags=0, weight_decay=0.1),
+          dict(numel=4096 + 37, tensor_id=4, flags=0, weight_decay=0.0),
+          dict(numel=3000, tensor_id=5, flags=0, weight_decay=0.1),
+          dict(numel=5000, tensor_id=6, flags=workloads.T_NORM, weight_decay=0.0),
+          dict(numel=128 * 40, tensor_id=7, flags=workloads.T_LM_HEAD, weight_decay=0.1)]
+    rng = np.random.default_rng(vcode)
+    w0 = [(rng.standard_normal(t["numel"]) * 0.02).astype(np.float32) for t in ts]
+    grads = [[workloads.bf16_bits((np.random.default_rng(10 * s + i).standard_normal(t["numel"])
+                                   * 1e-3).astype(np.float32)) for i, t in enumerate(ts)]
+             for s in (1, 2)]
+    seed, total = 77, 2
+    dev = torch.device("cuda", 0)
+
+    # handle-based step, twice
+    params = [torch.from_numpy(w.copy()).to(dev) for w in w0]
+    gbuf = [torch.zeros(t["numel"], dtype=torch.bfloat16, device=dev) for t in ts]
+    opt = B.AdamW4(params, gbuf, ts, vcode=vcode, seed=seed, total_steps=total)
+    for gs in grads:
+        for g, hg in zip(gbuf, gs):
+            g.view(torch.int16).copy_(torch.from_numpy(hg.view(np.int16)))
+        opt.step()
+    torch.cuda.synchronize()
+    ref_w = [p.cpu().numpy() for p in params]
+    ref_blob = opt.state_dict_blob()
+    opt.close()
+
+    # allocation-free step, twice, on buffers this test owns
+    params2 = [torch.from_numpy(w.copy()).to(dev) for w in w0]
+    gbuf2 = [torch.zeros(t["numel"], dtype=torch.bfloat16, device=dev) for t in ts]
+    nb4, n32 = _layout(ts)
+    bufs = [torch.zeros(nb4 * 64, dtype=torch.uint8, device=dev),
+            torch.zeros(nb4 * 64, dtype=torch.uint8, device=dev),
+            torch.zeros(max(nb4, 1), dtype=torch.float32, device=dev),
+            torch.zeros(max(nb4, 1), dtype=torch.float32, device=dev),
+            torch.zeros(max(n32, 4), dtype=torch.float32, device=dev),
+            torch.zeros(max(n32, 4), dtype=torch.float32, device=dev)]
+    sb = B.adamw4_state_buffers(*[b.data_ptr() for b in bufs])
+    cfg = B.adamw4_config(1e-3, 0.9, 0.999, 1e-8, vcode, seed, total)
+    descs = [B.adamw4_tensor(p.data_ptr(), g.data_ptr(), t["numel"], t["tensor_id"], t["flags"],
+                             t["weight_decay"]) for p, g, t in zip(params2, gbuf2, ts)]
+    stream = torch.cuda.current_stream().cuda_stream
+    for step, gs in enumerate(grads, start=1):
+        for g, hg in zip(gbuf2, gs):
+            g.view(torch.int16).copy_(torch.from_numpy(hg.view(np.int16)))
+        B.adamw4_step_noalloc(cfg, descs, sb, step, 1e-3, 0, stream)
+        torch.cuda.synchronize()
+        # after each call the weights follow the same arithmetic as the handle path
+        assert all(np.isfinite(p.cpu().numpy()).all() for p in params2)
+    for i, p in enumerate(params2):
+        assert_weights_close(p.cpu().numpy(), ref_w[i], w0[i], f"noalloc tensor {i}")
+    got_blob = _blob_from_buffers(ts, bufs, 2, vcode, seed)
+    assert_state_equal(got_blob, ref_blob, vcode, "noalloc")
+
+
+def test_noalloc_rejects_too_many_tensors():
+    import torch
+    B = binding()
+    n = B.ADAMW4_NOALLOC_MAX_TENSORS + 1
+    base = torch.zeros(16 * n, dtype=torch.float32, device="cuda")
+    gb = torch.zeros(16 * n, dtype=torch.bfloat16, device="cuda")
+    descs = [B.adamw4_tensor(base.data_ptr() + 64 * i, gb.data_ptr() + 32 * i, 16, i, 0, 0.0)
+             for i in range(n)]
+    sb = B.adamw4_state_buffers(0, 0, 0, 0, base.data_ptr(), base.data_ptr())
+    cfg = B.adamw4_config(1e-3, 0.9, 0.999, 1e-8, 0, 0, 0)
+    with pytest.raises(B.AdamW4Error) as err:
+        B.adamw4_step_noalloc(cfg, descs, sb, 1, 1e-3, 0, None)
+    assert err.value.code == -6
