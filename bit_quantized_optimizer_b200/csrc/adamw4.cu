@@ -64,19 +64,27 @@ constexpr int kConsumerThreads = 256;             // eight consumer warps
 constexpr int kCtaThreads = kConsumerThreads + 32;  // plus the producer warp
 constexpr int kHalves = kConsumerThreads / kLanesPerUnit;  // consumer half-warps per CTA
 constexpr int kProducerWarp = kConsumerThreads / 32;
-constexpr int kStages = 4;                        // units in flight per half-warp
-// Stage layout: header 64 B | w 512 B | g 256 B | m codes 64 B | v codes 64 B |
-// m scale 4 B | v scale 4 B
-constexpr int kOffHdr = 0, kOffW = 64, kOffG = 576, kOffMC = 832, kOffVC = 896, kOffMS = 960,
-              kOffVS = 964;
-constexpr int kStageBytes = 976;                  // 16-byte multiple
-constexpr uint32_t kStageTx = 896;                // bytes delivered by the bulk copies
-constexpr int kSmemStages = kHalves * kStages * kStageBytes;
+constexpr int kStages = 4;                        // tiles in flight per CTA
+// A tile is kHalves consecutive units; stage layout (CTA-wide):
+//   16 unit headers (64 B each) | w 16 x 512 B | g 16 x 256 B |
+//   m codes 16 x 64 B | v codes 16 x 64 B | m scales 16 x 4 B | v scales 16 x 4 B
+constexpr int kOffHdr = 0;
+constexpr int kOffW = kOffHdr + kHalves * 64;
+constexpr int kOffG = kOffW + kHalves * 512;
+constexpr int kOffMC = kOffG + kHalves * 256;
+constexpr int kOffVC = kOffMC + kHalves * 64;
+constexpr int kOffMS = kOffVC + kHalves * 64;
+constexpr int kOffVS = kOffMS + kHalves * 4;
+constexpr int kStageBytes = kOffVS + kHalves * 4; // 15,488 B, a 16-byte multiple
+constexpr uint32_t kUnitTx = 896;                 // bulk-copied bytes of one whole block
+constexpr int kSmemStages = kStages * kStageBytes;
+static_assert(kStageBytes % 16 == 0, "stage alignment");
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr int kVZip = ADAMW4_V_ZIPSR;
 constexpr int kVZe = ADAMW4_V_ZEEDEN;
 constexpr uint32_t kKindFp32 = 1u << 16;          // internal flag: fp32-state tensor
 constexpr uint32_t kStaged = 1u << 17;            // internal flag: unit data is in the stage
+constexpr uint32_t kNoUnit = 1u << 18;            // internal flag: empty slot of the last tile
 constexpr uint32_t kStreamV = 0u;                 // Philox stream of the v draw
 constexpr uint32_t kStreamM = 1u;                 // Philox stream of the LM-head m draw
 constexpr float kMagic = 12582912.0f;             // 1.5 * 2^23: adding it rounds to an integer
@@ -527,46 +535,34 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
 }
 
 // ---------------------------------------------------------------------------
-// Producer: lane j fills the stage ring of consumer half-warp j.
+// Producer: fills CTA-wide stages, one tile of kHalves consecutive units each.
+// Lane i handles unit i of the tile (header, scales); the lane that starts a
+// run of whole 4-bit blocks of one tensor issues that run's bulk copies.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t nunits,
                                         const StepArgs& a, const StateArena& st, uint8_t* stages,
-                                        uint32_t full0, uint32_t empty0, int j) {
-  const int64_t H = (int64_t)gridDim.x * kHalves;
+                                        uint32_t full0, uint32_t empty0, int lane) {
+  constexpr unsigned kMask = (1u << kHalves) - 1u;
+  const int64_t ntiles = (nunits + kHalves - 1) / kHalves;
   int ti = -1;
   int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0;
   float* t_param = nullptr;
   const uint16_t* t_grad = nullptr;
   uint32_t t_id = 0, t_flags = 0;
   float t_decay = 1.0f;
-  uint8_t* my = stages + j * (kStages * kStageBytes);
-  const uint32_t my_s = smem_addr(my);
+  const uint32_t stages_s = smem_addr(stages);
   int s = 0;
-  uint32_t round = 0;     // completed passes over the ring
-  uint64_t stalled_since = 0;
-  // Each lane refills its own ring as soon as its consumer hands a stage back,
-  // independently of the other lanes; the warp naps only when no lane could
-  // make progress.
-  for (int64_t u = (int64_t)blockIdx.x * kHalves + j; u < nunits;) {
-    const uint32_t full = full0 + 8u * (j * kStages + s);
-    const bool ready =
-        round == 0 || mbar_test_wait(empty0 + 8u * (j * kStages + s), (round - 1) & 1u);
-    const bool any_ready = __any_sync(__activemask(), ready);
-    if (!ready) {
-      const uint64_t now = global_ns();
-      if (stalled_since == 0) {
-        stalled_since = now;
-      } else if (now - stalled_since > kWaitLimitNs) {
-        atomicOr(a.status, 1u);
-        break;
-      }
-      // consumers spend microseconds per unit: when no stage is free, nap
-      // instead of taking issue slots from them
-      if (!any_ready) __nanosleep(1000);
-      continue;
+  uint32_t round = 0;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const uint32_t full = full0 + 8u * s;
+    if (round > 0 && !__all_sync(kMask, wait_phase(empty0 + 8u * s, (round - 1) & 1u,
+                                                   kWaitLimitNs))) {
+      if (lane == 0) atomicOr(a.status, 1u);
+      return;
     }
-    stalled_since = 0;
-    if (u >= t_end) {
+    const int64_t u = tile * kHalves + lane;
+    const bool has = u < nunits;
+    if (has && u >= t_end) {
       do {
         ++ti;
         t_end = __ldg(&T[ti].unit_end);
@@ -583,39 +579,51 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     }
     const int64_t ub = u - t_begin;
     const int64_t e0 = ub * kBlock;
-    const int nvalid = (int)min((int64_t)kBlock, t_numel - e0);
-    const bool staged = !(t_flags & kKindFp32) && nvalid == kBlock;
-    UnitHeader* hd = reinterpret_cast<UnitHeader*>(my + s * kStageBytes + kOffHdr);
+    const int nvalid = has ? (int)min((int64_t)kBlock, t_numel - e0) : 0;
+    const bool staged = has && !(t_flags & kKindFp32) && nvalid == kBlock;
+    uint8_t* sp = stages + s * kStageBytes;
+    UnitHeader* hd = reinterpret_cast<UnitHeader*>(sp + kOffHdr) + lane;
     hd->w = t_param + e0;
     hd->g = t_grad + e0;
     hd->e0 = (uint64_t)e0;
     hd->state = (t_flags & kKindFp32) ? (uint64_t)(t_soff + e0) : (uint64_t)(t_soff + ub);
     hd->tensor_id = t_id;
-    hd->flags = t_flags | (staged ? kStaged : 0u);
+    hd->flags = has ? (t_flags | (staged ? kStaged : 0u)) : kNoUnit;
     hd->decay = t_decay;
     hd->nvalid = nvalid;
-    if (staged && !a.fault_stall) {
-      const uint32_t dst = my_s + (uint32_t)(s * kStageBytes);
+    // Runs of whole blocks of one tensor are contiguous in global memory and
+    // in the stage: one bulk copy per array per run.
+    const unsigned staged_mask = __ballot_sync(kMask, staged);
+    const int prev_ti = __shfl_up_sync(kMask, ti, 1);
+    const bool cont = staged && lane > 0 && ((staged_mask >> (lane - 1)) & 1u) && prev_ti == ti;
+    const unsigned cont_mask = __ballot_sync(kMask, cont);
+    const uint32_t dst = stages_s + (uint32_t)(s * kStageBytes);
+    if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)__popc(staged_mask) * kUnitTx);
+    if (staged && !cont && !a.fault_stall) {
+      // this lane starts a run: it extends over the following lanes whose
+      // unit continues it
+      const unsigned rest = ~(cont_mask >> (lane + 1));
+      const int len = __ffs(rest);          // 1 + number of continuing lanes
       const int64_t blk = t_soff + ub;
-      mbar_arrive_expect_tx(full, kStageTx);
-      bulk_g2s(dst + kOffW, t_param + e0, 512, full);
-      bulk_g2s(dst + kOffG, t_grad + e0, 256, full);
-      bulk_g2s(dst + kOffMC, st.mcodes + blk * (kBlock / 2), 64, full);
-      bulk_g2s(dst + kOffVC, st.vcodes + blk * (kBlock / 2), 64, full);
-      cp_async4(dst + kOffMS, st.mscale + blk);
-      cp_async4(dst + kOffVS, st.vscale + blk);
-      cp_async_arrive_noinc(full);
-    } else if (!staged) {
-      mbar_arrive(full, 2);          // header only: complete the phase now
+      bulk_g2s(dst + kOffW + lane * 512, t_param + e0, 512u * len, full);
+      bulk_g2s(dst + kOffG + lane * 256, t_grad + e0, 256u * len, full);
+      bulk_g2s(dst + kOffMC + lane * 64, st.mcodes + blk * (kBlock / 2), 64u * len, full);
+      bulk_g2s(dst + kOffVC + lane * 64, st.vcodes + blk * (kBlock / 2), 64u * len, full);
     }
-    // (test hook: a staged unit with the stall armed never completes)
-    u += H;
+    if (staged && !a.fault_stall) {
+      const int64_t blk = t_soff + ub;
+      cp_async4(dst + kOffMS + lane * 4, st.mscale + blk);
+      cp_async4(dst + kOffVS + lane * 4, st.vscale + blk);
+    }
+    cp_async_arrive_noinc(full);            // one arrival per lane, when its copies land
+    // (test hook: with the stall armed no bulk copy is issued, so the expected
+    // bytes never arrive and the consumers' waits run out)
     if (++s == kStages) {
       s = 0;
       ++round;
     }
   }
-  cp_async_wait_all();               // this thread's 4-byte copies have landed
+  cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -627,8 +635,8 @@ __global__ void __launch_bounds__(kCtaThreads, 3)
 adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, CodeTables tabs,
                    StateArena st) {
   extern __shared__ __align__(128) uint8_t s_stage[];
-  __shared__ __align__(8) uint64_t s_full[kHalves * kStages];
-  __shared__ __align__(8) uint64_t s_empty[kHalves * kStages];
+  __shared__ __align__(8) uint64_t s_full[kStages];
+  __shared__ __align__(8) uint64_t s_empty[kStages];
   __shared__ SmemTables S;
 
   {
@@ -647,9 +655,11 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
       S.sqp[t] = make_float2(tabs.vz_sqrt[t], tabs.vz_sqrt[min(t + 1, 15)]);
       S.vzp[t] = make_float2(tabs.vz[t], tabs.vz[min(t + 1, 15)]);
     }
-    if (t < kHalves * kStages) {
-      mbar_init(smem_addr(&s_full[t]), 2);    // producer arrive + the scales' cp.async arrive
-      mbar_init(smem_addr(&s_empty[t]), 1);   // the consumer half-warp's release
+    if (t < kStages) {
+      // full: the producer's expect-tx arrive plus one cp.async arrive per
+      // producer lane; empty: one release per consumer half-warp
+      mbar_init(smem_addr(&s_full[t]), 1 + kHalves);
+      mbar_init(smem_addr(&s_empty[t]), kHalves);
     }
     fence_mbar_init();
   }
@@ -659,43 +669,44 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
   const uint32_t empty0 = smem_addr(&s_empty[0]);
   const int warp = threadIdx.x >> 5;
   if (warp == kProducerWarp) {
-    const int j = threadIdx.x & 31;
-    if (j < kHalves) produce(T, nunits, a, st, s_stage, full0, empty0, j);
+    const int lane = threadIdx.x & 31;
+    if (lane < kHalves) produce(T, nunits, a, st, s_stage, full0, empty0, lane);
     return;
   }
 
-  // ---- consumers ----
+  // ---- consumers: half-warp `half` takes unit `half` of every tile ----
   const int lane = threadIdx.x & 15;
   const int half = threadIdx.x >> 4;
   const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
-  const int64_t H = (int64_t)gridDim.x * kHalves;
-  const uint8_t* ring = s_stage + half * (kStages * kStageBytes);
+  const int64_t ntiles = (nunits + kHalves - 1) / kHalves;
   int s = 0;
   uint32_t parity = 0;
-  for (int64_t u = (int64_t)blockIdx.x * kHalves + half; u < nunits; u += H) {
-    const uint32_t full = full0 + 8u * (half * kStages + s);
-    const uint32_t empty = empty0 + 8u * (half * kStages + s);
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const uint32_t full = full0 + 8u * s;
+    const uint32_t empty = empty0 + 8u * s;
     if (!__all_sync(hmask, wait_phase(full, parity, kWaitLimitNs))) {
       if (lane == 0) atomicOr(a.status, 1u);
       return;
     }
-    const uint8_t* sp = ring + s * kStageBytes;
-    const UnitHeader* hdp = reinterpret_cast<const UnitHeader*>(sp + kOffHdr);
-    if (hdp->flags & kStaged) {
+    const uint8_t* sp = s_stage + s * kStageBytes;
+    const UnitHeader* hdp = reinterpret_cast<const UnitHeader*>(sp + kOffHdr) + half;
+    const uint32_t flags = hdp->flags;
+    if (flags & kStaged) {
       float w[kPerLane], g[kPerLane];
       {
-        const float4 wa = *reinterpret_cast<const float4*>(sp + kOffW + lane * 32);
-        const float4 wb = *reinterpret_cast<const float4*>(sp + kOffW + lane * 32 + 16);
-        const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + lane * 16);
+        const uint8_t* wsrc = sp + kOffW + half * 512 + lane * 32;
+        const float4 wa = *reinterpret_cast<const float4*>(wsrc);
+        const float4 wb = *reinterpret_cast<const float4*>(wsrc + 16);
+        const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
         w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
         w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
         g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
         g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
       }
-      const uint32_t mc = *reinterpret_cast<const uint32_t*>(sp + kOffMC + lane * 4);
-      const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + lane * 4);
-      const float sm = *reinterpret_cast<const float*>(sp + kOffMS);
-      const float sv = *reinterpret_cast<const float*>(sp + kOffVS);
+      const uint32_t mc = *reinterpret_cast<const uint32_t*>(sp + kOffMC + half * 64 + lane * 4);
+      const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + half * 64 + lane * 4);
+      const float sm = *reinterpret_cast<const float*>(sp + kOffMS + half * 4);
+      const float sv = *reinterpret_cast<const float*>(sp + kOffVS + half * 4);
 
       float m1[kPerLane], v1[kPerLane], den[kPerLane];
       update8(a, S, hdp->decay, w, g, mc, vc, sm, sv, m1, v1, den);
@@ -705,9 +716,9 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
       const uint64_t blk = hdp->state;
       uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
       uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
-      requant_store<VCODE, true>(a, S, hdp->tensor_id, hdp->flags, hdp->e0, lane, kPerLane, hmask,
-                                 m1, v1, den, mcw, vcw, st.mscale + blk, st.vscale + blk);
-    } else {
+      requant_store<VCODE, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, kPerLane, hmask, m1,
+                                 v1, den, mcw, vcw, st.mscale + blk, st.vscale + blk);
+    } else if (!(flags & kNoUnit)) {
       process_direct<VCODE>(a, S, st, hdp, lane, hmask);
     }
     // every read of the stage (header included) is done: hand it back
