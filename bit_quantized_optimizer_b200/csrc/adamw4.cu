@@ -237,6 +237,20 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// The producer's wait for a stage to come back: the consumers take
+// microseconds per tile, so it naps between polls instead of taking issue
+// slots from them.  False if `limit_ns` passed first.
+__device__ __forceinline__ bool wait_phase_napping(uint32_t bar, uint32_t parity,
+                                                   uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    __nanosleep(256);
+    if (mbar_test_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Arithmetic helpers
 // ---------------------------------------------------------------------------
@@ -314,7 +328,8 @@ struct SmemTables {
   float nf4[16];
   float gap[16];
   float vz[16];        // ZIP-SR code points k/15
-  float2 sqp[16];      // {sqrt(k/15), sqrt((k+1)/15)}
+  float4 zip[16];      // for k0 = nearest integer to 15x: {VZ[k0] (+inf for 15),
+                       //   sqrt VZ[k0-1], sqrt VZ[k0], sqrt VZ[k0+1]}
   float2 vzp[16];      // {k/15, (k+1)/15}
 };
 
@@ -332,28 +347,34 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
                                                  const float (&den)[kPerLane],
                                                  const float (&ud)[kPerLane], float inv, float R,
                                                  int myn) {
+  // elements from the last to the first, so that element i ends in bits 4i..4i+3
   uint32_t vco = 0;
 #pragma unroll
-  for (int j = 0; j < kPerLane / 2; ++j) {
+  for (int j = kPerLane / 2 - 1; j >= 0; --j) {
     const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
     const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 1; h >= 0; --h) {
       const int i = 2 * j + h;
       const float x = h ? x2.y : x2.x;
-      // the nearest integer to 15x is the bracket or one above it
-      int k = (int)(__float_as_uint(h ? t2.y : t2.x) & 31u);
-      k -= (x < S.vz[k]) ? 1 : 0;
-      k = min(k, 14);
-      const float2 dd = __ffma2_rn(S.sqp[k], f2(R), f2(a.eps));               // (da, db)
-      const float2 ad = __fadd2_rn(f2(dd.y), make_float2(-dd.x, -den[i]));   // (db-da, db-dv)
-      const float2 pr = __fmul2_rn(ad, make_float2(den[i], dd.x));           // (.*dv, .*da)
-      bool lower = __fmul_rn(ud[i], pr.x) < pr.y;
-      if (FLAT && dd.x == dd.y) {
+      // k0, the nearest integer to 15x, is the bracket or one above it (the
+      // top entry's threshold is +inf: its bracket is always 14)
+      const uint32_t k0 = __float_as_uint(h ? t2.y : t2.x) & 15u;
+      const float4 e = S.zip[k0];
+      const bool dec = x < e.x;
+      const float sa = dec ? e.y : e.z;            // sqrt of the lower code point
+      const float sb = dec ? e.z : e.w;            // and of the upper one
+      const float da = __fmaf_rn(sa, R, a.eps);
+      const float db = __fmaf_rn(sb, R, a.eps);
+      const float lhs = __fmul_rn(ud[i], __fmul_rn(__fsub_rn(db, da), den[i]));
+      const float rhs = __fmul_rn(__fsub_rn(db, den[i]), da);
+      bool lower = lhs < rhs;
+      const uint32_t k = k0 - (dec ? 1u : 0u);
+      if (FLAT && da == db) {
         const float2 z = S.vzp[k];
         lower = __fmul_rn(ud[i], __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
       }
-      if (FULL || i < myn) vco |= (uint32_t)(k + (lower ? 0 : 1)) << (4 * i);
+      vco = vco * 16u + ((FULL || i < myn) ? k + (lower ? 0u : 1u) : 0u);
     }
   }
   return vco;
@@ -391,13 +412,12 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
         if (FULL || i < myn) mco |= nf4_sr(__fmul_rn(m1[i], inv), ud[i], S.nf4, S.gap) << (4 * i);
     } else {
 #pragma unroll
-      for (int j = 0; j < kPerLane / 2; ++j) {
+      for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
         const float2 x = __fmul2_rn(make_float2(m1[2 * j], m1[2 * j + 1]), f2(inv));
         const float2 b = __ffma2_rn(x, f2(32.0f), f2(kMagic + 32.0f));
-        const uint32_t c0 = nf4_rtn_bucket(x.x, b.x, S.rtn);
-        const uint32_t c1 = nf4_rtn_bucket(x.y, b.y, S.rtn);
-        if (FULL || 2 * j < myn) mco |= c0 << (8 * j);
-        if (FULL || 2 * j + 1 < myn) mco |= c1 << (8 * j + 4);
+        const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? nf4_rtn_bucket(x.y, b.y, S.rtn) : 0u;
+        const uint32_t c0 = (FULL || 2 * j < myn) ? nf4_rtn_bucket(x.x, b.x, S.rtn) : 0u;
+        mco = (mco * 16u + c1) * 16u + c0;
       }
     }
     mso = am;
@@ -555,8 +575,8 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
   uint32_t round = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const uint32_t full = full0 + 8u * s;
-    if (round > 0 && !__all_sync(kMask, wait_phase(empty0 + 8u * s, (round - 1) & 1u,
-                                                   kWaitLimitNs))) {
+    if (round > 0 && !__all_sync(kMask, wait_phase_napping(empty0 + 8u * s, (round - 1) & 1u,
+                                                           kWaitLimitNs))) {
       if (lane == 0) atomicOr(a.status, 1u);
       return;
     }
@@ -652,7 +672,8 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
       S.nf4[t] = tabs.nf4[t];
       S.gap[t] = tabs.nf4_gap[t];
       S.vz[t] = tabs.vz[t];
-      S.sqp[t] = make_float2(tabs.vz_sqrt[t], tabs.vz_sqrt[min(t + 1, 15)]);
+      S.zip[t] = make_float4(t == 15 ? INFINITY : tabs.vz[t], tabs.vz_sqrt[max(t - 1, 0)],
+                             tabs.vz_sqrt[t], tabs.vz_sqrt[min(t + 1, 15)]);
       S.vzp[t] = make_float2(tabs.vz[t], tabs.vz[min(t + 1, 15)]);
     }
     if (t < kStages) {
