@@ -160,13 +160,22 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws):
+    """The maximum of a per-rank number (a device-timed duration) over all
+    ranks; NCCL reduces a CUDA tensor, gloo a CPU one."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(world_size, params_per_rank, max_ms_per_step):
+    """Whole-job throughput in Gparams/s: every rank steps its own replica of
+    the workload, and the job takes as long as the slowest rank."""
+    return world_size * params_per_rank / (max_ms_per_step * 1e-3) / 1e9
 
 
 def cpu_baseline(ts, params, grads, vcode, target_s=10.0, per_tensor_cap=1 << 18):
@@ -330,7 +339,7 @@ def run_ours(args):
         ms_per_step = total_ms / args.steps
         line = {
             "metric": METRIC,
-            "value": ws_ * nparams / (ms_per_step * 1e-3) / 1e9,
+            "value": weak_scaling_value(ws_, nparams, ms_per_step),
             "unit": "Gparams/s",
             "n_gpus": ws_,
             "steps": args.steps,

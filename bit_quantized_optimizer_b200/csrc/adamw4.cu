@@ -266,20 +266,23 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, const StepArgs& a) {
   return c;
 }
 
-// Uniform in [0,1): the top 23 bits of a word times 2^-23 (exact).
-__device__ __forceinline__ float uniform23(uint32_t w) {
-  return __fsub_rn(__uint_as_float((w >> 9) | 0x3F800000u), 1.0f);
+// 1 + u for the draw u in [0,1): the low 23 bits of a word as the mantissa of
+// a number in [1, 2).  u = (1 + u) - 1 is exact; u * B rounds like
+// fma(1 + u, B, -B).
+__device__ __forceinline__ float one_plus_u(uint32_t w) {
+  return __uint_as_float((w | 0x3F800000u) & 0x3FFFFFFFu);
 }
+__device__ __forceinline__ float uniform23(uint32_t w) { return __fsub_rn(one_plus_u(w), 1.0f); }
 
-// The eight draws of one lane: elements 4*quad .. 4*quad + 7.
-__device__ __forceinline__ void draws8(const StepArgs& a, uint32_t tensor_id, uint32_t stream,
-                                       uint64_t quad, float u[8]) {
+// The eight draw words of one lane: elements 4*quad .. 4*quad + 7.
+__device__ __forceinline__ void words8(const StepArgs& a, uint32_t tensor_id, uint32_t stream,
+                                       uint64_t quad, uint32_t r[8]) {
   const uint32_t c3 = tensor_id * 2u + stream;
   const uint4 r0 = philox4x32_10(make_uint4((uint32_t)quad, (uint32_t)(quad >> 32), a.t_lo, c3), a);
   const uint64_t q1 = quad + 1;
   const uint4 r1 = philox4x32_10(make_uint4((uint32_t)q1, (uint32_t)(q1 >> 32), a.t_lo, c3), a);
-  u[0] = uniform23(r0.x); u[1] = uniform23(r0.y); u[2] = uniform23(r0.z); u[3] = uniform23(r0.w);
-  u[4] = uniform23(r1.x); u[5] = uniform23(r1.y); u[6] = uniform23(r1.z); u[7] = uniform23(r1.w);
+  r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w;
+  r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }
@@ -345,37 +348,46 @@ template <bool FULL, bool FLAT>
 __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
                                                  const float (&v1)[kPerLane],
                                                  const float (&den)[kPerLane],
-                                                 const float (&ud)[kPerLane], float inv, float R,
-                                                 int myn) {
-  // elements from the last to the first, so that element i ends in bits 4i..4i+3
+                                                 const uint32_t (&rw)[kPerLane], float inv,
+                                                 float R, int myn) {
+  // two values at a time; from the last pair to the first, so that element i
+  // ends in bits 4i..4i+3
   uint32_t vco = 0;
 #pragma unroll
   for (int j = kPerLane / 2 - 1; j >= 0; --j) {
     const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
     const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
-#pragma unroll
-    for (int h = 1; h >= 0; --h) {
-      const int i = 2 * j + h;
-      const float x = h ? x2.y : x2.x;
-      // k0, the nearest integer to 15x, is the bracket or one above it (the
-      // top entry's threshold is +inf: its bracket is always 14)
-      const uint32_t k0 = __float_as_uint(h ? t2.y : t2.x) & 15u;
-      const float4 e = S.zip[k0];
-      const bool dec = x < e.x;
-      const float sa = dec ? e.y : e.z;            // sqrt of the lower code point
-      const float sb = dec ? e.z : e.w;            // and of the upper one
-      const float da = __fmaf_rn(sa, R, a.eps);
-      const float db = __fmaf_rn(sb, R, a.eps);
-      const float lhs = __fmul_rn(ud[i], __fmul_rn(__fsub_rn(db, da), den[i]));
-      const float rhs = __fmul_rn(__fsub_rn(db, den[i]), da);
-      bool lower = lhs < rhs;
-      const uint32_t k = k0 - (dec ? 1u : 0u);
-      if (FLAT && da == db) {
-        const float2 z = S.vzp[k];
-        lower = __fmul_rn(ud[i], __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
+    // k0, the nearest integer to 15x, is the bracket or one above it (the top
+    // entry's threshold is +inf: its bracket is always 14)
+    const uint32_t k0a = __float_as_uint(t2.x) & 15u, k0b = __float_as_uint(t2.y) & 15u;
+    const float4 ea = S.zip[k0a], eb = S.zip[k0b];
+    const bool deca = x2.x < ea.x, decb = x2.y < eb.x;
+    // square roots of the lower and upper code points of each value
+    const float2 sa = make_float2(deca ? ea.y : ea.z, decb ? eb.y : eb.z);
+    const float2 sb = make_float2(deca ? ea.z : ea.w, decb ? eb.z : eb.w);
+    const float2 da = __ffma2_rn(sa, f2(R), f2(a.eps));
+    const float2 db = __ffma2_rn(sb, f2(R), f2(a.eps));
+    const float2 dv = make_float2(den[2 * j], den[2 * j + 1]);
+    // fma(y, -1, x) rounds like x - y
+    const float2 B = __fmul2_rn(__ffma2_rn(da, f2(-1.0f), db), dv);      // (db - da) * dv
+    const float2 rhs = __fmul2_rn(__ffma2_rn(dv, f2(-1.0f), db), da);    // (db - dv) * da
+    const float2 f = make_float2(one_plus_u(rw[2 * j]), one_plus_u(rw[2 * j + 1]));
+    const float2 lhs = __ffma2_rn(f, B, make_float2(-B.x, -B.y));         // u * B
+    bool lowa = lhs.x < rhs.x, lowb = lhs.y < rhs.y;
+    const uint32_t ka = k0a - (deca ? 1u : 0u), kb = k0b - (decb ? 1u : 0u);
+    if (FLAT) {
+      if (da.x == db.x) {
+        const float2 z = S.vzp[ka];
+        lowa = __fmul_rn(__fsub_rn(f.x, 1.0f), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.x);
       }
-      vco = vco * 16u + ((FULL || i < myn) ? k + (lower ? 0u : 1u) : 0u);
+      if (da.y == db.y) {
+        const float2 z = S.vzp[kb];
+        lowb = __fmul_rn(__fsub_rn(f.y, 1.0f), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.y);
+      }
     }
+    const uint32_t ca = (FULL || 2 * j < myn) ? ka + (lowa ? 0u : 1u) : 0u;
+    const uint32_t cb = (FULL || 2 * j + 1 < myn) ? kb + (lowb ? 0u : 1u) : 0u;
+    vco = (vco * 16u + cb) * 16u + ca;
   }
   return vco;
 }
@@ -405,11 +417,12 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   if (am >= FLT_MIN) {
     const float inv = __fdiv_rn(1.0f, am);
     if ((flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
-      float ud[kPerLane];
-      draws8(a, tensor_id, kStreamM, (e0 + (uint64_t)(lane * kPerLane)) >> 2, ud);
+      uint32_t rw[kPerLane];
+      words8(a, tensor_id, kStreamM, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
 #pragma unroll
       for (int i = 0; i < kPerLane; ++i)
-        if (FULL || i < myn) mco |= nf4_sr(__fmul_rn(m1[i], inv), ud[i], S.nf4, S.gap) << (4 * i);
+        if (FULL || i < myn)
+          mco |= nf4_sr(__fmul_rn(m1[i], inv), uniform23(rw[i]), S.nf4, S.gap) << (4 * i);
     } else {
 #pragma unroll
       for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
@@ -433,14 +446,14 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
       // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
       const float R = __fmul_rn(__fsqrt_rn(av), a.rs_bc2);
-      float ud[kPerLane];
-      draws8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, ud);
+      uint32_t rw[kPerLane];
+      words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
       // d(a) == d(b) needs (sqrt(k+1/15) - sqrt(k/15)) R below two ulps of
       // R + eps; the smallest gap is 0.0339, so R > 1e-5 eps rules it out.
       if (R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN)
-        vco = zipsr_codes8<FULL, false>(a, S, v1, den, ud, inv, R, myn);
+        vco = zipsr_codes8<FULL, false>(a, S, v1, den, rw, inv, R, myn);
       else
-        vco = zipsr_codes8<FULL, true>(a, S, v1, den, ud, inv, R, myn);
+        vco = zipsr_codes8<FULL, true>(a, S, v1, den, rw, inv, R, myn);
       vso = av;
     } else {
       // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded

@@ -99,11 +99,11 @@ uint32_t oracle_draw_word(uint64_t seed, int64_t t, uint32_t tensor_id, uint32_t
     return out[e & 3u];
 }
 
-/* Uniform in [0,1) with 2^-23 granularity: the top 23 bits of the word,
+/* Uniform in [0,1) with 2^-23 granularity: the low 23 bits of the word,
  * scaled by 2^-23 (exact in binary32). */
 float oracle_uniform(uint32_t word)
 {
-    return (float)(word >> 9) * 0x1p-23f;
+    return (float)(word & 0x7FFFFFu) * 0x1p-23f;
 }
 
 /* ------------------------------------------------------------------------- */

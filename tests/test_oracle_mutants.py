@@ -55,8 +55,8 @@ MUTANTS = [
      "uint32_t y0 = hi0 ^ x1 ^ k0;"),
     ("draw counter words swapped", "(uint32_t)t,\n                       tensor_id * 2u + stream}",
      "tensor_id * 2u + stream,\n                       (uint32_t)t}"),
-    ("uniform scaled by the wrong power", "(float)(word >> 9) * 0x1p-23f",
-     "(float)(word >> 8) * 0x1p-23f"),
+    ("uniform takes 24 bits", "(float)(word & 0x7FFFFFu) * 0x1p-23f",
+     "(float)(word & 0xFFFFFFu) * 0x1p-23f"),
     ("NF4 offset", "const double offset = 0.9677083;", "const double offset = 0.96;"),
     ("NF4 negatives not normalised", "out[i] = neg[i] / top;", "out[i] = neg[i] / (top * 1.0001);"),
     ("first bias correction dropped", "s->step_size = (float)((double)lr / bc1);",

@@ -45,10 +45,12 @@ def test_draw_is_word_e_mod_4_of_one_call():
 
 
 def test_uniform_range_and_granularity():
+    """u is the word's low 23 bits times 2^-23."""
     assert oracle.uniform(0) == 0.0
     assert oracle.uniform(0xFFFFFFFF) == 1.0 - 2.0 ** -23
-    assert oracle.uniform(1 << 9) == 2.0 ** -23
-    assert oracle.uniform((1 << 9) - 1) == 0.0
+    assert oracle.uniform(1) == 2.0 ** -23
+    assert oracle.uniform(1 << 23) == 0.0
+    assert oracle.uniform(0x12345678) == (0x12345678 & 0x7FFFFF) * 2.0 ** -23
 
 
 def test_uniform_moments():
