@@ -31,6 +31,9 @@ BLOCK = 128
 MIN_QUANT_NUMEL = 4096
 VCODE_ZIPSR = 0
 VCODE_ZEEDEN = 1
+VCODE_ZI_RTN = 2      # zero-inclusive code, state-space round-to-nearest
+VCODE_ZI_SR = 3       # zero-inclusive code, state-space stochastic rounding
+VCODE_ZE_FLOOR = 4    # zero-excluded code, no rescale
 T_NORM = 1
 T_LM_HEAD = 2
 T_FP32_STATE = 4
@@ -93,6 +96,10 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_nf4_sr.argtypes = [c.c_float, c.c_float]
     L.oracle_zipsr_bracket.restype = c.c_int
     L.oracle_zipsr_bracket.argtypes = [c.c_float]
+    L.oracle_zi_rtn.restype = c.c_int
+    L.oracle_zi_rtn.argtypes = [c.c_float]
+    L.oracle_zi_sr.restype = c.c_int
+    L.oracle_zi_sr.argtypes = [c.c_float, c.c_float]
     L.oracle_zipsr_decide.restype = c.c_int
     L.oracle_zipsr_decide.argtypes = [c.c_float] * 5
     L.oracle_zeeden_code.restype = c.c_int
@@ -206,6 +213,14 @@ def nf4_sr(x: float, u: float) -> int:
 
 def zipsr_bracket(x: float) -> int:
     return int(lib().oracle_zipsr_bracket(x))
+
+
+def zi_rtn(x: float) -> int:
+    return int(lib().oracle_zi_rtn(x))
+
+
+def zi_sr(x: float, u: float) -> int:
+    return int(lib().oracle_zi_sr(x, u))
 
 
 def zipsr_decide(x: float, dv: float, R: float, eps: float, u: float) -> int:

@@ -44,6 +44,13 @@
 #define ORACLE_BLOCK 128          /* values per quantisation block [L, memory paragraph] */
 #define ORACLE_VCODE_ZIPSR 0
 #define ORACLE_VCODE_ZEEDEN 1
+/* State-space variants the pages compare the two methods with ([L, car /
+ * stochastic rounding paragraph]: the 834M ablation's state-space round-to-
+ * nearest and stochastic rounding on the zero-inclusive code; [L, memory
+ * paragraph]: a zero-excluded code with a positive floor and no rescale). */
+#define ORACLE_VCODE_ZI_RTN 2
+#define ORACLE_VCODE_ZI_SR 3
+#define ORACLE_VCODE_ZE_FLOOR 4
 #define ORACLE_STREAM_V 0u        /* Philox stream for the v draw (ZIP-SR)        */
 #define ORACLE_STREAM_M 1u        /* Philox stream for the LM-head m draw         */
 
@@ -153,6 +160,7 @@ static float g_nf4[16];       /* NF4 levels, ascending, binary32              */
 static float g_nf4_mid[15];   /* rounding thresholds between adjacent levels  */
 static float g_vz[16];        /* ZIP-SR v code points k/15                    */
 static float g_vz_sqrt[16];   /* sqrt of the ZIP-SR code points              */
+static float g_vz_mid[15];    /* nearest-point thresholds of the k/15 code     */
 static int g_tables_ready = 0;
 
 static void build_tables(void)
@@ -168,6 +176,8 @@ static void build_tables(void)
         g_vz[k] = (float)k / 15.0f;          /* correctly rounded k/15 */
         g_vz_sqrt[k] = sqrtf(g_vz[k]);       /* correctly rounded sqrt  */
     }
+    for (int k = 0; k < 15; ++k)
+        g_vz_mid[k] = (float)(((double)g_vz[k] + (double)g_vz[k + 1]) * 0.5);
     g_tables_ready = 1;
 }
 
@@ -300,6 +310,29 @@ int oracle_zipsr_bracket(float x)
     return k;
 }
 
+/* Zero-inclusive code, state-space round-to-nearest: the count of the
+ * binary32 midpoints between adjacent code points strictly below x (a value
+ * exactly on a midpoint goes low). */
+int oracle_zi_rtn(float x)
+{
+    build_tables();
+    int c = 0;
+    for (int k = 0; k < 15; ++k)
+        if (x > g_vz_mid[k]) ++c;
+    return c;
+}
+
+/* Zero-inclusive code, state-space stochastic rounding [K, Stochastic
+ * rounding]: x in the bracket [a, b] goes to a with probability
+ * (b - x)/(b - a), i.e. when u*(b - a) < b - x. */
+int oracle_zi_sr(float x, float u)
+{
+    build_tables();
+    int k = oracle_zipsr_bracket(x);
+    int lower = (u * (g_vz[k + 1] - g_vz[k])) < (g_vz[k + 1] - x);
+    return lower ? k : k + 1;
+}
+
 /* ZIP-SR decision for one element [D, Core equation]: the lower code point a
  * is kept with probability [h(v)-h(b)]/[h(a)-h(b)], h(y) = 1/(sqrt(y)*rs_bc2
  * + eps).  With d = 1/h this is (db - dv)*da / ((db - da)*dv); the element
@@ -316,7 +349,7 @@ int oracle_zipsr_decide(float x, float dv, float R, float eps, float u)
     float db = fmaf(g_vz_sqrt[k + 1], R, eps);
     int lower;
     if (da == db) {
-        lower = (u * (g_vz[k + 1] - g_vz[k])) < (g_vz[k + 1] - x);
+        return oracle_zi_sr(x, u);
     } else {
         float lhs = u * ((db - da) * dv);
         float rhs = (db - dv) * da;
@@ -375,8 +408,8 @@ void oracle_block4(const oracle_scalars *s, float decay, int vcode, int m_sr, ui
     for (int i = 0; i < nvalid; ++i) {
         float m0 = g_nf4[nibble(mcodes, i)] * sm;
         int cv = nibble(vcodes, i);
-        float v0 = (vcode == ORACLE_VCODE_ZIPSR) ? g_vz[cv] * sv
-                                                 : ((float)(cv + 1) * 0.0625f) * sv;
+        int zero_excluded = (vcode == ORACLE_VCODE_ZEEDEN || vcode == ORACLE_VCODE_ZE_FLOOR);
+        float v0 = zero_excluded ? ((float)(cv + 1) * 0.0625f) * sv : g_vz[cv] * sv;
         den[i] = oracle_update_elem(s, decay, bf16_to_f32(g[i]), m0, v0, &w[i], &m1[i], &v1[i]);
     }
     memset(mcodes, 0, ORACLE_BLOCK / 2);
@@ -404,7 +437,7 @@ void oracle_block4(const oracle_scalars *s, float decay, int vcode, int m_sr, ui
         *mscale = am;
     }
 
-    /* Second moment: max scale, then ZIP-SR or ZE-EDEN. */
+    /* Second moment: max scale, then ZIP-SR, ZE-EDEN or a state-space variant. */
     float av = 0.0f;
     for (int i = 0; i < nvalid; ++i) av = fmaxf(av, v1[i]);
     if (av < FLT_MIN) {
@@ -420,6 +453,23 @@ void oracle_block4(const oracle_scalars *s, float decay, int vcode, int m_sr, ui
                                                       elem0 + (uint64_t)i));
             set_nibble(vcodes, i, oracle_zipsr_decide(x, den[i], R, s->eps, u));
         }
+        *vscale = av;
+    } else if (vcode == ORACLE_VCODE_ZI_RTN || vcode == ORACLE_VCODE_ZI_SR) {
+        for (int i = 0; i < nvalid; ++i) {
+            float x = v1[i] * inv;
+            int c;
+            if (vcode == ORACLE_VCODE_ZI_RTN) {
+                c = oracle_zi_rtn(x);
+            } else {
+                float u = oracle_uniform(oracle_draw_word(s->seed, s->t, tensor_id,
+                                                          ORACLE_STREAM_V, elem0 + (uint64_t)i));
+                c = oracle_zi_sr(x, u);
+            }
+            set_nibble(vcodes, i, c);
+        }
+        *vscale = av;
+    } else if (vcode == ORACLE_VCODE_ZE_FLOOR) {
+        for (int i = 0; i < nvalid; ++i) set_nibble(vcodes, i, oracle_zeeden_code(v1[i] * inv));
         *vscale = av;
     } else {
         float xx[ORACLE_BLOCK], xq[ORACLE_BLOCK];

@@ -14,6 +14,7 @@ import test_oracle_driver as D
 import test_oracle_nf4 as N
 import test_oracle_philox as P
 import test_oracle_update as U
+import test_oracle_variants as V
 import test_oracle_zeeden as E
 import test_oracle_zipsr as Z
 
@@ -45,6 +46,11 @@ def pins(golden):
         ("first step", U.test_update_elem_values),
         ("ordering", U.test_weights_updated_before_quantising),
         ("nibble layout", D.test_nibble_layout_of_the_codes),
+        ("k/15 nearest", V.test_zi_rtn_is_nearest_code_point),
+        ("k/15 state-space SR", lambda: [V.test_zi_sr_unbiased_by_enumeration(x)
+                                         for x in (0.01, 0.2, 0.77)]),
+        ("worked example, state space", lambda: V.test_worked_example_state_space_rounding(golden)),
+        ("floor code", V.test_ze_floor_is_nearest_zero_excluded_without_rescale),
     ]
 
 
@@ -72,7 +78,14 @@ MUTANTS = [
      "*w = fmaf(s->step_size, m1 / den, w1);"),
     ("NF4 ties go high", "if (x > g_nf4_mid[j]) ++c;", "if (x >= g_nf4_mid[j]) ++c;"),
     ("state-space SR sides swapped", "return lower ? j : j + 1;", "return lower ? j + 1 : j;"),
-    ("ZIP-SR sides swapped", "return lower ? k : k + 1;", "return lower ? k + 1 : k;"),
+    ("ZIP-SR sides swapped", "return lower ? k : k + 1;\n}\n\n/* ZE-EDEN",
+     "return lower ? k + 1 : k;\n}\n\n/* ZE-EDEN"),
+    ("k/15 state-space SR sides swapped",
+     "(g_vz[k + 1] - x);\n    return lower ? k : k + 1;",
+     "(g_vz[k + 1] - x);\n    return lower ? k + 1 : k;"),
+    ("k/15 nearest ties go high", "if (x > g_vz_mid[k]) ++c;", "if (x >= g_vz_mid[k]) ++c;"),
+    ("floor code rescaled", "oracle_zeeden_code(v1[i] * inv));\n        *vscale = av;",
+     "oracle_zeeden_code(v1[i] * inv));\n        *vscale = av * 1.01f;"),
     ("ZIP-SR a and b swapped",
      "float da = fmaf(g_vz_sqrt[k], R, eps);\n    float db = fmaf(g_vz_sqrt[k + 1], R, eps);",
      "float db = fmaf(g_vz_sqrt[k], R, eps);\n    float da = fmaf(g_vz_sqrt[k + 1], R, eps);"),
