@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 WORKLOAD = "gpt-2.7b"        # the benchmark workload; --workload picks a profiling case
+VCODES = {"zipsr": 0, "zeeden": 1, "zi_rtn": 2, "zi_sr": 3, "ze_floor": 4}
 METRIC = "fused 4-bit AdamW step Gparams/s; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SRC = os.path.join(ROOT, "bit_quantized_optimizer_b200", "csrc", "adamw4.cu")
@@ -215,7 +216,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    vcode = 0 if args.vcode == "zipsr" else 1
+    vcode = VCODES[args.vcode]
     ts = workloads.tensor_list(WORKLOAD)
     # per step: the first up-to-64K values of every tensor (about 12M params);
     # inputs from the host generator, state zero-initialised
@@ -288,7 +289,7 @@ def run_ours(args):
     ws_, rank, local = dist_setup(args.gpus)
     import bit_quantized_optimizer_b200 as B
     B.lib()  # fail loudly if the extension is missing
-    vcode = B.ADAMW4_V_ZIPSR if args.vcode == "zipsr" else B.ADAMW4_V_ZEEDEN
+    vcode = VCODES[args.vcode]
     ts = workloads.tensor_list(WORKLOAD)
     params, grads = workloads.device_inputs(WORKLOAD, ts, seed=rank)
     torch.cuda.synchronize()
@@ -377,7 +378,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--vcode", choices=["zipsr", "zeeden"], default="zipsr")
+    ap.add_argument("--vcode", choices=list(VCODES), default="zipsr",
+                    help="second-moment code: the two methods, or a state-space variant")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -82,6 +82,9 @@ static_assert(kStageBytes % 16 == 0, "stage alignment");
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr int kVZip = ADAMW4_V_ZIPSR;
 constexpr int kVZe = ADAMW4_V_ZEEDEN;
+constexpr int kVZiRtn = ADAMW4_V_ZI_RTN;
+constexpr int kVZiSr = ADAMW4_V_ZI_SR;
+constexpr int kVZeFloor = ADAMW4_V_ZE_FLOOR;
 constexpr uint32_t kKindFp32 = 1u << 16;          // internal flag: fp32-state tensor
 constexpr uint32_t kStaged = 1u << 17;            // internal flag: unit data is in the stage
 constexpr uint32_t kNoUnit = 1u << 18;            // internal flag: empty slot of the last tile
@@ -129,6 +132,7 @@ struct CodeTables {
   float nf4_gap[16];    // nf4[j+1] - nf4[j]
   float vz[16];         // ZIP-SR code points k/15
   float vz_sqrt[16];    // sqrt(k/15)
+  float vz_mid[16];     // nearest-point thresholds of the k/15 code (15 used)
   float2 rtn[128];      // NF4 nearest-level buckets: .x threshold, .y base code (int bits)
 };
 
@@ -334,6 +338,7 @@ struct SmemTables {
   float4 zip[16];      // for k0 = nearest integer to 15x: {VZ[k0] (+inf for 15),
                        //   sqrt VZ[k0-1], sqrt VZ[k0], sqrt VZ[k0+1]}
   float2 vzp[16];      // {k/15, (k+1)/15}
+  float vzmid[16];     // thresholds between adjacent k/15 code points
 };
 
 // ---------------------------------------------------------------------------
@@ -454,6 +459,46 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
         vco = zipsr_codes8<FULL, false>(a, S, v1, den, rw, inv, R, myn);
       else
         vco = zipsr_codes8<FULL, true>(a, S, v1, den, rw, inv, R, myn);
+      vso = av;
+    } else if (VCODE == kVZiRtn || VCODE == kVZiSr) {
+      // State-space rules on the zero-inclusive code: nearest code point, or
+      // the lower one with probability (b - x)/(b - a).
+      uint32_t rw[kPerLane];
+      if (VCODE == kVZiSr) words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
+#pragma unroll
+      for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
+        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+        const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
+#pragma unroll
+        for (int h = 1; h >= 0; --h) {
+          const int i = 2 * j + h;
+          const float x = h ? x2.y : x2.x;
+          const uint32_t k0 = __float_as_uint(h ? t2.y : t2.x) & 15u;
+          const uint32_t k = k0 - ((x < S.zip[k0].x) ? 1u : 0u);   // the bracket
+          uint32_t c;
+          if (VCODE == kVZiRtn) {
+            c = k + ((x > S.vzmid[k]) ? 1u : 0u);
+          } else {
+            const float2 z = S.vzp[k];
+            const bool lower = __fmul_rn(uniform23(rw[i]), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
+            c = k + (lower ? 0u : 1u);
+          }
+          vco = vco * 16u + ((FULL || i < myn) ? c : 0u);
+        }
+      }
+      vso = av;
+    } else if (VCODE == kVZeFloor) {
+      // Zero-excluded code with a positive floor: nearest (k+1)/16, no rescale.
+#pragma unroll
+      for (int j = kPerLane / 2 - 1; j >= 0; --j) {
+        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+        const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
+        const uint32_t k0 = max(__float_as_uint(t2.x) & 31u, 1u) - 1u;
+        const uint32_t k1 = max(__float_as_uint(t2.y) & 31u, 1u) - 1u;
+        const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? k1 : 0u;
+        const uint32_t c0 = (FULL || 2 * j < myn) ? k0 : 0u;
+        vco = (vco * 16u + c1) * 16u + c0;
+      }
       vso = av;
     } else {
       // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
@@ -676,8 +721,9 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
     const int t = threadIdx.x;
     if (t < 256) {
       S.mpair[t] = make_float2(tabs.nf4[t & 15], tabs.nf4[t >> 4]);
-      const float lo = (VCODE == kVZip) ? tabs.vz[t & 15] : __fmul_rn((float)((t & 15) + 1), 0.0625f);
-      const float hi = (VCODE == kVZip) ? tabs.vz[t >> 4] : __fmul_rn((float)((t >> 4) + 1), 0.0625f);
+      const bool zx = (VCODE == kVZe || VCODE == kVZeFloor);   // zero-excluded code
+      const float lo = zx ? __fmul_rn((float)((t & 15) + 1), 0.0625f) : tabs.vz[t & 15];
+      const float hi = zx ? __fmul_rn((float)((t >> 4) + 1), 0.0625f) : tabs.vz[t >> 4];
       S.vpair[t] = make_float2(lo, hi);
     }
     if (t < 128) S.rtn[t] = tabs.rtn[t];
@@ -688,6 +734,7 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
       S.zip[t] = make_float4(t == 15 ? INFINITY : tabs.vz[t], tabs.vz_sqrt[max(t - 1, 0)],
                              tabs.vz_sqrt[t], tabs.vz_sqrt[min(t + 1, 15)]);
       S.vzp[t] = make_float2(tabs.vz[t], tabs.vz[min(t + 1, 15)]);
+      S.vzmid[t] = tabs.vz_mid[t];
     }
     if (t < kStages) {
       // full: the producer's expect-tx arrive plus one cp.async arrive per
@@ -844,6 +891,9 @@ void build_tables(CodeTables* T) {
     T->vz[k] = num / 15.0f;
     T->vz_sqrt[k] = std::sqrt(T->vz[k]);
   }
+  for (int k = 0; k < 15; ++k)
+    T->vz_mid[k] = (float)(((double)T->vz[k] + (double)T->vz[k + 1]) * 0.5);
+  T->vz_mid[15] = INFINITY;
   // Midpoints of adjacent binary32 levels, exact in binary64, rounded once.
   float mid[15];
   for (int j = 0; j < 15; ++j)
@@ -922,8 +972,8 @@ int validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n) {
     return fail(nullptr, ADAMW4_EINVAL, "eps must be positive and finite");
   if (!(cfg->lr >= 0.0f) || !std::isfinite(cfg->lr))
     return fail(nullptr, ADAMW4_EINVAL, "lr must be finite and non-negative");
-  if (cfg->vcode != ADAMW4_V_ZIPSR && cfg->vcode != ADAMW4_V_ZEEDEN)
-    return fail(nullptr, ADAMW4_EINVAL, "vcode must be ADAMW4_V_ZIPSR or ADAMW4_V_ZEEDEN");
+  if (cfg->vcode < ADAMW4_V_ZIPSR || cfg->vcode > ADAMW4_V_ZE_FLOOR)
+    return fail(nullptr, ADAMW4_EINVAL, "vcode must be one of the adamw4_vcode values");
   if (cfg->total_steps < 0) return fail(nullptr, ADAMW4_EINVAL, "total_steps must be >= 0");
   if (n < 0 || (n > 0 && ts == nullptr))
     return fail(nullptr, ADAMW4_EINVAL, "tensor list is NULL or n < 0");
@@ -984,6 +1034,40 @@ int occupancy_grid(int device, int* grid) {
   return 0;
 }
 
+// The launch grid (SM count x resident CTAs) of the instantiation for vcode.
+int grid_for(int vcode, int device, int* grid) {
+  switch (vcode) {
+    case kVZip: return occupancy_grid<kVZip>(device, grid);
+    case kVZe: return occupancy_grid<kVZe>(device, grid);
+    case kVZiRtn: return occupancy_grid<kVZiRtn>(device, grid);
+    case kVZiSr: return occupancy_grid<kVZiSr>(device, grid);
+    case kVZeFloor: return occupancy_grid<kVZeFloor>(device, grid);
+    default: return (int)cudaErrorInvalidValue;
+  }
+}
+
+// Enqueues the step kernel instantiated for vcode.
+void launch_vcode(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t nunits,
+                  const StepArgs& a, const CodeTables& tabs, const StateArena& st) {
+  switch (vcode) {
+    case kVZip:
+      adamw4_step_kernel<kVZip><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      break;
+    case kVZe:
+      adamw4_step_kernel<kVZe><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      break;
+    case kVZiRtn:
+      adamw4_step_kernel<kVZiRtn><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      break;
+    case kVZiSr:
+      adamw4_step_kernel<kVZiSr><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      break;
+    default:
+      adamw4_step_kernel<kVZeFloor><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      break;
+  }
+}
+
 int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
   if (h->nunits == 0) return ADAMW4_OK;
   const int64_t need = (h->nunits + kHalves - 1) / kHalves;
@@ -991,12 +1075,7 @@ int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
   a.status = h->d_status;
   a.fault_stall = h->fault_stall;
   h->fault_stall = 0;
-  if (h->cfg.vcode == kVZip)
-    adamw4_step_kernel<kVZip><<<grid, kCtaThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
-                                                                     h->tabs, h->st);
-  else
-    adamw4_step_kernel<kVZe><<<grid, kCtaThreads, kSmemStages, s>>>(h->d_tensors, h->nunits, a,
-                                                                    h->tabs, h->st);
+  launch_vcode(h->cfg.vcode, grid, s, h->d_tensors, h->nunits, a, h->tabs, h->st);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(h, e, "step kernel launch");
   return ADAMW4_OK;
@@ -1118,8 +1197,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
     delete h;
     return cuda_fail(nullptr, e, "initialising the state");
   }
-  int ge = (cfg->vcode == kVZip) ? occupancy_grid<kVZip>(device, &h->grid)
-                                 : occupancy_grid<kVZe>(device, &h->grid);
+  int ge = grid_for(cfg->vcode, device, &h->grid);
   if (ge != 0) {
     release(h);
     delete h;
@@ -1404,7 +1482,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 struct NoAllocDevice {
   bool ready;
   unsigned char* scratch;   // device address of g_noalloc_scratch on this device
-  int grid_zip, grid_ze;
+  int grid[ADAMW4_V_ZE_FLOOR + 1];   // per vcode
 };
 
 std::mutex g_noalloc_mu;
@@ -1421,7 +1499,7 @@ int na_validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n,
   if (!(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) || !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f))
     return ADAMW4_EINVAL;
   if (!(cfg->eps > 0.0f) || !std::isfinite(cfg->eps)) return ADAMW4_EINVAL;
-  if (cfg->vcode != ADAMW4_V_ZIPSR && cfg->vcode != ADAMW4_V_ZEEDEN) return ADAMW4_EINVAL;
+  if (cfg->vcode < ADAMW4_V_ZIPSR || cfg->vcode > ADAMW4_V_ZE_FLOOR) return ADAMW4_EINVAL;
   if (cfg->total_steps < 0 || t < 1) return ADAMW4_EINVAL;
   if (!(lr >= 0.0f) || !std::isfinite(lr)) return ADAMW4_EINVAL;
   if (n < 0 || (n > 0 && ts == nullptr)) return ADAMW4_EINVAL;
@@ -1469,9 +1547,8 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&nd.scratch), g_noalloc_scratch) !=
         cudaSuccess)
       return ADAMW4_ECUDA;
-    if (occupancy_grid<kVZip>(device, &nd.grid_zip) != 0 ||
-        occupancy_grid<kVZe>(device, &nd.grid_ze) != 0)
-      return ADAMW4_ECUDA;
+    for (int vc = ADAMW4_V_ZIPSR; vc <= ADAMW4_V_ZE_FLOOR; ++vc)
+      if (grid_for(vc, device, &nd.grid[vc]) != 0) return ADAMW4_ECUDA;
     nd.ready = true;
   }
   // The table adamw4_create would build, in the same order and layout.
@@ -1519,11 +1596,7 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   st.fm = state->m32;
   st.fv = state->v32;
   const int64_t need = (unit + kHalves - 1) / kHalves;
-  if (cfg->vcode == kVZip)
-    adamw4_step_kernel<kVZip><<<(int)std::min<int64_t>(nd.grid_zip, need), kCtaThreads,
-                                kSmemStages, s>>>(table, unit, a, tabs, st);
-  else
-    adamw4_step_kernel<kVZe><<<(int)std::min<int64_t>(nd.grid_ze, need), kCtaThreads,
-                               kSmemStages, s>>>(table, unit, a, tabs, st);
+  launch_vcode(cfg->vcode, (int)std::min<int64_t>(nd.grid[cfg->vcode], need), s, table, unit, a,
+               tabs, st);
   return cudaGetLastError() == cudaSuccess ? ADAMW4_OK : ADAMW4_ECUDA;
 }

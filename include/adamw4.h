@@ -66,9 +66,16 @@ enum {
     ADAMW4_FAULT_STALL_PIPELINE = 1  /* next step: stages marked pending, never filled */
 };
 
+/* Second-moment codes.  ZIPSR and ZEEDEN are the two methods; the other three
+ * are the state-space quantisers the pages compare them with (the controlled
+ * ablation's round-to-nearest and stochastic rounding on the zero-inclusive
+ * code, and a zero-excluded code with a positive floor and no rescale). */
 typedef enum {
     ADAMW4_V_ZIPSR = 0,     /* zero-inclusive code, preconditioner-space SR    */
-    ADAMW4_V_ZEEDEN = 1     /* zero-excluded code, EDEN block rescale          */
+    ADAMW4_V_ZEEDEN = 1,    /* zero-excluded code, EDEN block rescale          */
+    ADAMW4_V_ZI_RTN = 2,    /* zero-inclusive code, state-space nearest        */
+    ADAMW4_V_ZI_SR = 3,     /* zero-inclusive code, state-space SR             */
+    ADAMW4_V_ZE_FLOOR = 4   /* zero-excluded code, nearest, no rescale         */
 } adamw4_vcode;
 
 /* Per-tensor flags. */
@@ -104,7 +111,7 @@ typedef struct {
 /* Optimizer configuration.
  *   lr            default learning rate (each step passes its own lr)
  *   beta1, beta2  in [0, 1); eps > 0
- *   vcode         ADAMW4_V_ZIPSR or ADAMW4_V_ZEEDEN
+ *   vcode         an adamw4_vcode
  *   seed          key of the counter-based random draws
  *   total_steps   T for the final-10% LM-head phase (active when 10 t > 9 T);
  *                 0 means the phase never starts */

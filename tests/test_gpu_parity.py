@@ -24,6 +24,17 @@ def test_single_65k_zipsr_10_steps():
              what="single-65k")
 
 
+@pytest.mark.parametrize("vcode", [2, 3, 4])
+def test_single_65k_state_space_variants_10_steps(vcode):
+    """The state-space variants (zero-inclusive nearest and stochastic
+    rounding, zero-excluded floor without rescale) on the 65,536-element
+    workload with its near-zero coordinates, 10 steps."""
+    ts = workloads.tensor_list("single-65k")
+    ws = workloads.host_weights("single-65k", ts)
+    run_both(ts, ws, _grads_fn("single-65k", ts), 10, vcode=vcode, seed=12,
+             check_every_step=True, what=f"single-65k v{vcode}")
+
+
 def test_single_4m_zeeden_20_steps():
     """4,194,304 elements (32,768 blocks), 20 steps, ZE-EDEN, per-block
     gradient scales log-uniform over three decades."""
@@ -35,7 +46,10 @@ def test_single_4m_zeeden_20_steps():
 RAGGED = [1, 7, 100, 4095, 4096, 4097, 4096 + 5, 4096 + 37, 4096 + 120, 128 * 37 + 64, 8192]
 
 
-@pytest.mark.parametrize("vcode", [0, 1])
+ALL_VCODES = [0, 1, 2, 3, 4]   # ZIP-SR, ZE-EDEN, and the three state-space variants
+
+
+@pytest.mark.parametrize("vcode", ALL_VCODES)
 def test_ragged_mixed_tensor_list(vcode):
     """Every tail shape: whole blocks, a last lane with 1..7 values, lanes with
     nothing, fp32-state tensors below 4096 and flagged NORM / FP32_STATE,
@@ -57,7 +71,7 @@ def test_ragged_mixed_tensor_list(vcode):
              check_every_step=True, what=f"ragged v{vcode}")
 
 
-@pytest.mark.parametrize("vcode", [0, 1])
+@pytest.mark.parametrize("vcode", ALL_VCODES)
 def test_degenerate_values(vcode):
     """All-zero gradients (blocks stay exactly zero, then decay onto code
     points), gradients whose squares are subnormal, single huge outliers in a
