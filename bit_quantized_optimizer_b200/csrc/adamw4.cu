@@ -120,7 +120,7 @@ struct StepArgs {
   float rs_bc2;      // 1 / sqrt(1 - b2^t)
   float b1, omb1, b2, omb2, eps, lr;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
-  uint32_t t_lo;         // step, low word (Philox counter word 2)
+  uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
   int lm_sr_active;      // final-10% LM-head phase
   uint32_t* status;      // device status word (bit 0: a pipeline wait timed out)
   int fault_stall;       // test hook: mark stages filled without filling them
@@ -249,7 +249,7 @@ __device__ __forceinline__ bool wait_phase_napping(uint32_t bar, uint32_t parity
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
-    __nanosleep(256);
+    __nanosleep(1000);
     if (mbar_test_wait(bar, parity)) return true;
     if (global_ns() - t0 > limit_ns) return false;
   }
@@ -259,9 +259,16 @@ __device__ __forceinline__ bool wait_phase_napping(uint32_t bar, uint32_t parity
 // Arithmetic helpers
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const StepArgs& a) {
+// Philox4x32-10 of the counter (quad low, quad high, t, c3).  The counter's
+// third word is the step t for every draw of a launch, so round 0's product
+// M1 * t is a per-step constant the host supplies (r0_hi_k0 = hi(M1 t) ^ key0,
+// r0_lo = lo(M1 t)); rounds 1..9 are the usual ones.
+__device__ __forceinline__ uint4 philox4x32_10(uint64_t quad, uint32_t c3, const StepArgs& a) {
+  const uint64_t q0 = (uint64_t)kPhiloxM0 * (uint32_t)quad;
+  uint4 c = make_uint4(a.r0_hi_k0 ^ (uint32_t)(quad >> 32), a.r0_lo,
+                       (uint32_t)(q0 >> 32) ^ c3 ^ a.rk1[0], (uint32_t)q0);
 #pragma unroll
-  for (int r = 0; r < 10; ++r) {
+  for (int r = 1; r < 10; ++r) {
     const uint64_t p0 = (uint64_t)kPhiloxM0 * c.x;
     const uint64_t p1 = (uint64_t)kPhiloxM1 * c.z;
     c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ a.rk0[r], (uint32_t)p1,
@@ -282,9 +289,8 @@ __device__ __forceinline__ float uniform23(uint32_t w) { return __fsub_rn(one_pl
 __device__ __forceinline__ void words8(const StepArgs& a, uint32_t tensor_id, uint32_t stream,
                                        uint64_t quad, uint32_t r[8]) {
   const uint32_t c3 = tensor_id * 2u + stream;
-  const uint4 r0 = philox4x32_10(make_uint4((uint32_t)quad, (uint32_t)(quad >> 32), a.t_lo, c3), a);
-  const uint64_t q1 = quad + 1;
-  const uint4 r1 = philox4x32_10(make_uint4((uint32_t)q1, (uint32_t)(q1 >> 32), a.t_lo, c3), a);
+  const uint4 r0 = philox4x32_10(quad, c3, a);
+  const uint4 r1 = philox4x32_10(quad + 1, c3, a);
   r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w;
   r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
 }
@@ -955,7 +961,9 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
     a.rk0[r] = (uint32_t)c.seed + (uint32_t)r * kPhiloxW0;
     a.rk1[r] = (uint32_t)(c.seed >> 32) + (uint32_t)r * kPhiloxW1;
   }
-  a.t_lo = (uint32_t)t;
+  const uint64_t m1t = (uint64_t)kPhiloxM1 * (uint32_t)t;
+  a.r0_hi_k0 = (uint32_t)(m1t >> 32) ^ a.rk0[0];
+  a.r0_lo = (uint32_t)m1t;
   a.lm_sr_active = (c.total_steps > 0) && (10 * t > 9 * c.total_steps);
   a.status = nullptr;
   a.fault_stall = 0;

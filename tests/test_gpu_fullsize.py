@@ -54,8 +54,9 @@ def test_llama_1p1b_zeeden_lm_head_phase_sampled():
     assert n > 1000
 
 
-@pytest.mark.parametrize("vcode", [0, 1])
+@pytest.mark.parametrize("vcode", [0, 1, 2, 3, 4])
 def test_gpt_2p7b_sampled(vcode):
-    """GPT-style 2.7B list (the benchmark workload), two steps from zero state."""
+    """GPT-style 2.7B list (the benchmark workload), two steps from zero state,
+    for the two methods and the three state-space variants."""
     n = sampled_parity("gpt-2.7b", vcode=vcode, steps=2, t0=0, what=f"gpt-2.7b v{vcode}")
     assert n > 1500
