@@ -14,7 +14,7 @@ import os
 
 __all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_V_ZI_RTN", "ADAMW4_V_ZI_SR",
            "ADAMW4_V_ZE_FLOOR", "ADAMW4_T_NORM", "ADAMW4_T_LM_HEAD",
-           "ADAMW4_T_FP32_STATE", "AdamW4Error", "adamw4_tensor", "adamw4_config", "lib",
+           "ADAMW4_T_FP32_STATE", "ADAMW4_T_QUANT_STATE", "AdamW4Error", "adamw4_tensor", "adamw4_config", "lib",
            "adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
            "adamw4_get_step", "adamw4_set_step", "adamw4_state_bytes", "adamw4_state_export",
            "adamw4_state_import", "adamw4_launch_info", "adamw4_last_error", "adamw4_sync",
@@ -33,6 +33,7 @@ ADAMW4_V_ZE_FLOOR = 4    # zero-excluded code, nearest, no rescale
 ADAMW4_T_NORM = 1
 ADAMW4_T_LM_HEAD = 2
 ADAMW4_T_FP32_STATE = 4
+ADAMW4_T_QUANT_STATE = 8   # 4-bit state below 4096 elements (a piece of a larger tensor)
 MIN_QUANT_NUMEL = 4096
 BLOCK = 128
 
@@ -53,7 +54,8 @@ class AdamW4Error(RuntimeError):
 class adamw4_tensor(ctypes.Structure):
     _fields_ = [("param", ctypes.c_void_p), ("grad_bf16", ctypes.c_void_p),
                 ("numel", ctypes.c_int64), ("tensor_id", ctypes.c_uint32),
-                ("flags", ctypes.c_uint32), ("weight_decay", ctypes.c_float)]
+                ("flags", ctypes.c_uint32), ("weight_decay", ctypes.c_float),
+                ("elem_offset", ctypes.c_int64)]
 
 
 class adamw4_state_buffers(ctypes.Structure):
@@ -197,15 +199,18 @@ def adamw4_launch_info(h):
 
 
 def is_fp32_state(numel: int, flags: int) -> bool:
-    """The library's classification rule: fp32 state below 4096 elements or
-    for NORM / FP32_STATE tensors."""
-    return numel < MIN_QUANT_NUMEL or bool(flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE))
+    """The library's classification rule: fp32 state for NORM / FP32_STATE
+    tensors, and below 4096 elements unless flagged QUANT_STATE."""
+    if flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE):
+        return True
+    return numel < MIN_QUANT_NUMEL and not flags & ADAMW4_T_QUANT_STATE
 
 
 class AdamW4:
     """Optimizer over torch tensors: fp32 params and bf16 grads (contiguous,
     16-byte aligned, on one CUDA device).  ``specs`` is a list of dicts with
-    tensor_id, flags and weight_decay, parallel to ``params``."""
+    tensor_id, flags, weight_decay and (for a piece of a larger tensor)
+    elem_offset, parallel to ``params``."""
 
     def __init__(self, params, grads, specs, lr=1e-3, betas=(0.9, 0.999), eps=1e-8,
                  vcode=ADAMW4_V_ZIPSR, seed=0, total_steps=0):
@@ -219,7 +224,8 @@ class AdamW4:
             if not (p.is_contiguous() and g.is_contiguous()) or p.numel() != g.numel():
                 raise ValueError("params and grads must be contiguous and of equal size")
             ts.append(adamw4_tensor(p.data_ptr(), g.data_ptr(), p.numel(), s["tensor_id"],
-                                    s.get("flags", 0), s.get("weight_decay", 0.0)))
+                                    s.get("flags", 0), s.get("weight_decay", 0.0),
+                                    s.get("elem_offset", 0)))
         self.cfg = adamw4_config(lr, betas[0], betas[1], eps, vcode, seed, total_steps)
         self.lr = lr
         self.handle = adamw4_create(self.cfg, ts, dev)

@@ -110,7 +110,7 @@ struct __align__(16) DevTensor {
   uint32_t tensor_id;
   uint32_t flags;       // ADAMW4_T_* | kKindFp32
   float weight_decay;
-  uint32_t pad_;
+  uint32_t block_offset;  // elem_offset / 128: where this piece starts in its tensor
 };
 static_assert(sizeof(DevTensor) == 64, "DevTensor layout");
 
@@ -149,7 +149,7 @@ struct StateArena {
 struct __align__(16) UnitHeader {
   float* w;              // the unit's first weight
   const uint16_t* g;     // its first gradient
-  uint64_t e0;           // index of that element within its tensor
+  uint64_t e0;           // index of that element within its (logical) tensor
   uint64_t state;        // 4-bit: block index in the code arena; fp32: element index
   uint32_t tensor_id;
   uint32_t flags;        // ADAMW4_T_* | kKindFp32 | kStaged
@@ -629,7 +629,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
   constexpr unsigned kMask = (1u << kHalves) - 1u;
   const int64_t ntiles = (nunits + kHalves - 1) / kHalves;
   int ti = -1;
-  int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0;
+  int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0, t_eoff = 0;
   float* t_param = nullptr;
   const uint16_t* t_grad = nullptr;
   uint32_t t_id = 0, t_flags = 0;
@@ -655,6 +655,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
       t_begin = __ldg(&d->unit_begin);
       t_numel = __ldg(&d->numel);
       t_soff = __ldg(&d->state_off);
+      t_eoff = (int64_t)__ldg(&d->block_offset) * kBlock;
       t_param = d->param;
       t_grad = d->grad;
       t_id = __ldg(&d->tensor_id);
@@ -669,7 +670,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     UnitHeader* hd = reinterpret_cast<UnitHeader*>(sp + kOffHdr) + lane;
     hd->w = t_param + e0;
     hd->g = t_grad + e0;
-    hd->e0 = (uint64_t)e0;
+    hd->e0 = (uint64_t)(t_eoff + e0);   // keys the draws
     hd->state = (t_flags & kKindFp32) ? (uint64_t)(t_soff + e0) : (uint64_t)(t_soff + ub);
     hd->tensor_id = t_id;
     hd->flags = has ? (t_flags | (staged ? kStaged : 0u)) : kNoUnit;
@@ -972,6 +973,45 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+constexpr uint32_t kUserFlags =
+    ADAMW4_T_NORM | ADAMW4_T_LM_HEAD | ADAMW4_T_FP32_STATE | ADAMW4_T_QUANT_STATE;
+
+// fp32 state for normalisation tensors, tensors flagged FP32_STATE and tensors
+// under 4096 elements -- unless QUANT_STATE marks a piece of a larger tensor
+// that keeps 4-bit state.
+bool fp32_state(const adamw4_tensor& t) {
+  if (t.flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE)) return true;
+  if (t.flags & ADAMW4_T_QUANT_STATE) return false;
+  return t.numel < ADAMW4_MIN_QUANT_NUMEL;
+}
+
+// The flag and piece checks of one descriptor: nullptr when they pass.
+const char* piece_error(const adamw4_tensor& t) {
+  if (t.flags & ~kUserFlags) return "unknown flag bits";
+  if ((t.flags & ADAMW4_T_QUANT_STATE) && (t.flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE)))
+    return "QUANT_STATE cannot be combined with NORM or FP32_STATE";
+  if (t.elem_offset < 0 || t.elem_offset % kBlock != 0 || t.elem_offset >= ((int64_t)1 << 39))
+    return "elem_offset must be a multiple of 128 in [0, 2^39)";
+  return nullptr;
+}
+
+// The kernel's descriptor of tensor x, whose units start at `unit` and whose
+// state starts at `state_off`.
+DevTensor dev_tensor(const adamw4_tensor& x, bool fp32, int64_t unit, int64_t state_off) {
+  DevTensor d;
+  d.param = x.param;
+  d.grad = x.grad_bf16;
+  d.numel = x.numel;
+  d.unit_begin = unit;
+  d.unit_end = unit + (x.numel + kBlock - 1) / kBlock;
+  d.state_off = state_off;
+  d.tensor_id = x.tensor_id;
+  d.flags = x.flags | (fp32 ? kKindFp32 : 0u);
+  d.weight_decay = x.weight_decay;
+  d.block_offset = (uint32_t)(x.elem_offset / kBlock);
+  return d;
+}
+
 int validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n) {
   if (cfg == nullptr) return fail(nullptr, ADAMW4_EINVAL, "config is NULL");
   if (!(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) || !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f))
@@ -999,6 +1039,7 @@ int validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n) {
       return fail(nullptr, ADAMW4_EALIGN, at + "param and grad must be 16-byte aligned");
     if (!std::isfinite(t.weight_decay))
       return fail(nullptr, ADAMW4_EINVAL, at + "weight_decay must be finite");
+    if (const char* why = piece_error(t)) return fail(nullptr, ADAMW4_EINVAL, at + why);
     if (!ids.insert(t.tensor_id).second)
       return fail(nullptr, ADAMW4_EINVAL, at + "duplicate tensor_id " + std::to_string(t.tensor_id));
     const uintptr_t p = reinterpret_cast<uintptr_t>(t.param);
@@ -1127,8 +1168,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
   for (int i = 0; i < n; ++i) {
     HostTensor ht{};
     ht.desc = tensors[i];
-    ht.fp32 = tensors[i].numel < ADAMW4_MIN_QUANT_NUMEL ||
-              (tensors[i].flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE)) != 0;
+    ht.fp32 = fp32_state(tensors[i]);
     ht.nblocks = (tensors[i].numel + kBlock - 1) / kBlock;
     if (ht.fp32) {
       ht.state_off = h->nfp32;
@@ -1137,17 +1177,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
       ht.state_off = h->nblocks4;
       h->nblocks4 += ht.nblocks;
     }
-    DevTensor& d = dev[i];
-    d.param = tensors[i].param;
-    d.grad = tensors[i].grad_bf16;
-    d.numel = tensors[i].numel;
-    d.unit_begin = unit;
-    d.unit_end = unit + ht.nblocks;
-    d.state_off = ht.state_off;
-    d.tensor_id = tensors[i].tensor_id;
-    d.flags = tensors[i].flags | (ht.fp32 ? kKindFp32 : 0u);
-    d.weight_decay = tensors[i].weight_decay;
-    d.pad_ = 0;
+    dev[i] = dev_tensor(tensors[i], ht.fp32, unit, ht.state_off);
     unit += ht.nblocks;
     h->tensors.push_back(ht);
   }
@@ -1518,7 +1548,7 @@ int na_validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n,
   for (int i = 0; i < n; ++i) {
     const adamw4_tensor& x = ts[i];
     if (x.param == nullptr || x.grad_bf16 == nullptr || x.numel <= 0 ||
-        x.numel > ((int64_t)1 << 40) || !std::isfinite(x.weight_decay))
+        x.numel > ((int64_t)1 << 40) || !std::isfinite(x.weight_decay) || piece_error(x) != nullptr)
       return ADAMW4_EINVAL;
     if (!na_aligned(x.param, 16) || !na_aligned(x.grad_bf16, 16)) return ADAMW4_EALIGN;
     const uintptr_t p0 = reinterpret_cast<uintptr_t>(x.param), p1 = p0 + (uintptr_t)x.numel * 4u;
@@ -1563,20 +1593,9 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   int64_t unit = 0, blocks4 = 0, elems32 = 0;
   for (int i = 0; i < n; ++i) {
     const adamw4_tensor& x = tensors[i];
-    const bool fp32 = x.numel < ADAMW4_MIN_QUANT_NUMEL ||
-                      (x.flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE)) != 0;
+    const bool fp32 = fp32_state(x);
     const int64_t nb = (x.numel + kBlock - 1) / kBlock;
-    DevTensor& d = g_noalloc_table[i];
-    d.param = x.param;
-    d.grad = x.grad_bf16;
-    d.numel = x.numel;
-    d.unit_begin = unit;
-    d.unit_end = unit + nb;
-    d.state_off = fp32 ? elems32 : blocks4;
-    d.tensor_id = x.tensor_id;
-    d.flags = x.flags | (fp32 ? kKindFp32 : 0u);
-    d.weight_decay = x.weight_decay;
-    d.pad_ = 0;
+    g_noalloc_table[i] = dev_tensor(x, fp32, unit, fp32 ? elems32 : blocks4);
     if (fp32) elems32 += nb * kBlock; else blocks4 += nb;
     unit += nb;
   }

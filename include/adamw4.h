@@ -82,7 +82,9 @@ typedef enum {
 enum {
     ADAMW4_T_NORM = 1u,       /* normalisation-layer tensor: fp32 state        */
     ADAMW4_T_LM_HEAD = 2u,    /* LM head: m rounded stochastically in the final 10% */
-    ADAMW4_T_FP32_STATE = 4u  /* force fp32 state                              */
+    ADAMW4_T_FP32_STATE = 4u, /* force fp32 state                              */
+    ADAMW4_T_QUANT_STATE = 8u /* force 4-bit state below 4096 elements: a piece of a
+                                 larger 4-bit tensor (not with NORM / FP32_STATE) */
 };
 
 /* Tensors below this many elements keep fp32 state. */
@@ -90,13 +92,23 @@ enum {
 /* Values per quantisation block (one fp32 scale per block per moment). */
 #define ADAMW4_BLOCK 128
 
-/* One parameter tensor, flattened row-major.
+/* One parameter tensor, flattened row-major, or a piece of one.
  *   param      device, fp32, numel elements, 16-byte aligned; updated in place
  *   grad_bf16  device, bf16 bit patterns, numel elements, 16-byte aligned; read
  *   tensor_id  unique within a handle; keys the random draws, so it must stay
  *              the same across a checkpoint and resume
- *   flags      ADAMW4_T_* bits
+ *   flags      ADAMW4_T_* bits (other bits: ADAMW4_EINVAL)
  *   weight_decay  decoupled weight decay of this tensor (w <- w (1 - lr wd))
+ *   elem_offset   0 for a whole tensor.  For a piece of a larger (logical)
+ *              tensor, the index of the piece's first element in it: a
+ *              multiple of 128 in [0, 2^39).  Blocks and random draws are
+ *              keyed by the logical index, so stepping the pieces of a tensor
+ *              (in one handle each, on one device or on several) gives the
+ *              same bits as stepping the whole tensor.  A piece under 4096
+ *              elements of a 4-bit tensor needs ADAMW4_T_QUANT_STATE, and a
+ *              piece of an fp32-state tensor ADAMW4_T_FP32_STATE, so that it is
+ *              classified like the whole.  The pages describe single-device
+ *              training; the pieces are this library's ZeRO-1 sharding.
  * Both buffers are borrowed: they stay owned by the caller, and must stay
  * allocated and at the same address until adamw4_destroy. */
 typedef struct {
@@ -106,6 +118,7 @@ typedef struct {
     uint32_t tensor_id;
     uint32_t flags;
     float weight_decay;
+    int64_t elem_offset;
 } adamw4_tensor;
 
 /* Optimizer configuration.
@@ -126,8 +139,9 @@ typedef struct adamw4_handle adamw4_handle;
 
 /* Creates an optimizer over n tensors on CUDA device `device`.
  * Validates every descriptor on the host (non-NULL pointers, 16-byte
- * alignment, numel > 0, unique tensor_id), classifies each tensor (fp32 state
- * when numel < 4096 or flagged NORM/FP32_STATE, else 4-bit), allocates the
+ * alignment, numel > 0, unique tensor_id, known flags, elem_offset), classifies
+ * each tensor (fp32 state when flagged NORM/FP32_STATE, or when numel < 4096
+ * and not flagged QUANT_STATE; else 4-bit), allocates the
  * packed state (owned by the handle) and zeroes it, which is the all-zero
  * initial state m = v = 0.  The step counter starts at t = 0.
  * Returns ADAMW4_EINVAL / EALIGN for bad input, ENOMEM, ECUDA.

@@ -69,6 +69,13 @@ def test_bad_config(L, kw, code):
     (B.adamw4_tensor(P0, P0 + (1 << 30), 0, 0, 0, 0.0), -1, "numel"),
     (B.adamw4_tensor(P0, P0 + (1 << 30), -5, 0, 0, 0.0), -1, "numel"),
     (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, float("inf")), -1, "weight_decay"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 16, 0.0), -1, "unknown flag"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 1 << 16, 0.0), -1, "unknown flag"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 8 | 1, 0.0), -1, "QUANT_STATE"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 8 | 4, 0.0), -1, "QUANT_STATE"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, 0.0, 64), -1, "elem_offset"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, 0.0, -128), -1, "elem_offset"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, 0.0, 1 << 39), -1, "elem_offset"),
 ])
 def test_bad_tensor(L, t, code, msg):
     rc, _ = _create(_cfg(), [t])
@@ -115,3 +122,21 @@ def test_null_out_pointer(L):
     cfg = _cfg()
     arr = (B.adamw4_tensor * 1)(B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, 0.0))
     assert L.adamw4_create(ctypes.byref(cfg), arr, 1, 0, None) == -1
+
+
+def test_piece_descriptors_pass_validation(L):
+    """A block-aligned piece (elem_offset a multiple of 128, below 2^39) with
+    QUANT_STATE gets past validation: the fake addresses then stop it at the
+    injected allocation failure, before any device work."""
+    t = B.adamw4_tensor(P0, P0 + (1 << 30), 256, 0, 8 | 2, 0.0, (1 << 39) - 128)
+    os.environ["ADAMW4_FAIL_ALLOC"] = "1"
+    try:
+        rc, _ = _create(_cfg(), [t])
+    finally:
+        del os.environ["ADAMW4_FAIL_ALLOC"]
+    assert rc == -3 and "injected" in B.adamw4_last_error()
+
+
+def test_descriptor_layout_matches_the_header():
+    assert ctypes.sizeof(B.adamw4_tensor) == 48
+    assert B.adamw4_tensor.elem_offset.offset == 40
