@@ -14,6 +14,11 @@ the workload on its own GPU: the path has no exchange step, so there is no
 data-path collective (weak scaling); the time is the max over ranks.
 `--impl reference` times the CPU oracle on a bounded sample of the same
 workload (rank 0 only).
+
+`--zero1 [--chunks C]` times the ZeRO-1 sharded step instead: the N ranks
+share one copy of the workload, each steps 1/N of it between a reduce-scatter
+of the bf16 gradients and an all-gather of the fp32 weights over NCCL (strong
+scaling; at N = 1 a one-rank group, whose collectives are local copies).
 """
 from __future__ import annotations
 
@@ -44,18 +49,23 @@ def is_fp32_state(numel, flags):
     return numel < 4096 or bool(flags & (workloads.T_NORM | workloads.T_FP32_STATE))
 
 
-def algorithmic_bytes(ts):
-    """HBM bytes one step must move: per 4-bit value, w read+write (8), bf16
-    grad read (2); per 128-value block, m and v codes (64 B each) and scales
-    (4 B each), read and written; per fp32-state value 4+4+2+8+8."""
+def algorithmic_bytes(ts, wbytes=4):
+    """HBM bytes one step must move: per 4-bit value, w read+write (2 x 4, or
+    2 x 2 for bf16 weights), bf16 grad read (2); per 128-value block, m and v
+    codes (64 B each) and scales (4 B each), read and written; per fp32-state
+    value w read+write, grad read, and m, v (4 + 4 each) read and written."""
     b = 0
     for t in ts:
         n = t["numel"]
         if is_fp32_state(n, t["flags"]):
-            b += 26 * n
+            b += (2 * wbytes + 2 + 16) * n
         else:
-            b += 10 * n + 2 * 136 * ((n + 127) // 128)
+            b += (2 * wbytes + 2) * n + 2 * 136 * ((n + 127) // 128)
     return b
+
+
+def variant_name(args):
+    return args.vcode + ("_bf16w" if args.bf16_params else "")
 
 
 def peaks():
@@ -190,8 +200,12 @@ def cpu_baseline(ts, params, grads, vcode, target_s=10.0, per_tensor_cap=1 << 18
         n = min(t["numel"], per_tensor_cap)
         tt = dict(t)
         tt["numel"] = n
+        if p.dtype == torch.bfloat16:
+            tt["flags"] = tt["flags"] | oracle.T_BF16_PARAM
+            ws.append(p[:n].view(torch.int16).cpu().numpy().view(np.uint16).copy())
+        else:
+            ws.append(p[:n].cpu().numpy().copy())
         sub.append(tt)
-        ws.append(p[:n].cpu().numpy().copy())
         gs.append(g[:n].view(torch.int16).cpu().numpy().view(np.uint16).copy())
     nthreads = max(1, oracle.max_threads())
     o = oracle.OracleAdamW4(vcode=vcode, tensors=sub, nthreads=nthreads)
@@ -259,11 +273,12 @@ def e2e_run(B, opt, ts, grads, nparams, stream, ws_, args):
     params back to pinned host memory."""
     import torch
     e2e_steps = max(1, min(3, args.steps))
+    wbytes = 2 if args.bf16_params else 4
     hg = torch.empty(nparams, dtype=torch.int16).pin_memory()
-    hp = torch.empty(nparams, dtype=torch.float32).pin_memory()
+    hp = torch.empty(nparams, dtype=torch.int16 if wbytes == 2 else torch.float32).pin_memory()
     offs = np.cumsum([0] + [t["numel"] for t in ts])
     gptrs = [hg.data_ptr() + 2 * int(o) for o in offs[:-1]]
-    pptrs = [hp.data_ptr() + 4 * int(o) for o in offs[:-1]]
+    pptrs = [hp.data_ptr() + wbytes * int(o) for o in offs[:-1]]
     for g, o, t in zip(grads, offs[:-1], ts):
         hg[int(o):int(o) + t["numel"]].copy_(g.view(torch.int16).cpu())
     B.adamw4_step_host(opt.handle, 1e-3, gptrs, pptrs, stream.cuda_stream)   # warm
@@ -278,7 +293,7 @@ def e2e_run(B, opt, ts, grads, nparams, stream, ws_, args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws_)
     h2d = 2 * nparams
-    d2h = 4 * nparams
+    d2h = wbytes * nparams
     del hg, hp
     return {"value": ws_ * nparams / (e2e_ms * 1e-3) / 1e9, "unit": "Gparams/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
@@ -292,11 +307,15 @@ def run_ours(args):
     vcode = VCODES[args.vcode]
     ts = workloads.tensor_list(WORKLOAD)
     params, grads = workloads.device_inputs(WORKLOAD, ts, seed=rank)
+    if args.bf16_params:                  # bf16 weights: the nearest bf16 of the same draw
+        for i in range(len(params)):
+            params[i] = params[i].to(torch.bfloat16)
     torch.cuda.synchronize()
     opt = B.AdamW4(params, grads, ts, lr=1e-3, vcode=vcode, seed=rank)
     grid, block, units = B.adamw4_launch_info(opt.handle)
     nparams = sum(t["numel"] for t in ts)
-    alg_bytes = algorithmic_bytes(ts)
+    alg_bytes = algorithmic_bytes(ts, 2 if args.bf16_params else 4)
+    resident = (4 if not args.bf16_params else 2) * nparams + 2 * nparams + opt.state_bytes()
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
@@ -352,14 +371,15 @@ def run_ours(args):
             "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "vcode": args.vcode, "params": nparams,
+                       "weights": "bf16" if args.bf16_params else "fp32",
                        "tensors": len(ts), "algorithmic_bytes_per_step": alg_bytes,
                        "parallelism": f"replicas x{ws_} (no data-path collective)",
-                       "l2": "inputs 19.7 GB > 126 MB L2; no flush",
+                       "l2": f"inputs {resident / 1e9:.1f} GB > 126 MB L2; no flush",
                        "grid": grid, "block": block, "units": units},
             "hbm_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": traffic_record(args.vcode)},
+                         "traffic": traffic_record(variant_name(args))},
             "e2e": e2e,
             "gpu_launches": args.steps,
             "clocks": clk,
@@ -373,6 +393,92 @@ def run_ours(args):
     return 0
 
 
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def run_zero1(args):
+    """The ZeRO-1 step: reduce-scatter (bf16, sum) -> the step kernel on the
+    rank's shard, one handle per chunk -> all-gather (fp32), chunked so the
+    collectives of one chunk run under the step of another.  value = the
+    workload's params / the max over ranks of the device time per step."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    ws_, rank, local = dist_setup(args.gpus)
+    if ws_ == 1:
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", 0))
+    import bit_quantized_optimizer_b200 as B
+    from bit_quantized_optimizer_b200.zero1 import FlatLayout, ZeroAdamW4
+    B.lib()  # fail loudly if the extension is missing
+    vcode = VCODES[args.vcode]
+    ts = workloads.tensor_list(WORKLOAD)
+    layout = FlatLayout([t["numel"] for t in ts], ws_, args.chunks)
+    fp = torch.empty(layout.padded, dtype=torch.float32, device="cuda")
+    fg = torch.zeros(layout.padded, dtype=torch.bfloat16, device="cuda")
+    # the same weights on every rank, each rank's own gradients
+    params, _ = workloads.device_inputs(WORKLOAD, ts, seed=0)
+    for i, p in enumerate(params):
+        layout.tensor_view(fp, i).copy_(p)
+    del params, _
+    _, grads = workloads.device_inputs(WORKLOAD, ts, seed=rank + 1)
+    for i, g in enumerate(grads):
+        layout.tensor_view(fg, i).copy_(g)
+    del grads, _
+    torch.cuda.synchronize()
+    opt = ZeroAdamW4(fp, fg, layout, ts, lr=1e-3, vcode=vcode, seed=0)
+    nparams = sum(t["numel"] for t in ts)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        opt.step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(ws_)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        opt.step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws_)
+    clk = clocks.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), ws_) / args.steps
+    launches = sum(1 for s_ in opt.steppers if s_ is not None)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": nparams / (ms * 1e-3) / 1e9, "unit": "Gparams/s",
+            "n_gpus": ws_, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "vcode": args.vcode, "params": nparams,
+                       "tensors": len(ts), "parallelism": f"zero1 x{ws_}",
+                       "chunks": args.chunks, "shard_elems_per_chunk": layout.shard,
+                       "reduce_scatter_bytes_per_rank": 2 * layout.padded,
+                       "all_gather_bytes_per_rank": 4 * layout.padded,
+                       "algorithmic_bytes_per_step": algorithmic_bytes(ts),
+                       "l2": "inputs 19.7 GB > 126 MB L2; no flush"},
+            "roofline": None,
+            "e2e": None,
+            "gpu_launches": args.steps * launches,
+            "clocks": clk,
+            "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    for s_ in opt.steppers:
+        if s_ is not None:
+            s_.close()
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,6 +489,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--bf16-params", action="store_true",
+                    help="keep every tensor's weights in bf16 (ADAMW4_T_BF16_PARAM)")
+    ap.add_argument("--zero1", action="store_true",
+                    help="time the ZeRO-1 sharded step (reduce-scatter, step, all-gather)")
+    ap.add_argument("--chunks", type=int, default=4,
+                    help="ZeRO-1 pipeline chunks (collectives of one overlap the step of another)")
     ap.add_argument("--workload", default=WORKLOAD, choices=["gpt-2.7b", "llama-1.1b", "gpt-130m"],
                     help="tensor list (the benchmark is gpt-2.7b; the others are profiling cases)")
     args = ap.parse_args()
@@ -390,6 +502,8 @@ def main():
     globals()["WORKLOAD"] = args.workload
     if args.impl == "reference":
         return run_reference(args)
+    if args.zero1:
+        return run_zero1(args)
     return run_ours(args)
 
 

@@ -14,7 +14,7 @@ import os
 
 __all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_V_ZI_RTN", "ADAMW4_V_ZI_SR",
            "ADAMW4_V_ZE_FLOOR", "ADAMW4_T_NORM", "ADAMW4_T_LM_HEAD",
-           "ADAMW4_T_FP32_STATE", "ADAMW4_T_QUANT_STATE", "AdamW4Error", "adamw4_tensor", "adamw4_config", "lib",
+           "ADAMW4_T_FP32_STATE", "ADAMW4_T_QUANT_STATE", "ADAMW4_T_BF16_PARAM", "AdamW4Error", "adamw4_tensor", "adamw4_config", "lib",
            "adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
            "adamw4_get_step", "adamw4_set_step", "adamw4_state_bytes", "adamw4_state_export",
            "adamw4_state_import", "adamw4_launch_info", "adamw4_last_error", "adamw4_sync",
@@ -34,6 +34,7 @@ ADAMW4_T_NORM = 1
 ADAMW4_T_LM_HEAD = 2
 ADAMW4_T_FP32_STATE = 4
 ADAMW4_T_QUANT_STATE = 8   # 4-bit state below 4096 elements (a piece of a larger tensor)
+ADAMW4_T_BF16_PARAM = 16   # bf16 weights (rounded to nearest even after each update)
 MIN_QUANT_NUMEL = 4096
 BLOCK = 128
 
@@ -207,10 +208,11 @@ def is_fp32_state(numel: int, flags: int) -> bool:
 
 
 class AdamW4:
-    """Optimizer over torch tensors: fp32 params and bf16 grads (contiguous,
-    16-byte aligned, on one CUDA device).  ``specs`` is a list of dicts with
-    tensor_id, flags, weight_decay and (for a piece of a larger tensor)
-    elem_offset, parallel to ``params``."""
+    """Optimizer over torch tensors: fp32 (or bf16) params and bf16 grads
+    (contiguous, 16-byte aligned, on one CUDA device).  ``specs`` is a list of
+    dicts with tensor_id, flags, weight_decay and (for a piece of a larger
+    tensor) elem_offset, parallel to ``params``.  A bf16 param sets
+    ADAMW4_T_BF16_PARAM for its tensor."""
 
     def __init__(self, params, grads, specs, lr=1e-3, betas=(0.9, 0.999), eps=1e-8,
                  vcode=ADAMW4_V_ZIPSR, seed=0, total_steps=0):
@@ -219,13 +221,15 @@ class AdamW4:
         dev = self.params[0].device.index if self.params else 0
         ts = []
         for p, g, s in zip(self.params, self.grads, specs):
-            if p.dtype != torch.float32 or g.dtype != torch.bfloat16:
-                raise TypeError("params must be float32 and grads bfloat16")
+            if p.dtype not in (torch.float32, torch.bfloat16) or g.dtype != torch.bfloat16:
+                raise TypeError("params must be float32 or bfloat16 and grads bfloat16")
             if not (p.is_contiguous() and g.is_contiguous()) or p.numel() != g.numel():
                 raise ValueError("params and grads must be contiguous and of equal size")
+            flags = int(s.get("flags", 0)) & ~ADAMW4_T_BF16_PARAM
+            if p.dtype == torch.bfloat16:
+                flags |= ADAMW4_T_BF16_PARAM
             ts.append(adamw4_tensor(p.data_ptr(), g.data_ptr(), p.numel(), s["tensor_id"],
-                                    s.get("flags", 0), s.get("weight_decay", 0.0),
-                                    s.get("elem_offset", 0)))
+                                    flags, s.get("weight_decay", 0.0), s.get("elem_offset", 0)))
         self.cfg = adamw4_config(lr, betas[0], betas[1], eps, vcode, seed, total_steps)
         self.lr = lr
         self.handle = adamw4_create(self.cfg, ts, dev)

@@ -85,6 +85,7 @@ constexpr int kVZe = ADAMW4_V_ZEEDEN;
 constexpr int kVZiRtn = ADAMW4_V_ZI_RTN;
 constexpr int kVZiSr = ADAMW4_V_ZI_SR;
 constexpr int kVZeFloor = ADAMW4_V_ZE_FLOOR;
+constexpr uint32_t kBf16W = ADAMW4_T_BF16_PARAM;  // weights stored as bf16
 constexpr uint32_t kKindFp32 = 1u << 16;          // internal flag: fp32-state tensor
 constexpr uint32_t kStaged = 1u << 17;            // internal flag: unit data is in the stage
 constexpr uint32_t kNoUnit = 1u << 18;            // internal flag: empty slot of the last tile
@@ -297,6 +298,19 @@ __device__ __forceinline__ void words8(const StepArgs& a, uint32_t tensor_id, ui
 
 __device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+// binary32 -> bf16, IEEE round to nearest even (the cvt instruction).  Two
+// values: lo in bits 0-15, hi in bits 16-31.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint16_t bf16_rn(float x) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+  return r;
+}
 __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
 // Max of non-negative binary32 values over a half-warp: their bit patterns
@@ -571,23 +585,38 @@ __device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, 
   }
 }
 
+// Weight i of a lane's run, fp32 or (BF16W and flagged) bf16.
+template <bool BF16W>
+__device__ __forceinline__ float load_w(const float* wp, const uint16_t* wp16, bool wbf, int i) {
+  if (BF16W && wbf) return __uint_as_float((uint32_t)wp16[i] << 16);
+  return wp[i];
+}
+template <bool BF16W>
+__device__ __forceinline__ void store_w(float* wp, uint16_t* wp16, bool wbf, int i, float x) {
+  if (BF16W && wbf) wp16[i] = bf16_rn(x);
+  else wp[i] = x;
+}
+
 // A unit read straight from global memory: a ragged last 4-bit block or a
 // chunk of an fp32-state tensor.
-template <int VCODE>
+template <int VCODE, bool BF16W>
 __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTables& S,
                                             const StateArena& st, const UnitHeader* hdp,
                                             int lane, unsigned hmask) {
   const int my0 = lane * kPerLane;
   const int myn = min(max(hdp->nvalid - my0, 0), kPerLane);
   const uint32_t flags = hdp->flags;
+  const bool wbf = BF16W && (flags & kBf16W);
   const float decay = hdp->decay;
   const uint64_t state = hdp->state;
-  float* wp = hdp->w + my0;
+  // the header's w is the unit's first weight, of either width
+  float* wp = wbf ? nullptr : hdp->w + my0;
+  uint16_t* wp16 = wbf ? reinterpret_cast<uint16_t*>(hdp->w) + my0 : nullptr;
   const uint16_t* gp = hdp->g + my0;
   float w[kPerLane], g[kPerLane];
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
-    w[i] = (i < myn) ? wp[i] : 0.0f;
+    w[i] = (i < myn) ? load_w<BF16W>(wp, wp16, wbf, i) : 0.0f;
     g[i] = (i < myn) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
   }
   if (flags & kKindFp32) {
@@ -599,7 +628,8 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
         const float m1 = __fmaf_rn(a.b1, mp[i], __fmul_rn(a.omb1, g[i]));
         const float v1 = __fmaf_rn(a.b2, vp[i], __fmul_rn(a.omb2, __fmul_rn(g[i], g[i])));
         const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
-        wp[i] = __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay));
+        store_w<BF16W>(wp, wp16, wbf, i,
+                       __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay)));
         mp[i] = m1;
         vp[i] = v1;
       }
@@ -613,7 +643,7 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
   update8(a, S, decay, w, g, *mcw, *vcw, st.mscale[blk], st.vscale[blk], m1, v1, den);
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i)
-    if (i < myn) wp[i] = w[i];
+    if (i < myn) store_w<BF16W>(wp, wp16, wbf, i, w[i]);
   requant_store<VCODE, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask, m1, v1,
                               den, mcw, vcw, st.mscale + blk, st.vscale + blk);
 }
@@ -623,6 +653,7 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
 // Lane i handles unit i of the tile (header, scales); the lane that starts a
 // run of whole 4-bit blocks of one tensor issues that run's bulk copies.
 // ---------------------------------------------------------------------------
+template <bool BF16W>
 __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t nunits,
                                         const StepArgs& a, const StateArena& st, uint8_t* stages,
                                         uint32_t full0, uint32_t empty0, int lane) {
@@ -666,9 +697,11 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     const int64_t e0 = ub * kBlock;
     const int nvalid = has ? (int)min((int64_t)kBlock, t_numel - e0) : 0;
     const bool staged = has && !(t_flags & kKindFp32) && nvalid == kBlock;
+    const bool wbf = BF16W && (t_flags & kBf16W);       // bf16 weights: 256 B per unit
     uint8_t* sp = stages + s * kStageBytes;
     UnitHeader* hd = reinterpret_cast<UnitHeader*>(sp + kOffHdr) + lane;
-    hd->w = t_param + e0;
+    hd->w = wbf ? reinterpret_cast<float*>(reinterpret_cast<uint16_t*>(t_param) + e0)
+                : t_param + e0;
     hd->g = t_grad + e0;
     hd->e0 = (uint64_t)(t_eoff + e0);   // keys the draws
     hd->state = (t_flags & kKindFp32) ? (uint64_t)(t_soff + e0) : (uint64_t)(t_soff + ub);
@@ -683,14 +716,19 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     const bool cont = staged && lane > 0 && ((staged_mask >> (lane - 1)) & 1u) && prev_ti == ti;
     const unsigned cont_mask = __ballot_sync(kMask, cont);
     const uint32_t dst = stages_s + (uint32_t)(s * kStageBytes);
-    if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)__popc(staged_mask) * kUnitTx);
+    uint32_t tx = (uint32_t)__popc(staged_mask) * kUnitTx;
+    if (BF16W) tx -= (uint32_t)__popc(__ballot_sync(kMask, staged && wbf)) * 256u;
+    if (lane == 0) mbar_arrive_expect_tx(full, tx);
+    if (BF16W && staged && wbf && !a.fault_stall)      // bf16 weights: one copy per unit
+      bulk_g2s(dst + kOffW + lane * 512, reinterpret_cast<const uint16_t*>(t_param) + e0, 256u,
+               full);
     if (staged && !cont && !a.fault_stall) {
       // this lane starts a run: it extends over the following lanes whose
       // unit continues it
       const unsigned rest = ~(cont_mask >> (lane + 1));
       const int len = __ffs(rest);          // 1 + number of continuing lanes
       const int64_t blk = t_soff + ub;
-      bulk_g2s(dst + kOffW + lane * 512, t_param + e0, 512u * len, full);
+      if (!wbf) bulk_g2s(dst + kOffW + lane * 512, t_param + e0, 512u * len, full);
       bulk_g2s(dst + kOffG + lane * 256, t_grad + e0, 256u * len, full);
       bulk_g2s(dst + kOffMC + lane * 64, st.mcodes + blk * (kBlock / 2), 64u * len, full);
       bulk_g2s(dst + kOffVC + lane * 64, st.vcodes + blk * (kBlock / 2), 64u * len, full);
@@ -715,7 +753,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
 // The step kernel
 // ---------------------------------------------------------------------------
 
-template <int VCODE>
+template <int VCODE, bool BF16W>
 __global__ void __launch_bounds__(kCtaThreads, 3)
 adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, CodeTables tabs,
                    StateArena st) {
@@ -758,7 +796,7 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
   const int warp = threadIdx.x >> 5;
   if (warp == kProducerWarp) {
     const int lane = threadIdx.x & 31;
-    if (lane < kHalves) produce(T, nunits, a, st, s_stage, full0, empty0, lane);
+    if (lane < kHalves) produce<BF16W>(T, nunits, a, st, s_stage, full0, empty0, lane);
     return;
   }
 
@@ -781,13 +819,20 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
     const uint32_t flags = hdp->flags;
     if (flags & kStaged) {
       float w[kPerLane], g[kPerLane];
+      const bool wbf = BF16W && (flags & kBf16W);
       {
-        const uint8_t* wsrc = sp + kOffW + half * 512 + lane * 32;
-        const float4 wa = *reinterpret_cast<const float4*>(wsrc);
-        const float4 wb = *reinterpret_cast<const float4*>(wsrc + 16);
         const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
-        w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
-        w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
+        if (wbf) {
+          const uint4 wr = *reinterpret_cast<const uint4*>(sp + kOffW + half * 512 + lane * 16);
+          w[0] = bf16lo(wr.x); w[1] = bf16hi(wr.x); w[2] = bf16lo(wr.y); w[3] = bf16hi(wr.y);
+          w[4] = bf16lo(wr.z); w[5] = bf16hi(wr.z); w[6] = bf16lo(wr.w); w[7] = bf16hi(wr.w);
+        } else {
+          const uint8_t* wsrc = sp + kOffW + half * 512 + lane * 32;
+          const float4 wa = *reinterpret_cast<const float4*>(wsrc);
+          const float4 wb = *reinterpret_cast<const float4*>(wsrc + 16);
+          w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
+          w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
+        }
         g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
         g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
       }
@@ -798,16 +843,22 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
 
       float m1[kPerLane], v1[kPerLane], den[kPerLane];
       update8(a, S, hdp->decay, w, g, mc, vc, sm, sv, m1, v1, den);
-      float* wp = hdp->w + lane * kPerLane;
-      *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
+      if (wbf) {
+        uint16_t* wp = reinterpret_cast<uint16_t*>(hdp->w) + lane * kPerLane;
+        *reinterpret_cast<uint4*>(wp) = make_uint4(bf16x2_rn(w[0], w[1]), bf16x2_rn(w[2], w[3]),
+                                                   bf16x2_rn(w[4], w[5]), bf16x2_rn(w[6], w[7]));
+      } else {
+        float* wp = hdp->w + lane * kPerLane;
+        *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
+      }
       const uint64_t blk = hdp->state;
       uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
       uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
       requant_store<VCODE, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, kPerLane, hmask, m1,
                                  v1, den, mcw, vcw, st.mscale + blk, st.vscale + blk);
     } else if (!(flags & kNoUnit)) {
-      process_direct<VCODE>(a, S, st, hdp, lane, hmask);
+      process_direct<VCODE, BF16W>(a, S, st, hdp, lane, hmask);
     }
     // every read of the stage (header included) is done: hand it back
     fence_proxy_async_smem();
@@ -845,6 +896,7 @@ struct adamw4_handle {
   int64_t nblocks4 = 0;       // 4-bit blocks
   int64_t nfp32 = 0;          // fp32 arena elements (with alignment)
   int64_t nunits = 0;
+  bool bf16w = false;             // some tensor keeps bf16 weights
   int grid = 0;
   uint32_t* d_status = nullptr;   // device status word (in the arena)
   int fault_stall = 0;            // test hook for the next step
@@ -973,8 +1025,11 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-constexpr uint32_t kUserFlags =
-    ADAMW4_T_NORM | ADAMW4_T_LM_HEAD | ADAMW4_T_FP32_STATE | ADAMW4_T_QUANT_STATE;
+constexpr uint32_t kUserFlags = ADAMW4_T_NORM | ADAMW4_T_LM_HEAD | ADAMW4_T_FP32_STATE |
+                                ADAMW4_T_QUANT_STATE | ADAMW4_T_BF16_PARAM;
+
+// Bytes of one weight of tensor t.
+uintptr_t param_bytes(const adamw4_tensor& t) { return (t.flags & ADAMW4_T_BF16_PARAM) ? 2u : 4u; }
 
 // fp32 state for normalisation tensors, tensors flagged FP32_STATE and tensors
 // under 4096 elements -- unless QUANT_STATE marks a piece of a larger tensor
@@ -1044,7 +1099,7 @@ int validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n) {
       return fail(nullptr, ADAMW4_EINVAL, at + "duplicate tensor_id " + std::to_string(t.tensor_id));
     const uintptr_t p = reinterpret_cast<uintptr_t>(t.param);
     const uintptr_t g = reinterpret_cast<uintptr_t>(t.grad_bf16);
-    ranges.push_back({p, p + (uintptr_t)t.numel * 4u, i, true});
+    ranges.push_back({p, p + (uintptr_t)t.numel * param_bytes(t), i, true});
     ranges.push_back({g, g + (uintptr_t)t.numel * 2u, i, false});
   }
   // Params are written in place: no param may overlap another param or a grad.
@@ -1067,54 +1122,71 @@ int validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n) {
   return ADAMW4_OK;
 }
 
-template <int VCODE>
+template <int VCODE, bool BF16W>
 int occupancy_grid(int device, int* grid) {
   int sms = 0, per_sm = 0;
   cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
   if (e != cudaSuccess) return (int)e;
   // The stage rings live in dynamic shared memory above the 48 KB default.
-  e = cudaFuncSetAttribute(adamw4_step_kernel<VCODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemStages);
+  e = cudaFuncSetAttribute(adamw4_step_kernel<VCODE, BF16W>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemStages);
   if (e != cudaSuccess) return (int)e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adamw4_step_kernel<VCODE>,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adamw4_step_kernel<VCODE, BF16W>,
                                                     kCtaThreads, kSmemStages);
   if (e != cudaSuccess) return (int)e;
   *grid = sms * std::max(per_sm, 1);
   return 0;
 }
 
-// The launch grid (SM count x resident CTAs) of the instantiation for vcode.
-int grid_for(int vcode, int device, int* grid) {
+template <bool BF16W>
+int grid_for_w(int vcode, int device, int* grid) {
   switch (vcode) {
-    case kVZip: return occupancy_grid<kVZip>(device, grid);
-    case kVZe: return occupancy_grid<kVZe>(device, grid);
-    case kVZiRtn: return occupancy_grid<kVZiRtn>(device, grid);
-    case kVZiSr: return occupancy_grid<kVZiSr>(device, grid);
-    case kVZeFloor: return occupancy_grid<kVZeFloor>(device, grid);
+    case kVZip: return occupancy_grid<kVZip, BF16W>(device, grid);
+    case kVZe: return occupancy_grid<kVZe, BF16W>(device, grid);
+    case kVZiRtn: return occupancy_grid<kVZiRtn, BF16W>(device, grid);
+    case kVZiSr: return occupancy_grid<kVZiSr, BF16W>(device, grid);
+    case kVZeFloor: return occupancy_grid<kVZeFloor, BF16W>(device, grid);
     default: return (int)cudaErrorInvalidValue;
   }
 }
 
-// Enqueues the step kernel instantiated for vcode.
-void launch_vcode(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t nunits,
-                  const StepArgs& a, const CodeTables& tabs, const StateArena& st) {
+// The launch grid (SM count x resident CTAs) of the instantiation for vcode,
+// with (bf16w) or without support for bf16 weights.
+int grid_for(int vcode, bool bf16w, int device, int* grid) {
+  return bf16w ? grid_for_w<true>(vcode, device, grid) : grid_for_w<false>(vcode, device, grid);
+}
+
+template <bool BF16W>
+void launch_w(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t nunits,
+              const StepArgs& a, const CodeTables& tabs, const StateArena& st) {
+  const int n = kCtaThreads;
+  const int smem = kSmemStages;
   switch (vcode) {
     case kVZip:
-      adamw4_step_kernel<kVZip><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZip, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
       break;
     case kVZe:
-      adamw4_step_kernel<kVZe><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZe, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
       break;
     case kVZiRtn:
-      adamw4_step_kernel<kVZiRtn><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZiRtn, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
       break;
     case kVZiSr:
-      adamw4_step_kernel<kVZiSr><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZiSr, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
       break;
     default:
-      adamw4_step_kernel<kVZeFloor><<<grid, kCtaThreads, kSmemStages, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZeFloor, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
       break;
   }
+}
+
+// Enqueues the step kernel instantiated for vcode; bf16w selects the
+// instantiation that reads and writes bf16 weights where a tensor asks for it.
+void launch_vcode(int vcode, bool bf16w, int grid, cudaStream_t s, const DevTensor* T,
+                  int64_t nunits, const StepArgs& a, const CodeTables& tabs,
+                  const StateArena& st) {
+  if (bf16w) launch_w<true>(vcode, grid, s, T, nunits, a, tabs, st);
+  else launch_w<false>(vcode, grid, s, T, nunits, a, tabs, st);
 }
 
 int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
@@ -1124,7 +1196,7 @@ int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
   a.status = h->d_status;
   a.fault_stall = h->fault_stall;
   h->fault_stall = 0;
-  launch_vcode(h->cfg.vcode, grid, s, h->d_tensors, h->nunits, a, h->tabs, h->st);
+  launch_vcode(h->cfg.vcode, h->bf16w, grid, s, h->d_tensors, h->nunits, a, h->tabs, h->st);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(h, e, "step kernel launch");
   return ADAMW4_OK;
@@ -1169,6 +1241,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
     HostTensor ht{};
     ht.desc = tensors[i];
     ht.fp32 = fp32_state(tensors[i]);
+    if (tensors[i].flags & ADAMW4_T_BF16_PARAM) h->bf16w = true;
     ht.nblocks = (tensors[i].numel + kBlock - 1) / kBlock;
     if (ht.fp32) {
       ht.state_off = h->nfp32;
@@ -1235,7 +1308,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
     delete h;
     return cuda_fail(nullptr, e, "initialising the state");
   }
-  int ge = grid_for(cfg->vcode, device, &h->grid);
+  int ge = grid_for(cfg->vcode, h->bf16w, device, &h->grid);
   if (ge != 0) {
     release(h);
     delete h;
@@ -1285,7 +1358,7 @@ extern "C" int adamw4_step_host(adamw4_handle* h, float lr, const uint16_t* cons
     for (size_t i = 0; i < h->tensors.size(); ++i) {
       const adamw4_tensor& d = h->tensors[i].desc;
       if (params_host[i] == nullptr) return fail(h, ADAMW4_EINVAL, "params_host entry is NULL");
-      e = cudaMemcpyAsync(params_host[i], d.param, (size_t)d.numel * sizeof(float),
+      e = cudaMemcpyAsync(params_host[i], d.param, (size_t)d.numel * param_bytes(d),
                           cudaMemcpyDeviceToHost, s);
       if (e != cudaSuccess) return cuda_fail(h, e, "copying params to the host");
     }
@@ -1520,7 +1593,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 struct NoAllocDevice {
   bool ready;
   unsigned char* scratch;   // device address of g_noalloc_scratch on this device
-  int grid[ADAMW4_V_ZE_FLOOR + 1];   // per vcode
+  int grid[ADAMW4_V_ZE_FLOOR + 1][2];   // per vcode, without / with bf16 weights
 };
 
 std::mutex g_noalloc_mu;
@@ -1551,13 +1624,15 @@ int na_validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n,
         x.numel > ((int64_t)1 << 40) || !std::isfinite(x.weight_decay) || piece_error(x) != nullptr)
       return ADAMW4_EINVAL;
     if (!na_aligned(x.param, 16) || !na_aligned(x.grad_bf16, 16)) return ADAMW4_EALIGN;
-    const uintptr_t p0 = reinterpret_cast<uintptr_t>(x.param), p1 = p0 + (uintptr_t)x.numel * 4u;
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(x.param),
+                    p1 = p0 + (uintptr_t)x.numel * param_bytes(x);
     const uintptr_t g0 = reinterpret_cast<uintptr_t>(x.grad_bf16), g1 = g0 + (uintptr_t)x.numel * 2u;
     if (p0 < g1 && g0 < p1) return ADAMW4_EINVAL;                 // own grad
     for (int k = 0; k < i; ++k) {
       const adamw4_tensor& y = ts[k];
       if (y.tensor_id == x.tensor_id) return ADAMW4_EINVAL;
-      const uintptr_t q0 = reinterpret_cast<uintptr_t>(y.param), q1 = q0 + (uintptr_t)y.numel * 4u;
+      const uintptr_t q0 = reinterpret_cast<uintptr_t>(y.param),
+                      q1 = q0 + (uintptr_t)y.numel * param_bytes(y);
       const uintptr_t h0 = reinterpret_cast<uintptr_t>(y.grad_bf16), h1 = h0 + (uintptr_t)y.numel * 2u;
       if ((p0 < q1 && q0 < p1) || (p0 < h1 && h0 < p1) || (q0 < g1 && g0 < q1))
         return ADAMW4_EINVAL;                                     // a param overlaps
@@ -1586,14 +1661,17 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
         cudaSuccess)
       return ADAMW4_ECUDA;
     for (int vc = ADAMW4_V_ZIPSR; vc <= ADAMW4_V_ZE_FLOOR; ++vc)
-      if (grid_for(vc, device, &nd.grid[vc]) != 0) return ADAMW4_ECUDA;
+      for (int bw = 0; bw < 2; ++bw)
+        if (grid_for(vc, bw != 0, device, &nd.grid[vc][bw]) != 0) return ADAMW4_ECUDA;
     nd.ready = true;
   }
   // The table adamw4_create would build, in the same order and layout.
   int64_t unit = 0, blocks4 = 0, elems32 = 0;
+  int bf16w = 0;
   for (int i = 0; i < n; ++i) {
     const adamw4_tensor& x = tensors[i];
     const bool fp32 = fp32_state(x);
+    if (x.flags & ADAMW4_T_BF16_PARAM) bf16w = 1;
     const int64_t nb = (x.numel + kBlock - 1) / kBlock;
     g_noalloc_table[i] = dev_tensor(x, fp32, unit, fp32 ? elems32 : blocks4);
     if (fp32) elems32 += nb * kBlock; else blocks4 += nb;
@@ -1623,7 +1701,7 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   st.fm = state->m32;
   st.fv = state->v32;
   const int64_t need = (unit + kHalves - 1) / kHalves;
-  launch_vcode(cfg->vcode, (int)std::min<int64_t>(nd.grid[cfg->vcode], need), s, table, unit, a,
-               tabs, st);
+  launch_vcode(cfg->vcode, bf16w, (int)std::min<int64_t>(nd.grid[cfg->vcode][bf16w], need), s,
+               table, unit, a, tabs, st);
   return cudaGetLastError() == cudaSuccess ? ADAMW4_OK : ADAMW4_ECUDA;
 }

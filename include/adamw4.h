@@ -83,8 +83,9 @@ enum {
     ADAMW4_T_NORM = 1u,       /* normalisation-layer tensor: fp32 state        */
     ADAMW4_T_LM_HEAD = 2u,    /* LM head: m rounded stochastically in the final 10% */
     ADAMW4_T_FP32_STATE = 4u, /* force fp32 state                              */
-    ADAMW4_T_QUANT_STATE = 8u /* force 4-bit state below 4096 elements: a piece of a
-                                 larger 4-bit tensor (not with NORM / FP32_STATE) */
+    ADAMW4_T_QUANT_STATE = 8u, /* force 4-bit state below 4096 elements: a piece of a
+                                  larger 4-bit tensor (not with NORM / FP32_STATE) */
+    ADAMW4_T_BF16_PARAM = 16u  /* the weights are bf16, not fp32 (see adamw4_tensor) */
 };
 
 /* Tensors below this many elements keep fp32 state. */
@@ -93,7 +94,14 @@ enum {
 #define ADAMW4_BLOCK 128
 
 /* One parameter tensor, flattened row-major, or a piece of one.
- *   param      device, fp32, numel elements, 16-byte aligned; updated in place
+ *   param      device, fp32, numel elements, 16-byte aligned; updated in place.
+ *              With ADAMW4_T_BF16_PARAM it holds numel bf16 bit patterns
+ *              instead (pass it cast to float*): the step reads them exactly,
+ *              computes the update in binary32 as for fp32 weights, and stores
+ *              the result rounded to the nearest bf16 (ties to even).  Updates
+ *              below half a bf16 ulp of a weight are then lost; the pages keep
+ *              no bf16 weights, this is a lower-memory option (2 B/param less
+ *              read and written per step).
  *   grad_bf16  device, bf16 bit patterns, numel elements, 16-byte aligned; read
  *   tensor_id  unique within a handle; keys the random draws, so it must stay
  *              the same across a checkpoint and resume
@@ -161,7 +169,8 @@ int adamw4_step(adamw4_handle *h, float lr, void *cuda_stream);
  * (numel bf16) to the tensor's device grad buffer, runs adamw4_step, then
  * copies the updated params back to params_host[i] (numel fp32), all on
  * `cuda_stream`, and waits for the stream.  Pinned host memory gives
- * asynchronous copies; pageable memory works but is slower.
+ * asynchronous copies; pageable memory works but is slower.  A tensor flagged
+ * ADAMW4_T_BF16_PARAM copies back numel bf16 values (2 bytes each).
  * Either array may be NULL to skip that direction. */
 int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_host,
                      float *const *params_host, void *cuda_stream);

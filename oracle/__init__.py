@@ -37,6 +37,7 @@ VCODE_ZE_FLOOR = 4    # zero-excluded code, no rescale
 T_NORM = 1
 T_LM_HEAD = 2
 T_FP32_STATE = 4
+T_BF16_PARAM = 16      # weights stored as bf16 (a library option, not the pages')
 STREAM_V = 0
 STREAM_M = 1
 
@@ -115,6 +116,9 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
                                       c.c_int64, c.c_int64, _i64p, _f32p, _u16p, _u8p,
                                       _f32p, _u8p, _f32p]
     L.oracle_step_fp32.argtypes = [S, c.c_float, c.c_int64, _f32p, _u16p, _f32p, _f32p]
+    L.oracle_f32_to_bf16.restype = c.c_uint16
+    L.oracle_f32_to_bf16.argtypes = [c.c_float]
+    L.oracle_round_bf16.argtypes = [_f32p, _u16p, c.c_int64]
     L.oracle_max_threads.restype = c.c_int
     return L
 
@@ -261,11 +265,24 @@ def is_fp32_state(numel: int, flags: int) -> bool:
     return numel < MIN_QUANT_NUMEL or bool(flags & (T_NORM | T_FP32_STATE))
 
 
+def f32_to_bf16(x: float) -> int:
+    return int(lib().oracle_f32_to_bf16(x))
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """binary32 array -> bf16 bit patterns (nearest, ties to even)."""
+    x = np.ascontiguousarray(x, np.float32)
+    out = np.empty(x.size, np.uint16)
+    lib().oracle_round_bf16(x, out, x.size)
+    return out
+
+
 class TensorState:
     def __init__(self, numel: int, tensor_id: int, flags: int, weight_decay: float):
         self.numel = int(numel)
         self.tensor_id = int(tensor_id)
         self.flags = int(flags)
+        self.bf16w = bool(self.flags & T_BF16_PARAM)
         self.weight_decay = float(weight_decay)
         self.fp32 = is_fp32_state(self.numel, self.flags)
         if self.fp32:
@@ -317,14 +334,21 @@ class OracleAdamW4:
     def step(self, params, grads, lr=None, only=None, advance=True):
         """One step over every tensor, or over the tensors listed in `only`
         (then params/grads hold just those, in that order).  With
-        advance=False the step counter is not incremented first."""
+        advance=False the step counter is not incremented first.  The params
+        of a T_BF16_PARAM tensor are uint16 arrays of bf16 bit patterns: read
+        exactly, stepped in binary32, stored rounded to the nearest bf16."""
         L = lib()
         if advance:
             self.t += 1
         s = self.scalars(self.lr if lr is None else lr)
         idx = range(len(self.tensors)) if only is None else list(only)
-        for i, w, g in zip(idx, params, grads):
+        for i, w_in, g in zip(idx, params, grads):
             ts = self.tensors[i]
+            if ts.bf16w:
+                assert w_in.dtype == np.uint16
+                w = (w_in.astype(np.uint32) << 16).view(np.float32)
+            else:
+                w = w_in
             assert w.dtype == np.float32 and g.dtype == np.uint16 and w.size == ts.numel
             if ts.fp32:
                 L.oracle_step_fp32(ctypes.byref(s), ts.weight_decay, ts.numel, w, g, ts.m, ts.v)
@@ -332,6 +356,8 @@ class OracleAdamW4:
                 L.oracle_step_tensor4(ctypes.byref(s), ts.weight_decay, self.vcode,
                                       self.m_sr(ts, s), ts.tensor_id, ts.numel, w, g,
                                       ts.mcodes, ts.mscale, ts.vcodes, ts.vscale, self.nthreads)
+            if ts.bf16w:
+                w_in[:] = round_bf16(w)
 
     def step_blocks(self, index: int, blocks, w_sel, g_sel, mc_sel, ms_sel, vc_sel, vs_sel,
                     lr=None, advance=True):
@@ -343,6 +369,7 @@ class OracleAdamW4:
             self.t += 1
         s = self.scalars(self.lr if lr is None else lr)
         ts = self.tensors[index]
+        assert not ts.bf16w, "step_blocks takes fp32 weights"
         blocks = np.ascontiguousarray(blocks, np.int64)
         L.oracle_step_blocks4(ctypes.byref(s), ts.weight_decay, self.vcode, self.m_sr(ts, s),
                               ts.tensor_id, ts.numel, len(blocks), blocks, w_sel, g_sel, mc_sel,

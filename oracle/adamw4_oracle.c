@@ -241,6 +241,27 @@ static float bf16_to_f32(uint16_t h)
     return f;
 }
 
+/* Storage of bf16 weights (the library's lower-memory option; the pages keep
+ * fp32 weights).  binary32 -> bf16 rounded to nearest, ties to even, the IEEE
+ * 754 rounding: keep the top 16 bits after adding 0x7FFF plus the lowest kept
+ * bit, so that a value exactly halfway moves to the even neighbour and
+ * anything above halfway carries into the kept bits (an overflow of the
+ * largest finite values carries into the infinity pattern, as rounding must).
+ * A NaN stays a NaN. */
+uint16_t oracle_f32_to_bf16(float x)
+{
+    uint32_t b;
+    memcpy(&b, &x, 4);
+    if ((b & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((b >> 16) | 0x0040u);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return (uint16_t)(b >> 16);
+}
+
+void oracle_round_bf16(const float *x, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16(x[i]);
+}
+
 static int nibble(const uint8_t *codes, int i)
 {
     return (i & 1) ? (codes[i >> 1] >> 4) : (codes[i >> 1] & 15);

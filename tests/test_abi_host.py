@@ -69,7 +69,7 @@ def test_bad_config(L, kw, code):
     (B.adamw4_tensor(P0, P0 + (1 << 30), 0, 0, 0, 0.0), -1, "numel"),
     (B.adamw4_tensor(P0, P0 + (1 << 30), -5, 0, 0, 0.0), -1, "numel"),
     (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, float("inf")), -1, "weight_decay"),
-    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 16, 0.0), -1, "unknown flag"),
+    (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 32, 0.0), -1, "unknown flag"),
     (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 1 << 16, 0.0), -1, "unknown flag"),
     (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 8 | 1, 0.0), -1, "QUANT_STATE"),
     (B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 8 | 4, 0.0), -1, "QUANT_STATE"),
@@ -140,3 +140,19 @@ def test_piece_descriptors_pass_validation(L):
 def test_descriptor_layout_matches_the_header():
     assert ctypes.sizeof(B.adamw4_tensor) == 48
     assert B.adamw4_tensor.elem_offset.offset == 40
+
+
+def test_bf16_params_span_two_bytes_per_weight(L):
+    """A bf16 weight tensor of 4096 values ends 8 KB after its start; the same
+    tensor with fp32 weights would overlap a param placed there."""
+    b = B.adamw4_tensor(P0 + 8192, P0 + (1 << 31), 4096, 2, 16, 0.0)
+    a32 = B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 1, 0, 0.0)
+    rc, _ = _create(_cfg(), [a32, b])
+    assert rc == -1 and "overlaps" in B.adamw4_last_error()
+    a16 = B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 1, 16, 0.0)
+    os.environ["ADAMW4_FAIL_ALLOC"] = "1"
+    try:
+        rc, _ = _create(_cfg(), [a16, b])
+    finally:
+        del os.environ["ADAMW4_FAIL_ALLOC"]
+    assert rc == -3 and "injected" in B.adamw4_last_error()

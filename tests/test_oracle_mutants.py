@@ -10,6 +10,7 @@ import os
 import pytest
 
 import oracle
+import test_oracle_bf16 as BF
 import test_oracle_driver as D
 import test_oracle_nf4 as N
 import test_oracle_philox as P
@@ -51,6 +52,8 @@ def pins(golden):
                                          for x in (0.01, 0.2, 0.77)]),
         ("worked example, state space", lambda: V.test_worked_example_state_space_rounding(golden)),
         ("floor code", V.test_ze_floor_is_nearest_zero_excluded_without_rescale),
+        ("bf16 library", BF.test_round_matches_the_library_conversion),
+        ("bf16 nearest", BF.test_round_is_the_nearest_bf16_by_brute_force),
     ]
 
 
@@ -98,6 +101,8 @@ MUTANTS = [
     ("ZE-EDEN factor inverted", "return sxx / fmaxf(sxq, 1e-12f);",
      "return sxq / fmaxf(sxx, 1e-12f);"),
     ("final 10% off by one", "(10 * t > 9 * total_steps)", "(10 * t >= 9 * total_steps)"),
+    ("bf16 ties rounded up", "b += 0x7FFFu + ((b >> 16) & 1u);", "b += 0x8000u;"),
+    ("bf16 truncated", "b += 0x7FFFu + ((b >> 16) & 1u);", "b += 0u;"),
     ("nibble order swapped",
      "return (i & 1) ? (codes[i >> 1] >> 4) : (codes[i >> 1] & 15);",
      "return (i & 1) ? (codes[i >> 1] & 15) : (codes[i >> 1] >> 4);"),

@@ -122,3 +122,71 @@ def test_noalloc_rejects_too_many_tensors():
     with pytest.raises(B.AdamW4Error) as err:
         B.adamw4_step_noalloc(cfg, descs, sb, 1, 1e-3, 0, None)
     assert err.value.code == -6
+
+
+def test_noalloc_bf16_weights_and_pieces():
+    """The same descriptor fields as the handle path: bf16 weights and a piece
+    of a tensor (elem_offset, QUANT_STATE) give the handle step's bits."""
+    import torch
+    B = binding()
+    BF, Q = B.ADAMW4_T_BF16_PARAM, B.ADAMW4_T_QUANT_STATE
+    ts = [dict(numel=128 * 90 + 5, tensor_id=1, flags=BF, weight_decay=0.1, elem_offset=0),
+          dict(numel=1280, tensor_id=2, flags=Q, weight_decay=0.1, elem_offset=128 * 700),
+          dict(numel=5000, tensor_id=3, flags=BF | workloads.T_NORM, weight_decay=0.0,
+               elem_offset=0)]
+    dev = torch.device("cuda", 0)
+    rng = np.random.default_rng(5)
+
+    def make_params():
+        out = []
+        for t in ts:
+            w = torch.from_numpy((np.random.default_rng(t["tensor_id"]).standard_normal(
+                t["numel"]) * 0.02).astype(np.float32)).to(dev)
+            out.append(w.to(torch.bfloat16) if t["flags"] & BF else w)
+        return out
+    grads = [workloads.bf16_bits((rng.standard_normal(t["numel"]) * 1e-3).astype(np.float32))
+             for t in ts]
+    gbuf = [torch.from_numpy(g.view(np.int16)).to(dev).view(torch.bfloat16) for g in grads]
+
+    params = make_params()
+    opt = B.AdamW4(params, gbuf, ts, vcode=0, seed=3)
+    opt.step()
+    torch.cuda.synchronize()
+    ref = [p.view(torch.int16).cpu().numpy() if p.dtype == torch.bfloat16 else p.cpu().numpy()
+           for p in params]
+    ref_blob = opt.state_dict_blob()
+    opt.close()
+
+    params2 = make_params()
+    nb4 = sum((t["numel"] + 127) // 128 for t in ts if not t["flags"] & workloads.T_NORM)
+    n32 = 5120
+    bufs = [torch.zeros(nb4 * 64, dtype=torch.uint8, device=dev),
+            torch.zeros(nb4 * 64, dtype=torch.uint8, device=dev),
+            torch.zeros(nb4, dtype=torch.float32, device=dev),
+            torch.zeros(nb4, dtype=torch.float32, device=dev),
+            torch.zeros(n32, dtype=torch.float32, device=dev),
+            torch.zeros(n32, dtype=torch.float32, device=dev)]
+    sb = B.adamw4_state_buffers(*[b.data_ptr() for b in bufs])
+    cfg = B.adamw4_config(1e-3, 0.9, 0.999, 1e-8, 0, 3, 0)
+    descs = [B.adamw4_tensor(p.data_ptr(), g.data_ptr(), t["numel"], t["tensor_id"], t["flags"],
+                             t["weight_decay"], t["elem_offset"])
+             for p, g, t in zip(params2, gbuf, ts)]
+    B.adamw4_step_noalloc(cfg, descs, sb, 1, 1e-3, 0, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    for i, p in enumerate(params2):
+        got = p.view(torch.int16).cpu().numpy() if p.dtype == torch.bfloat16 else p.cpu().numpy()
+        assert got.tobytes() == ref[i].tobytes(), f"tensor {i}"
+    st = parse_blob(ref_blob)["tensors"]
+    mc, vc, ms, vs, m32, v32 = (b.cpu().numpy() for b in bufs)
+    b4 = 0
+    for t, r in zip(ts, st):
+        if r["fp32"]:
+            assert r["m"].tobytes() == m32[:t["numel"]].tobytes()
+            assert r["v"].tobytes() == v32[:t["numel"]].tobytes()
+            continue
+        nb = (t["numel"] + 127) // 128
+        assert r["mcodes"].tobytes() == mc[b4 * 64:(b4 + nb) * 64].tobytes()
+        assert r["vcodes"].tobytes() == vc[b4 * 64:(b4 + nb) * 64].tobytes()
+        assert r["mscale"].tobytes() == ms[b4:b4 + nb].tobytes()
+        assert r["vscale"].tobytes() == vs[b4:b4 + nb].tobytes()
+        b4 += nb
