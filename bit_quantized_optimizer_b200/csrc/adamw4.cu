@@ -654,11 +654,12 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
 // run of whole 4-bit blocks of one tensor issues that run's bulk copies.
 // ---------------------------------------------------------------------------
 template <bool BF16W>
-__device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t nunits,
-                                        const StepArgs& a, const StateArena& st, uint8_t* stages,
-                                        uint32_t full0, uint32_t empty0, int lane) {
+__device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t u_begin,
+                                        int64_t u_end, const StepArgs& a, const StateArena& st,
+                                        uint8_t* stages, uint32_t full0, uint32_t empty0,
+                                        int lane) {
   constexpr unsigned kMask = (1u << kHalves) - 1u;
-  const int64_t ntiles = (nunits + kHalves - 1) / kHalves;
+  const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
   int ti = -1;
   int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0, t_eoff = 0;
   float* t_param = nullptr;
@@ -675,8 +676,8 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
       if (lane == 0) atomicOr(a.status, 1u);
       return;
     }
-    const int64_t u = tile * kHalves + lane;
-    const bool has = u < nunits;
+    const int64_t u = u_begin + tile * kHalves + lane;
+    const bool has = u < u_end;
     if (has && u >= t_end) {
       do {
         ++ti;
@@ -755,8 +756,8 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
 
 template <int VCODE, bool BF16W>
 __global__ void __launch_bounds__(kCtaThreads, 3)
-adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, CodeTables tabs,
-                   StateArena st) {
+adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_end, StepArgs a,
+                   CodeTables tabs, StateArena st) {
   extern __shared__ __align__(128) uint8_t s_stage[];
   __shared__ __align__(8) uint64_t s_full[kStages];
   __shared__ __align__(8) uint64_t s_empty[kStages];
@@ -796,7 +797,7 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
   const int warp = threadIdx.x >> 5;
   if (warp == kProducerWarp) {
     const int lane = threadIdx.x & 31;
-    if (lane < kHalves) produce<BF16W>(T, nunits, a, st, s_stage, full0, empty0, lane);
+    if (lane < kHalves) produce<BF16W>(T, u_begin, u_end, a, st, s_stage, full0, empty0, lane);
     return;
   }
 
@@ -804,7 +805,7 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t nunits, StepArgs a, 
   const int lane = threadIdx.x & 15;
   const int half = threadIdx.x >> 4;
   const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
-  const int64_t ntiles = (nunits + kHalves - 1) / kHalves;
+  const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
   int s = 0;
   uint32_t parity = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -880,6 +881,7 @@ struct HostTensor {
   bool fp32;
   int64_t nblocks;      // 4-bit: blocks; fp32: 128-element chunks
   int64_t state_off;    // 4-bit: first block; fp32: first element
+  int64_t unit_begin;   // its first unit in the flat unit list
 };
 
 }  // namespace
@@ -899,6 +901,9 @@ struct adamw4_handle {
   bool bf16w = false;             // some tensor keeps bf16 weights
   int grid = 0;
   uint32_t* d_status = nullptr;   // device status word (in the arena)
+  cudaStream_t s_in = nullptr;    // adamw4_step_host: host-to-device copies
+  cudaStream_t s_out = nullptr;   // adamw4_step_host: device-to-host copies
+  std::vector<cudaEvent_t> events;
   int fault_stall = 0;            // test hook for the next step
   CodeTables tabs{};
   std::string err;
@@ -1157,46 +1162,48 @@ int grid_for(int vcode, bool bf16w, int device, int* grid) {
 }
 
 template <bool BF16W>
-void launch_w(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t nunits,
+void launch_w(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t u0, int64_t u1,
               const StepArgs& a, const CodeTables& tabs, const StateArena& st) {
   const int n = kCtaThreads;
   const int smem = kSmemStages;
   switch (vcode) {
     case kVZip:
-      adamw4_step_kernel<kVZip, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZip, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
       break;
     case kVZe:
-      adamw4_step_kernel<kVZe, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZe, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
       break;
     case kVZiRtn:
-      adamw4_step_kernel<kVZiRtn, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZiRtn, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
       break;
     case kVZiSr:
-      adamw4_step_kernel<kVZiSr, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZiSr, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
       break;
     default:
-      adamw4_step_kernel<kVZeFloor, BF16W><<<grid, n, smem, s>>>(T, nunits, a, tabs, st);
+      adamw4_step_kernel<kVZeFloor, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
       break;
   }
 }
 
-// Enqueues the step kernel instantiated for vcode; bf16w selects the
-// instantiation that reads and writes bf16 weights where a tensor asks for it.
+// Enqueues the step kernel instantiated for vcode over units [u0, u1) of the
+// table; bf16w selects the instantiation that reads and writes bf16 weights
+// where a tensor asks for it.
 void launch_vcode(int vcode, bool bf16w, int grid, cudaStream_t s, const DevTensor* T,
-                  int64_t nunits, const StepArgs& a, const CodeTables& tabs,
+                  int64_t u0, int64_t u1, const StepArgs& a, const CodeTables& tabs,
                   const StateArena& st) {
-  if (bf16w) launch_w<true>(vcode, grid, s, T, nunits, a, tabs, st);
-  else launch_w<false>(vcode, grid, s, T, nunits, a, tabs, st);
+  if (bf16w) launch_w<true>(vcode, grid, s, T, u0, u1, a, tabs, st);
+  else launch_w<false>(vcode, grid, s, T, u0, u1, a, tabs, st);
 }
 
-int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
-  if (h->nunits == 0) return ADAMW4_OK;
-  const int64_t need = (h->nunits + kHalves - 1) / kHalves;
+// One launch over units [u0, u1) of the handle's list.
+int launch(adamw4_handle* h, StepArgs a, cudaStream_t s, int64_t u0, int64_t u1) {
+  if (u1 <= u0) return ADAMW4_OK;
+  const int64_t need = (u1 - u0 + kHalves - 1) / kHalves;
   const int grid = (int)std::min<int64_t>(h->grid, need);
   a.status = h->d_status;
   a.fault_stall = h->fault_stall;
   h->fault_stall = 0;
-  launch_vcode(h->cfg.vcode, h->bf16w, grid, s, h->d_tensors, h->nunits, a, h->tabs, h->st);
+  launch_vcode(h->cfg.vcode, h->bf16w, grid, s, h->d_tensors, u0, u1, a, h->tabs, h->st);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(h, e, "step kernel launch");
   return ADAMW4_OK;
@@ -1205,8 +1212,24 @@ int launch(adamw4_handle* h, StepArgs a, cudaStream_t s) {
 void release(adamw4_handle* h) {
   if (h->d_tensors) cudaFree(h->d_tensors);
   if (h->d_arena) cudaFree(h->d_arena);
+  for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
+  if (h->s_in) cudaStreamDestroy(h->s_in);
+  if (h->s_out) cudaStreamDestroy(h->s_out);
   h->d_tensors = nullptr;
   h->d_arena = nullptr;
+  h->events.clear();
+  h->s_in = h->s_out = nullptr;
+}
+
+// Units per piece of the pipelined adamw4_step_host: 2^19 units (64 Mi values,
+// 128 MB of grads up, 256 MB of fp32 weights down).  ADAMW4_HOST_CHUNK_UNITS
+// overrides it (tests use small pieces to cut tensors at many places).
+int64_t host_chunk_units() {
+  if (const char* v = std::getenv("ADAMW4_HOST_CHUNK_UNITS")) {
+    const long long n = std::atoll(v);
+    if (n > 0) return (int64_t)n;
+  }
+  return (int64_t)1 << 19;
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -1251,6 +1274,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
       h->nblocks4 += ht.nblocks;
     }
     dev[i] = dev_tensor(tensors[i], ht.fp32, unit, ht.state_off);
+    ht.unit_begin = unit;
     unit += ht.nblocks;
     h->tensors.push_back(ht);
   }
@@ -1330,7 +1354,7 @@ extern "C" int adamw4_step(adamw4_handle* h, float lr, void* cuda_stream) {
   if (!dg.ok) return cuda_fail(h, dg.err, "selecting the device");
   const int64_t t = h->t + 1;
   const StepArgs a = make_args(h->cfg, lr, t);
-  const int rc = launch(h, a, static_cast<cudaStream_t>(cuda_stream));
+  const int rc = launch(h, a, static_cast<cudaStream_t>(cuda_stream), 0, h->nunits);
   if (rc != ADAMW4_OK) return rc;
   h->t = t;
   return ADAMW4_OK;
@@ -1339,30 +1363,90 @@ extern "C" int adamw4_step(adamw4_handle* h, float lr, void* cuda_stream) {
 extern "C" int adamw4_step_host(adamw4_handle* h, float lr, const uint16_t* const* grads_host,
                                 float* const* params_host, void* cuda_stream) {
   if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
+  if (!(lr >= 0.0f) || !std::isfinite(lr))
+    return fail(h, ADAMW4_EINVAL, "lr must be finite and non-negative");
+  for (size_t i = 0; i < h->tensors.size(); ++i) {
+    if (grads_host != nullptr && grads_host[i] == nullptr)
+      return fail(h, ADAMW4_EINVAL, "grads_host entry is NULL");
+    if (params_host != nullptr && params_host[i] == nullptr)
+      return fail(h, ADAMW4_EINVAL, "params_host entry is NULL");
+  }
   DeviceGuard dg(h->device);
   if (!dg.ok) return cuda_fail(h, dg.err, "selecting the device");
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e;
-  if (grads_host != nullptr) {
-    for (size_t i = 0; i < h->tensors.size(); ++i) {
-      const adamw4_tensor& d = h->tensors[i].desc;
-      if (grads_host[i] == nullptr) return fail(h, ADAMW4_EINVAL, "grads_host entry is NULL");
-      e = cudaMemcpyAsync(const_cast<uint16_t*>(d.grad_bf16), grads_host[i],
-                          (size_t)d.numel * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
-      if (e != cudaSuccess) return cuda_fail(h, e, "copying grads to the device");
+  const int64_t chunk = host_chunk_units();
+  const int64_t nchunks = (h->nunits + chunk - 1) / chunk;
+  if (h->s_in == nullptr) {
+    if ((e = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(h, e, "creating the copy streams");
+  }
+  while ((int64_t)h->events.size() < 2 * nchunks + 2) {
+    cudaEvent_t ev;
+    if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(h, e, "creating events");
+    h->events.push_back(ev);
+  }
+  const int64_t t = h->t + 1;
+  const StepArgs a = make_args(h->cfg, lr, t);
+  // The copies wait for the caller's earlier work on the buffers.
+  cudaEvent_t ev_start = h->events[2 * nchunks], ev_end = h->events[2 * nchunks + 1];
+  if ((e = cudaEventRecord(ev_start, s)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(h->s_in, ev_start, 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(h->s_out, ev_start, 0)) != cudaSuccess)
+    return cuda_fail(h, e, "ordering the copy streams");
+  // Piece k: its grads go up on s_in, it steps on the caller's stream, its
+  // weights come down on s_out; piece k+1's grads go up meanwhile.
+  size_t first = 0;   // first tensor that can reach into the current piece
+  for (int64_t k = 0; k < nchunks; ++k) {
+    const int64_t u0 = k * chunk, u1 = std::min(h->nunits, u0 + chunk);
+    while (first < h->tensors.size() &&
+           h->tensors[first].unit_begin + h->tensors[first].nblocks <= u0)
+      ++first;
+    // copies of the values of piece k, tensor by tensor
+    auto copy_piece = [&](bool up) -> cudaError_t {
+      for (size_t i = first; i < h->tensors.size() && h->tensors[i].unit_begin < u1; ++i) {
+        const HostTensor& ht = h->tensors[i];
+        const adamw4_tensor& d = ht.desc;
+        const int64_t v0 = (std::max(u0, ht.unit_begin) - ht.unit_begin) * kBlock;
+        const int64_t v1 = std::min(
+            (std::min(u1, ht.unit_begin + ht.nblocks) - ht.unit_begin) * (int64_t)kBlock, d.numel);
+        if (v1 <= v0) continue;
+        cudaError_t ce;
+        if (up) {
+          ce = cudaMemcpyAsync(const_cast<uint16_t*>(d.grad_bf16) + v0, grads_host[i] + v0,
+                               (size_t)(v1 - v0) * sizeof(uint16_t), cudaMemcpyHostToDevice,
+                               h->s_in);
+        } else {
+          const size_t wb = param_bytes(d);
+          ce = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(params_host[i]) + v0 * wb,
+                               reinterpret_cast<const uint8_t*>(d.param) + v0 * wb,
+                               (size_t)(v1 - v0) * wb, cudaMemcpyDeviceToHost, h->s_out);
+        }
+        if (ce != cudaSuccess) return ce;
+      }
+      return cudaSuccess;
+    };
+    if (grads_host != nullptr) {
+      if ((e = copy_piece(true)) != cudaSuccess) return cuda_fail(h, e, "copying grads to the device");
+      if ((e = cudaEventRecord(h->events[2 * k], h->s_in)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(s, h->events[2 * k], 0)) != cudaSuccess)
+        return cuda_fail(h, e, "ordering the copy streams");
+    }
+    const int rc = launch(h, a, s, u0, u1);
+    if (rc != ADAMW4_OK) return rc;
+    if (params_host != nullptr) {
+      if ((e = cudaEventRecord(h->events[2 * k + 1], s)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(h->s_out, h->events[2 * k + 1], 0)) != cudaSuccess)
+        return cuda_fail(h, e, "ordering the copy streams");
+      if ((e = copy_piece(false)) != cudaSuccess) return cuda_fail(h, e, "copying params to the host");
     }
   }
-  int rc = adamw4_step(h, lr, cuda_stream);
-  if (rc != ADAMW4_OK) return rc;
-  if (params_host != nullptr) {
-    for (size_t i = 0; i < h->tensors.size(); ++i) {
-      const adamw4_tensor& d = h->tensors[i].desc;
-      if (params_host[i] == nullptr) return fail(h, ADAMW4_EINVAL, "params_host entry is NULL");
-      e = cudaMemcpyAsync(params_host[i], d.param, (size_t)d.numel * param_bytes(d),
-                          cudaMemcpyDeviceToHost, s);
-      if (e != cudaSuccess) return cuda_fail(h, e, "copying params to the host");
-    }
-  }
+  if ((e = cudaEventRecord(ev_end, h->s_out)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(s, ev_end, 0)) != cudaSuccess)
+    return cuda_fail(h, e, "ordering the copy streams");
+  h->t = t;
   e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(h, e, "synchronising the stream");
   return ADAMW4_OK;
@@ -1702,6 +1786,6 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   st.fv = state->v32;
   const int64_t need = (unit + kHalves - 1) / kHalves;
   launch_vcode(cfg->vcode, bf16w, (int)std::min<int64_t>(nd.grid[cfg->vcode][bf16w], need), s,
-               table, unit, a, tabs, st);
+               table, 0, unit, a, tabs, st);
   return cudaGetLastError() == cudaSuccess ? ADAMW4_OK : ADAMW4_ECUDA;
 }

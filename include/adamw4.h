@@ -166,12 +166,18 @@ int adamw4_create(const adamw4_config *cfg, const adamw4_tensor *tensors, int n,
 int adamw4_step(adamw4_handle *h, float lr, void *cuda_stream);
 
 /* The same step with host buffers: for each tensor i, copies grads_host[i]
- * (numel bf16) to the tensor's device grad buffer, runs adamw4_step, then
- * copies the updated params back to params_host[i] (numel fp32), all on
- * `cuda_stream`, and waits for the stream.  Pinned host memory gives
- * asynchronous copies; pageable memory works but is slower.  A tensor flagged
- * ADAMW4_T_BF16_PARAM copies back numel bf16 values (2 bytes each).
- * Either array may be NULL to skip that direction. */
+ * (numel bf16) to the tensor's device grad buffer, runs the step, copies the
+ * updated params back to params_host[i] (numel fp32; numel bf16 for a tensor
+ * flagged ADAMW4_T_BF16_PARAM), and waits for `cuda_stream`.
+ * The work is pipelined over pieces of about 64 Mi values (whole 128-value
+ * units, cutting tensors where they fall): piece k's grads go up on a copy
+ * stream of the handle, piece k steps on `cuda_stream` (one launch per piece,
+ * all at the same t, so the result equals adamw4_step's), and its params come
+ * down on a second copy stream while the next pieces go up and step.  The
+ * copies start after the work already queued on `cuda_stream`.  Pinned host
+ * memory lets the copies overlap; pageable memory works but serialises them.
+ * Either array may be NULL to skip that direction.  A CUDA error part-way
+ * leaves the step partly applied. */
 int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_host,
                      float *const *params_host, void *cuda_stream);
 

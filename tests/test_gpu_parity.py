@@ -203,3 +203,62 @@ def test_pipeline_wait_timeout_is_reported_and_context_survives():
         assert all(np.isfinite(w).all() for w in g.weights())
     finally:
         g.close()
+
+
+def test_pipelined_host_step_cuts_tensors_anywhere():
+    """adamw4_step_host pipelines pieces of whole units; with 7-unit pieces
+    every tensor of a mixed list (ragged, fp32-state, bf16 weights) is cut at
+    several places.  Weights and state equal the one-launch device step."""
+    import os
+    import torch
+    B = binding()
+    ts = [dict(numel=65536, tensor_id=0, flags=0, weight_decay=0.1),
+          dict(numel=1000, tensor_id=5, flags=0, weight_decay=0.1),
+          dict(numel=4096 + 37, tensor_id=6, flags=workloads.T_LM_HEAD, weight_decay=0.0),
+          dict(numel=5000, tensor_id=7, flags=workloads.T_NORM, weight_decay=0.0),
+          dict(numel=128 * 50 + 3, tensor_id=8, flags=B.ADAMW4_T_BF16_PARAM, weight_decay=0.1)]
+    bf = [bool(t["flags"] & B.ADAMW4_T_BF16_PARAM) for t in ts]
+
+    def weights0():
+        out = []
+        for i, t in enumerate(ts):
+            w = torch.from_numpy((np.random.default_rng(i).standard_normal(t["numel"]) * 0.02)
+                                 .astype(np.float32))
+            out.append(w.to(torch.bfloat16) if bf[i] else w)
+        return out
+    gs = [workloads.bf16_bits((np.random.default_rng(9 + i).standard_normal(t["numel"]) * 1e-3)
+                              .astype(np.float32)) for i, t in enumerate(ts)]
+
+    def run(host):
+        params = [w.cuda() for w in weights0()]
+        grads = [torch.zeros(t["numel"], dtype=torch.bfloat16, device="cuda") for t in ts]
+        opt = B.AdamW4(params, grads, ts, vcode=0, seed=3, total_steps=2)
+        hp = [torch.empty(t["numel"], dtype=torch.int16 if bf[i] else torch.float32).pin_memory()
+              for i, t in enumerate(ts)]
+        hg = [torch.from_numpy(g.view(np.int16)).pin_memory() for g in gs]
+        for _ in range(2):
+            if host:
+                B.adamw4_step_host(opt.handle, 1e-3, [x.data_ptr() for x in hg],
+                                   [x.data_ptr() for x in hp],
+                                   torch.cuda.current_stream().cuda_stream)
+            else:
+                for g, x in zip(grads, hg):
+                    g.view(torch.int16).copy_(x)
+                opt.step()
+        torch.cuda.synchronize()
+        dev_w = [p.view(torch.int16).cpu().numpy() if bf[i] else p.cpu().numpy()
+                 for i, p in enumerate(params)]
+        blob = opt.state_dict_blob()
+        opt.close()
+        return dev_w, [x.numpy() for x in hp], blob
+
+    ref_w, _, ref_blob = run(False)
+    os.environ["ADAMW4_HOST_CHUNK_UNITS"] = "7"
+    try:
+        dev_w, host_w, blob = run(True)
+    finally:
+        del os.environ["ADAMW4_HOST_CHUNK_UNITS"]
+    assert blob == ref_blob
+    for i in range(len(ts)):
+        assert dev_w[i].tobytes() == ref_w[i].tobytes(), f"tensor {i} (device)"
+        assert host_w[i].tobytes() == ref_w[i].tobytes(), f"tensor {i} (host copy)"
