@@ -64,7 +64,7 @@ constexpr int kConsumerThreads = 256;             // eight consumer warps
 constexpr int kCtaThreads = kConsumerThreads + 32;  // plus the producer warp
 constexpr int kHalves = kConsumerThreads / kLanesPerUnit;  // consumer half-warps per CTA
 constexpr int kProducerWarp = kConsumerThreads / 32;
-constexpr int kStages = 4;                        // tiles in flight per CTA
+constexpr int kStages = 3;                        // tiles in flight per CTA
 // A tile is kHalves consecutive units; stage layout (CTA-wide):
 //   16 unit headers (64 B each) | w 16 x 512 B | g 16 x 256 B |
 //   m codes 16 x 64 B | v codes 16 x 64 B | m scales 16 x 4 B | v scales 16 x 4 B

@@ -91,7 +91,10 @@ class GpuRun:
         import torch
         Bm = binding()
         self.torch = torch
-        self.params = [torch.from_numpy(np.ascontiguousarray(w)).cuda() for w in host_ws]
+        # uint16 host arrays are bf16 weights (tensors flagged ADAMW4_T_BF16_PARAM)
+        self.params = [torch.from_numpy(np.ascontiguousarray(w).view(np.int16)).cuda()
+                       .view(torch.bfloat16) if w.dtype == np.uint16 else
+                       torch.from_numpy(np.ascontiguousarray(w)).cuda() for w in host_ws]
         self.grads = [torch.zeros(t["numel"], dtype=torch.bfloat16, device="cuda") for t in ts]
         self.opt = Bm.AdamW4(self.params, self.grads, ts, lr=lr, betas=(beta1, beta2), eps=eps,
                              vcode=vcode, seed=seed, total_steps=total_steps)
@@ -111,7 +114,8 @@ class GpuRun:
 
     def weights(self):
         self.torch.cuda.synchronize()
-        return [p.cpu().numpy() for p in self.params]
+        return [p.view(self.torch.int16).cpu().numpy().view(np.uint16)
+                if p.dtype == self.torch.bfloat16 else p.cpu().numpy() for p in self.params]
 
     def blob(self):
         return self.opt.state_dict_blob()
@@ -149,7 +153,10 @@ def run_both(ts, host_ws, grads_fn, steps, vcode=0, seed=0, total_steps=0, blob=
             if check_every_step or s == steps:
                 wg = gpu.weights()
                 for i, (a, b, o) in enumerate(zip(wg, ws, old)):
-                    assert_weights_close(a, b, o, f"{what} step {s} tensor {i}")
+                    if a.dtype == np.uint16:          # bf16 weights: bit for bit
+                        assert np.array_equal(a, b), f"{what} step {s} tensor {i} (bf16)"
+                    else:
+                        assert_weights_close(a, b, o, f"{what} step {s} tensor {i}")
                 assert_state_equal(gpu.blob(), ref.export_state(), vcode, f"{what} step {s}")
         return gpu, ref, ws
     finally:
