@@ -238,3 +238,51 @@ def test_two_gloo_ranks_equal_the_whole_step(vcode, chunks):
         assert a.tobytes() == b.tobytes()
     st = parse_blob(final0)
     assert st["t"] == TOTAL_STEPS and len(st["tensors"]) == len(SPECS)
+
+
+def _rank_dies(rank, world, port, root, out):
+    import sys
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import time
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    from bit_quantized_optimizer_b200.zero1 import FlatLayout, ZeroAdamW4
+    from oracle_pieces import OraclePieces
+    L = FlatLayout([s["numel"] for s in SPECS], world, 2)
+    fp, fg = torch.zeros(L.padded), torch.zeros(L.padded, dtype=torch.bfloat16)
+    opt = ZeroAdamW4(fp, fg, L, SPECS, vcode=0, seed=1,
+                     make_stepper=lambda p, g, s: OraclePieces(p, g, s, vcode=0, seed=1,
+                                                               total_steps=0))
+    opt.step()                             # one good step on both ranks
+    dist.barrier()
+    if rank == 1:
+        os._exit(0)                        # leaves between steps, nothing in flight
+    time.sleep(0.5)
+    t0 = time.monotonic()
+    try:
+        opt.step()
+        out.put(("no error", time.monotonic() - t0))
+    except Exception as e:                 # the survivor's next collective fails
+        out.put((type(e).__name__, time.monotonic() - t0))
+
+
+def test_a_lost_rank_surfaces_as_an_error_on_the_survivor():
+    """Failure detection on the host: rank 1 leaves between steps; rank 0's
+    next sharded step raises (peer gone or the 5 s process-group timeout)
+    instead of hanging."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies, args=(r, 2, port, root, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    what, took = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+    assert what != "no error"
+    assert took < 30
