@@ -80,6 +80,7 @@ constexpr uint32_t kUnitTx = 896;                 // bulk-copied bytes of one wh
 constexpr int kSmemStages = kStages * kStageBytes;
 static_assert(kStageBytes % 16 == 0, "stage alignment");
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr uint64_t kDrainLimitNs = 100000000ull;  // 0.1 s per stage when leaving early
 constexpr int kVZip = ADAMW4_V_ZIPSR;
 constexpr int kVZe = ADAMW4_V_ZEEDEN;
 constexpr int kVZiRtn = ADAMW4_V_ZI_RTN;
@@ -673,7 +674,16 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     const uint32_t full = full0 + 8u * s;
     if (round > 0 && !__all_sync(kMask, wait_phase_napping(empty0 + 8u * s, (round - 1) & 1u,
                                                            kWaitLimitNs))) {
+      // Leaving early: flag it, then wait (bounded) for the copies this warp
+      // issued into stages not yet handed back.  Stage j was last filled in
+      // this round if j < s, else in the previous one; its full barrier
+      // completes that fill's phase once the bytes have landed.
       if (lane == 0) atomicOr(a.status, 1u);
+      for (int j = 0; j < kStages; ++j) {
+        const uint32_t last = (j < s) ? round : round - 1;
+        wait_phase_napping(full0 + 8u * j, last & 1u, kDrainLimitNs);
+      }
+      cp_async_wait_all();
       return;
     }
     const int64_t u = u_begin + tile * kHalves + lane;
