@@ -81,17 +81,20 @@ def kernel_sha():
     return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
 
 
-def traffic_record(vcode_name):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+def profile_record(vcode_name):
+    """The committed ncu summary of the step kernel for this workload and
+    v code, if it was taken on the current kernel source; else {}."""
     p = os.path.join(ROOT, "profiles", f"adamw4_step_{WORKLOAD}_{vcode_name}_traffic.json")
     try:
         d = json.load(open(p))
     except Exception:
-        return None
-    if d.get("kernel_source_sha256") != kernel_sha():
-        return None
-    return d.get("traffic_bytes_per_launch")
+        return {}
+    return d if d.get("kernel_source_sha256") == kernel_sha() else {}
+
+
+def traffic_record(vcode_name):
+    """DRAM bytes per launch (ncu), or None."""
+    return profile_record(vcode_name).get("traffic_bytes_per_launch")
 
 
 class ClockSampler:
@@ -379,7 +382,9 @@ def run_ours(args):
             "hbm_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": traffic_record(variant_name(args))},
+                         "traffic": traffic_record(variant_name(args)),
+                         # the step is bound by instruction issue, not HBM: ncu figures
+                         "issue": profile_record(variant_name(args)).get("issue")},
             "e2e": e2e,
             "gpu_launches": args.steps,
             "clocks": clk,
