@@ -157,7 +157,8 @@ struct __align__(16) UnitHeader {
   uint32_t flags;        // ADAMW4_T_* | kKindFp32 | kStaged
   float decay;           // 1 - lr * weight_decay of the tensor
   int32_t nvalid;        // values in the unit (1..128)
-  uint32_t pad_[4];
+  uint32_t w_soff;       // bf16-weight units: stage offset of the unit's weights
+  uint32_t pad_[3];
 };
 static_assert(sizeof(UnitHeader) == 64, "UnitHeader layout");
 
@@ -730,16 +731,24 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     uint32_t tx = (uint32_t)__popc(staged_mask) * kUnitTx;
     if (BF16W) tx -= (uint32_t)__popc(__ballot_sync(kMask, staged && wbf)) * 256u;
     if (lane == 0) mbar_arrive_expect_tx(full, tx);
-    if (BF16W && staged && wbf && !a.fault_stall)      // bf16 weights: one copy per unit
-      bulk_g2s(dst + kOffW + lane * 512, reinterpret_cast<const uint16_t*>(t_param) + e0, 256u,
-               full);
+    if (BF16W) {
+      // A run's weights land packed at the start of its own units' 512-B w
+      // slots: 512 B per unit for fp32, 256 B for bf16.  The run starts at the
+      // nearest lane at or below this one that does not continue a run.
+      const int start = 31 - __clz(~cont_mask & ((2u << lane) - 1u));
+      hd->w_soff = (uint32_t)(kOffW + start * 512 + (lane - start) * (wbf ? 256 : 512));
+    }
     if (staged && !cont && !a.fault_stall) {
       // this lane starts a run: it extends over the following lanes whose
       // unit continues it
       const unsigned rest = ~(cont_mask >> (lane + 1));
       const int len = __ffs(rest);          // 1 + number of continuing lanes
       const int64_t blk = t_soff + ub;
-      if (!wbf) bulk_g2s(dst + kOffW + lane * 512, t_param + e0, 512u * len, full);
+      if (wbf)
+        bulk_g2s(dst + kOffW + lane * 512, reinterpret_cast<const uint16_t*>(t_param) + e0,
+                 256u * len, full);
+      else
+        bulk_g2s(dst + kOffW + lane * 512, t_param + e0, 512u * len, full);
       bulk_g2s(dst + kOffG + lane * 256, t_grad + e0, 256u * len, full);
       bulk_g2s(dst + kOffMC + lane * 64, st.mcodes + blk * (kBlock / 2), 64u * len, full);
       bulk_g2s(dst + kOffVC + lane * 64, st.vcodes + blk * (kBlock / 2), 64u * len, full);
@@ -834,7 +843,7 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
       {
         const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
         if (wbf) {
-          const uint4 wr = *reinterpret_cast<const uint4*>(sp + kOffW + half * 512 + lane * 16);
+          const uint4 wr = *reinterpret_cast<const uint4*>(sp + hdp->w_soff + lane * 16);
           w[0] = bf16lo(wr.x); w[1] = bf16hi(wr.x); w[2] = bf16lo(wr.y); w[3] = bf16hi(wr.y);
           w[4] = bf16lo(wr.z); w[5] = bf16hi(wr.z); w[6] = bf16lo(wr.w); w[7] = bf16hi(wr.w);
         } else {
