@@ -24,6 +24,7 @@ def pins(golden):
     return [
         ("philox known answers", lambda: P.test_known_answer_vectors(golden)),
         ("philox keying", P.test_draw_is_word_e_mod_4_of_one_call),
+        ("philox library", P.test_matches_the_curand_library_generator),
         ("uniform", P.test_uniform_range_and_granularity),
         ("nf4 quantiles", N.test_levels_match_library_quantiles),
         ("nf4 structure", N.test_level_structure),

@@ -1,4 +1,6 @@
 """Pins of the oracle's counter-based generator (CPU only)."""
+import ctypes
+import ctypes.util
 import os
 
 import numpy as np
@@ -59,3 +61,46 @@ def test_uniform_moments():
     u = np.array([oracle.uniform(oracle.draw_word(1, 1, 0, 0, e)) for e in range(n)])
     assert abs(u.mean() - 0.5) < 5 * np.sqrt(1 / 12 / n)
     assert abs(u.var() - 1 / 12) < 5 * np.sqrt(1 / 180 / n)
+
+
+def _curand():
+    for cand in ("/usr/local/cuda/lib64/libcurand.so", ctypes.util.find_library("curand")):
+        if cand:
+            try:
+                return ctypes.CDLL(cand)
+            except OSError:
+                pass
+    return None
+
+
+def _curand_quads(L, seed, nquads, first_quad):
+    """Words of cuRAND's host Philox4x32-10 generator (it runs on the CPU)."""
+    gen = ctypes.c_void_p()
+    assert L.curandCreateGeneratorHost(ctypes.byref(gen), 161) == 0   # PHILOX4_32_10
+    try:
+        assert L.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+        assert L.curandSetGeneratorOffset(gen, ctypes.c_ulonglong(4 * first_quad)) == 0
+        buf = (ctypes.c_uint32 * (4 * nquads))()
+        assert L.curandGenerate(gen, buf, 4 * nquads) == 0
+    finally:
+        L.curandDestroyGenerator(gen)
+    return np.array(buf, dtype=np.uint32).reshape(-1, 4)
+
+
+def test_matches_the_curand_library_generator():
+    """cuRAND's Philox4x32-10 (host generator, library code run on the CPU):
+    key = (seed lo, seed hi), and its output quad q is the block of counter
+    (q >> 16 as a 64-bit value in words 0-1, q & 0xFFFF in word 2, 0 in
+    word 3).  Seeds and offsets make every key bit and counter words 0-2
+    matter; word 3 is covered by the known-answer vectors."""
+    L = _curand()
+    assert L is not None, "libcurand from the CUDA toolkit is needed"
+    for seed in (0, 1, 0x0123456789ABCDEF, (1 << 64) - 1):
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        for q0 in (0, 65536 * 3 + 17, (1 << 48) + 5 * 65536 + 9, (1 << 61) + 65530):
+            w = _curand_quads(L, seed, 12, q0)
+            for i in range(12):
+                q = q0 + i
+                ctr = [(q >> 16) & 0xFFFFFFFF, (q >> 48) & 0xFFFFFFFF, q & 0xFFFF, 0]
+                assert [int(x) for x in oracle.philox4x32_10(ctr, key)] == [int(x) for x in w[i]], \
+                    (hex(seed), q)
