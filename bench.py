@@ -42,7 +42,8 @@ WORKLOAD = "gpt-2.7b"        # the benchmark workload; --workload picks a profil
 VCODES = {"zipsr": 0, "zeeden": 1, "zi_rtn": 2, "zi_sr": 3, "ze_floor": 4}
 METRIC = "fused 4-bit AdamW step Gparams/s; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "bit_quantized_optimizer_b200", "csrc", "adamw4.cu")
+# the device code of the step (the C ABI around it is in adamw4.cu)
+KERNEL_SRC = os.path.join(ROOT, "bit_quantized_optimizer_b200", "csrc", "adamw4_kernel.cuh")
 
 
 def is_fp32_state(numel, flags):

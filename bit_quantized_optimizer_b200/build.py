@@ -13,7 +13,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "csrc", "adamw4.cu")
 OUT = os.path.join(HERE, "libadamw4.so")
-DEPS = [SRC, os.path.join(HERE, "csrc", "nf4_table.h"),
+DEPS = [SRC, os.path.join(HERE, "csrc", "adamw4_kernel.cuh"), os.path.join(HERE, "csrc", "nf4_table.h"),
         os.path.join(os.path.dirname(HERE), "include", "adamw4.h")]
 
 

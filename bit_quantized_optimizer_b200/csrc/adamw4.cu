@@ -1,44 +1,11 @@
-// adamw4.cu -- fused 4-bit AdamW optimizer step (ZIP-SR / ZE-EDEN) for B200
-// (sm_100a), and the C ABI declared in include/adamw4.h.
-//
-// One kernel launch per step covers every parameter tensor.  The work is a flat
-// list of 128-value units: each block of a 4-bit tensor is one unit, and each
-// fp32-state tensor is cut into 128-element chunks.  The grid is persistent
-// (SM count x resident CTAs) and the units are dealt out round-robin, so all
-// SMs stream one contiguous window of HBM.
-//
-// A CTA has one producer warp and eight consumer warps.  Each consumer
-// half-warp owns a ring of kStages shared-memory stages; producer lane j feeds
-// the ring of half-warp j.  For every unit the producer writes a 64-byte header
-// (addresses, block index, tensor id, flags, decay) into the stage and, for a
-// whole 4-bit block, fills the stage with TMA bulk copies (cp.async.bulk: 512 B
-// of fp32 weights, 256 B of bf16 grads, 64 + 64 B of codes) plus two 4-byte
-// cp.async copies of the block scales, all completing on the stage's "full"
-// mbarrier.  The consumer half-warp waits on it, computes from the stage,
-// stores the results straight to global memory and hands the stage back on
-// its "empty" mbarrier.  Units that are not whole
-// 4-bit blocks (a ragged last block, fp32-state chunks) carry only the header
-// and are read from global memory by the consumer.  Every wait is bounded by
-// a timer; on expiry the kernel records the failure in a status word and the
-// waiting warp leaves.
-//
-// Per unit, following the method flowchart of "ZIP-SR / ZE-EDEN: 4-bit AdamW
-// state quantization" (daiwk.github.io, Method): decode the prior moments,
-// update them, update the weights, requantise (ZIP-SR or ZE-EDEN for v, NF4 for
-// m), pack.  The weights use the unquantised working moments (same page, Core
-// equation: weights are updated before the moments are quantised).
-//
-// Arithmetic follows one fixed binary32 evaluation order with IEEE division
-// and square root (__fdiv_rn, __fsqrt_rn) and fused multiply-add only where
-// written (__fmaf_rn, or __ffma2_rn on value pairs, which rounds each lane like
-// __fmaf_rn); the file is built with -fmad=false so nothing else is contracted.
-// With that, codes, scales and weights are reproducible bit for bit by any
-// IEEE implementation of the same order.
-//
-// No tensor cores: the step is a streaming codec, bound by HBM bandwidth.  No
-// TMA multicast: every copy is this GPU's global memory into its own CTA.
+// adamw4.cu -- the C ABI (include/adamw4.h) of the fused 4-bit AdamW step
+// (ZIP-SR / ZE-EDEN) for B200 (sm_100a): validation and classification of the
+// tensor list, the state arena, step scalars and code tables, launches (one per
+// step, or one per piece of the pipelined host-buffer step), checkpoints, and
+// the allocation-free entry point.  The kernel is in adamw4_kernel.cuh.
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>   // header-only; ranges show up under a profiler
 
 #include <algorithm>
 #include <cfloat>
@@ -54,842 +21,9 @@
 
 #include "../../include/adamw4.h"
 #include "nf4_table.h"
+#include "adamw4_kernel.cuh"
 
 namespace {
-
-constexpr int kBlock = ADAMW4_BLOCK;              // values per quantisation block
-constexpr int kLanesPerUnit = 16;                 // a half-warp per block
-constexpr int kPerLane = kBlock / kLanesPerUnit;  // 8 values per lane
-constexpr int kConsumerThreads = 256;             // eight consumer warps
-constexpr int kCtaThreads = kConsumerThreads + 32;  // plus the producer warp
-constexpr int kHalves = kConsumerThreads / kLanesPerUnit;  // consumer half-warps per CTA
-constexpr int kProducerWarp = kConsumerThreads / 32;
-constexpr int kStages = 3;                        // tiles in flight per CTA
-// A tile is kHalves consecutive units; stage layout (CTA-wide):
-//   16 unit headers (64 B each) | w 16 x 512 B | g 16 x 256 B |
-//   m codes 16 x 64 B | v codes 16 x 64 B | m scales 16 x 4 B | v scales 16 x 4 B
-constexpr int kOffHdr = 0;
-constexpr int kOffW = kOffHdr + kHalves * 64;
-constexpr int kOffG = kOffW + kHalves * 512;
-constexpr int kOffMC = kOffG + kHalves * 256;
-constexpr int kOffVC = kOffMC + kHalves * 64;
-constexpr int kOffMS = kOffVC + kHalves * 64;
-constexpr int kOffVS = kOffMS + kHalves * 4;
-constexpr int kStageBytes = kOffVS + kHalves * 4; // 15,488 B, a 16-byte multiple
-constexpr uint32_t kUnitTx = 896;                 // bulk-copied bytes of one whole block
-constexpr int kSmemStages = kStages * kStageBytes;
-static_assert(kStageBytes % 16 == 0, "stage alignment");
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
-constexpr uint64_t kDrainLimitNs = 100000000ull;  // 0.1 s per stage when leaving early
-constexpr int kVZip = ADAMW4_V_ZIPSR;
-constexpr int kVZe = ADAMW4_V_ZEEDEN;
-constexpr int kVZiRtn = ADAMW4_V_ZI_RTN;
-constexpr int kVZiSr = ADAMW4_V_ZI_SR;
-constexpr int kVZeFloor = ADAMW4_V_ZE_FLOOR;
-constexpr uint32_t kBf16W = ADAMW4_T_BF16_PARAM;  // weights stored as bf16
-constexpr uint32_t kKindFp32 = 1u << 16;          // internal flag: fp32-state tensor
-constexpr uint32_t kStaged = 1u << 17;            // internal flag: unit data is in the stage
-constexpr uint32_t kNoUnit = 1u << 18;            // internal flag: empty slot of the last tile
-constexpr uint32_t kStreamV = 0u;                 // Philox stream of the v draw
-constexpr uint32_t kStreamM = 1u;                 // Philox stream of the LM-head m draw
-constexpr float kMagic = 12582912.0f;             // 1.5 * 2^23: adding it rounds to an integer
-
-// Philox4x32-10 round multipliers (Salmon et al., SC'11).  The per-round keys
-// (key + r * Weyl constants) are formed on the host.
-constexpr uint32_t kPhiloxM0 = 0xD2511F53u;
-constexpr uint32_t kPhiloxM1 = 0xCD9E8D57u;
-constexpr uint32_t kPhiloxW0 = 0x9E3779B9u;
-constexpr uint32_t kPhiloxW1 = 0xBB67AE85u;
-
-// One parameter tensor as the kernel sees it (64 bytes).
-struct __align__(16) DevTensor {
-  float* param;
-  const uint16_t* grad;
-  int64_t numel;
-  int64_t unit_begin;   // first unit of this tensor in the flat unit list
-  int64_t unit_end;     // one past its last unit
-  int64_t state_off;    // 4-bit: first block in the code arena; fp32: first element
-  uint32_t tensor_id;
-  uint32_t flags;       // ADAMW4_T_* | kKindFp32
-  float weight_decay;
-  uint32_t block_offset;  // elem_offset / 128: where this piece starts in its tensor
-};
-static_assert(sizeof(DevTensor) == 64, "DevTensor layout");
-
-// Per-step scalars, formed on the host in binary64 and rounded once.
-struct StepArgs {
-  float step_size;   // lr / (1 - b1^t)
-  float rs_bc2;      // 1 / sqrt(1 - b2^t)
-  float b1, omb1, b2, omb2, eps, lr;
-  uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
-  uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
-  int lm_sr_active;      // final-10% LM-head phase
-  uint32_t* status;      // device status word (bit 0: a pipeline wait timed out)
-  int fault_stall;       // test hook: mark stages filled without filling them
-};
-
-// Code tables, passed by value and staged in shared memory by each CTA.
-struct CodeTables {
-  float nf4[16];        // NF4 levels, ascending
-  float nf4_gap[16];    // nf4[j+1] - nf4[j]
-  float vz[16];         // ZIP-SR code points k/15
-  float vz_sqrt[16];    // sqrt(k/15)
-  float vz_mid[16];     // nearest-point thresholds of the k/15 code (15 used)
-  float2 rtn[128];      // NF4 nearest-level buckets: .x threshold, .y base code (int bits)
-};
-
-struct StateArena {
-  uint8_t* mcodes;   // 64 bytes per block, element 2i in the low nibble of byte i
-  uint8_t* vcodes;
-  float* mscale;     // one per block
-  float* vscale;
-  float* fm;         // fp32-state tensors
-  float* fv;
-};
-
-// What the producer tells the consumer about one unit (64 bytes).
-struct __align__(16) UnitHeader {
-  float* w;              // the unit's first weight
-  const uint16_t* g;     // its first gradient
-  uint64_t e0;           // index of that element within its (logical) tensor
-  uint64_t state;        // 4-bit: block index in the code arena; fp32: element index
-  uint32_t tensor_id;
-  uint32_t flags;        // ADAMW4_T_* | kKindFp32 | kStaged
-  float decay;           // 1 - lr * weight_decay of the tensor
-  int32_t nvalid;        // values in the unit (1..128)
-  uint32_t w_soff;       // bf16-weight units: stage offset of the unit's weights
-  uint32_t pad_[3];
-};
-static_assert(sizeof(UnitHeader) == 64, "UnitHeader layout");
-
-// ---------------------------------------------------------------------------
-// PTX wrappers: mbarrier, bulk copies, timer
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                         uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Waits for a barrier phase; false if `limit_ns` passed first.  The timer is
-// read once per 64 polls.
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > limit_ns) return false;
-  }
-}
-
-// The producer's wait for a stage to come back: the consumers take
-// microseconds per tile, so it naps between polls instead of taking issue
-// slots from them.  False if `limit_ns` passed first.
-__device__ __forceinline__ bool wait_phase_napping(uint32_t bar, uint32_t parity,
-                                                   uint64_t limit_ns) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    __nanosleep(1000);
-    if (mbar_test_wait(bar, parity)) return true;
-    if (global_ns() - t0 > limit_ns) return false;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Arithmetic helpers
-// ---------------------------------------------------------------------------
-
-// Philox4x32-10 of the counter (quad low, quad high, t, c3).  The counter's
-// third word is the step t for every draw of a launch, so round 0's product
-// M1 * t is a per-step constant the host supplies (r0_hi_k0 = hi(M1 t) ^ key0,
-// r0_lo = lo(M1 t)); rounds 1..9 are the usual ones.
-__device__ __forceinline__ uint4 philox4x32_10(uint64_t quad, uint32_t c3, const StepArgs& a) {
-  const uint64_t q0 = (uint64_t)kPhiloxM0 * (uint32_t)quad;
-  uint4 c = make_uint4(a.r0_hi_k0 ^ (uint32_t)(quad >> 32), a.r0_lo,
-                       (uint32_t)(q0 >> 32) ^ c3 ^ a.rk1[0], (uint32_t)q0);
-#pragma unroll
-  for (int r = 1; r < 10; ++r) {
-    const uint64_t p0 = (uint64_t)kPhiloxM0 * c.x;
-    const uint64_t p1 = (uint64_t)kPhiloxM1 * c.z;
-    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ a.rk0[r], (uint32_t)p1,
-                   (uint32_t)(p0 >> 32) ^ c.w ^ a.rk1[r], (uint32_t)p0);
-  }
-  return c;
-}
-
-// 1 + u for the draw u in [0,1): the low 23 bits of a word as the mantissa of
-// a number in [1, 2).  u = (1 + u) - 1 is exact; u * B rounds like
-// fma(1 + u, B, -B).
-__device__ __forceinline__ float one_plus_u(uint32_t w) {
-  return __uint_as_float((w | 0x3F800000u) & 0x3FFFFFFFu);
-}
-__device__ __forceinline__ float uniform23(uint32_t w) { return __fsub_rn(one_plus_u(w), 1.0f); }
-
-// The eight draw words of one lane: elements 4*quad .. 4*quad + 7.
-__device__ __forceinline__ void words8(const StepArgs& a, uint32_t tensor_id, uint32_t stream,
-                                       uint64_t quad, uint32_t r[8]) {
-  const uint32_t c3 = tensor_id * 2u + stream;
-  const uint4 r0 = philox4x32_10(quad, c3, a);
-  const uint4 r1 = philox4x32_10(quad + 1, c3, a);
-  r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w;
-  r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
-}
-
-__device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
-
-// binary32 -> bf16, IEEE round to nearest even (the cvt instruction).  Two
-// values: lo in bits 0-15, hi in bits 16-31.
-__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ uint16_t bf16_rn(float x) {
-  uint16_t r;
-  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
-
-// Max of non-negative binary32 values over a half-warp: their bit patterns
-// order like the values, so an integer reduction gives the exact maximum.
-__device__ __forceinline__ float hmax16_nonneg(float v, unsigned mask) {
-  return __uint_as_float(__reduce_max_sync(mask, __float_as_uint(v)));
-}
-
-// Balanced pairwise sum of (x, y) pairs over the half-warp: partner offsets 1,
-// 2, 4, 8 join adjacent 8-value groups in index order (IEEE addition is
-// commutative, so both partners hold the same bits).
-__device__ __forceinline__ float2 hsum16_tree2(float2 v, unsigned mask) {
-#pragma unroll
-  for (int off = 1; off < 16; off <<= 1) {
-    const float2 o = make_float2(__shfl_xor_sync(mask, v.x, off), __shfl_xor_sync(mask, v.y, off));
-    v = __fadd2_rn(v, o);
-  }
-  return v;
-}
-
-// NF4 nearest level: #{j : x > mid[j]}.  Bucket round(32 x + 32) holds at most
-// one threshold; the table has 128 entries so any 7-bit index stays inside.
-__device__ __forceinline__ uint32_t nf4_rtn_bucket(float x, float bucket_sum, const float2* rtn) {
-  const float2 e = rtn[__float_as_uint(bucket_sum) & 127u];
-  return (uint32_t)(__float_as_int(e.y) + (x > e.x ? 1 : 0));
-}
-
-// State-space stochastic rounding on the NF4 grid (LM-head m, final 10%).
-__device__ __forceinline__ uint32_t nf4_sr(float x, float u, const float* nf4, const float* gap) {
-  int j = 0;
-#pragma unroll
-  for (int i = 1; i <= 14; ++i) j = (nf4[i] <= x) ? i : j;
-  const bool lower = __fmul_rn(u, gap[j]) < __fsub_rn(nf4[j + 1], x);
-  return lower ? (uint32_t)j : (uint32_t)(j + 1);
-}
-
-// Shared tables of one CTA.
-struct SmemTables {
-  float2 mpair[256];   // byte of two m codes -> their two NF4 levels
-  float2 vpair[256];   // byte of two v codes -> their two code points
-  float2 rtn[128];
-  float nf4[16];
-  float gap[16];
-  float vz[16];        // ZIP-SR code points k/15
-  float4 zip[16];      // for k0 = nearest integer to 15x: {VZ[k0] (+inf for 15),
-                       //   sqrt VZ[k0-1], sqrt VZ[k0], sqrt VZ[k0+1]}
-  float2 vzp[16];      // {k/15, (k+1)/15}
-  float vzmid[16];     // thresholds between adjacent k/15 code points
-};
-
-// ---------------------------------------------------------------------------
-// Requantisation of one 4-bit block held by a half-warp (8 values per lane).
-// FULL: all 128 values valid.  Otherwise `myn` values of this lane are valid.
-// ---------------------------------------------------------------------------
-
-// ZIP-SR codes of 8 values.  FLAT: also test for d(a) == d(b), which needs the
-// state-space fallback; callers skip it when the block's R makes that
-// impossible.
-template <bool FULL, bool FLAT>
-__device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
-                                                 const float (&v1)[kPerLane],
-                                                 const float (&den)[kPerLane],
-                                                 const uint32_t (&rw)[kPerLane], float inv,
-                                                 float R, int myn) {
-  // two values at a time; from the last pair to the first, so that element i
-  // ends in bits 4i..4i+3
-  uint32_t vco = 0;
-#pragma unroll
-  for (int j = kPerLane / 2 - 1; j >= 0; --j) {
-    const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
-    const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
-    // k0, the nearest integer to 15x, is the bracket or one above it (the top
-    // entry's threshold is +inf: its bracket is always 14)
-    const uint32_t k0a = __float_as_uint(t2.x) & 15u, k0b = __float_as_uint(t2.y) & 15u;
-    const float4 ea = S.zip[k0a], eb = S.zip[k0b];
-    const bool deca = x2.x < ea.x, decb = x2.y < eb.x;
-    // square roots of the lower and upper code points of each value
-    const float2 sa = make_float2(deca ? ea.y : ea.z, decb ? eb.y : eb.z);
-    const float2 sb = make_float2(deca ? ea.z : ea.w, decb ? eb.z : eb.w);
-    const float2 da = __ffma2_rn(sa, f2(R), f2(a.eps));
-    const float2 db = __ffma2_rn(sb, f2(R), f2(a.eps));
-    const float2 dv = make_float2(den[2 * j], den[2 * j + 1]);
-    // fma(y, -1, x) rounds like x - y
-    const float2 B = __fmul2_rn(__ffma2_rn(da, f2(-1.0f), db), dv);      // (db - da) * dv
-    const float2 rhs = __fmul2_rn(__ffma2_rn(dv, f2(-1.0f), db), da);    // (db - dv) * da
-    const float2 f = make_float2(one_plus_u(rw[2 * j]), one_plus_u(rw[2 * j + 1]));
-    const float2 lhs = __ffma2_rn(f, B, make_float2(-B.x, -B.y));         // u * B
-    bool lowa = lhs.x < rhs.x, lowb = lhs.y < rhs.y;
-    const uint32_t ka = k0a - (deca ? 1u : 0u), kb = k0b - (decb ? 1u : 0u);
-    if (FLAT) {
-      if (da.x == db.x) {
-        const float2 z = S.vzp[ka];
-        lowa = __fmul_rn(__fsub_rn(f.x, 1.0f), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.x);
-      }
-      if (da.y == db.y) {
-        const float2 z = S.vzp[kb];
-        lowb = __fmul_rn(__fsub_rn(f.y, 1.0f), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.y);
-      }
-    }
-    const uint32_t ca = (FULL || 2 * j < myn) ? ka + (lowa ? 0u : 1u) : 0u;
-    const uint32_t cb = (FULL || 2 * j + 1 < myn) ? kb + (lowb ? 0u : 1u) : 0u;
-    vco = (vco * 16u + cb) * 16u + ca;
-  }
-  return vco;
-}
-
-template <int VCODE, bool FULL>
-__device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTables& S,
-                                              uint32_t tensor_id, uint32_t flags, uint64_t e0,
-                                              int lane, int myn, unsigned hmask,
-                                              const float (&m1)[kPerLane],
-                                              const float (&v1)[kPerLane],
-                                              const float (&den)[kPerLane], uint32_t* mcw,
-                                              uint32_t* vcw, float* msp, float* vsp) {
-  float am = 0.0f, av = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    if (FULL || i < myn) {
-      am = fmaxf(am, fabsf(m1[i]));
-      av = fmaxf(av, fabsf(v1[i]));
-    }
-  }
-  am = hmax16_nonneg(am, hmask);
-  av = hmax16_nonneg(av, hmask);
-
-  // ---- first moment: absmax scale, NF4 codes ----
-  uint32_t mco = 0;
-  float mso = 0.0f;
-  if (am >= FLT_MIN) {
-    const float inv = __fdiv_rn(1.0f, am);
-    if ((flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
-      uint32_t rw[kPerLane];
-      words8(a, tensor_id, kStreamM, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
-#pragma unroll
-      for (int i = 0; i < kPerLane; ++i)
-        if (FULL || i < myn)
-          mco |= nf4_sr(__fmul_rn(m1[i], inv), uniform23(rw[i]), S.nf4, S.gap) << (4 * i);
-    } else {
-#pragma unroll
-      for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
-        const float2 x = __fmul2_rn(make_float2(m1[2 * j], m1[2 * j + 1]), f2(inv));
-        const float2 b = __ffma2_rn(x, f2(32.0f), f2(kMagic + 32.0f));
-        const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? nf4_rtn_bucket(x.y, b.y, S.rtn) : 0u;
-        const uint32_t c0 = (FULL || 2 * j < myn) ? nf4_rtn_bucket(x.x, b.x, S.rtn) : 0u;
-        mco = (mco * 16u + c1) * 16u + c0;
-      }
-    }
-    mso = am;
-  }
-
-  // ---- second moment ----
-  uint32_t vco = 0;
-  float vso = 0.0f;
-  if (av >= FLT_MIN) {
-    const float inv = __fdiv_rn(1.0f, av);
-    if (VCODE == kVZip) {
-      // ZIP-SR ("ZIP-SR / ZE-EDEN", Core equation): keep the lower code point
-      // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
-      // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
-      const float R = __fmul_rn(__fsqrt_rn(av), a.rs_bc2);
-      uint32_t rw[kPerLane];
-      words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
-      // d(a) == d(b) needs (sqrt(k+1/15) - sqrt(k/15)) R below two ulps of
-      // R + eps; the smallest gap is 0.0339, so R > 1e-5 eps rules it out.
-      if (R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN)
-        vco = zipsr_codes8<FULL, false>(a, S, v1, den, rw, inv, R, myn);
-      else
-        vco = zipsr_codes8<FULL, true>(a, S, v1, den, rw, inv, R, myn);
-      vso = av;
-    } else if (VCODE == kVZiRtn || VCODE == kVZiSr) {
-      // State-space rules on the zero-inclusive code: nearest code point, or
-      // the lower one with probability (b - x)/(b - a).
-      uint32_t rw[kPerLane];
-      if (VCODE == kVZiSr) words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
-#pragma unroll
-      for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
-        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
-        const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
-#pragma unroll
-        for (int h = 1; h >= 0; --h) {
-          const int i = 2 * j + h;
-          const float x = h ? x2.y : x2.x;
-          const uint32_t k0 = __float_as_uint(h ? t2.y : t2.x) & 15u;
-          const uint32_t k = k0 - ((x < S.zip[k0].x) ? 1u : 0u);   // the bracket
-          uint32_t c;
-          if (VCODE == kVZiRtn) {
-            c = k + ((x > S.vzmid[k]) ? 1u : 0u);
-          } else {
-            const float2 z = S.vzp[k];
-            const bool lower = __fmul_rn(uniform23(rw[i]), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
-            c = k + (lower ? 0u : 1u);
-          }
-          vco = vco * 16u + ((FULL || i < myn) ? c : 0u);
-        }
-      }
-      vso = av;
-    } else if (VCODE == kVZeFloor) {
-      // Zero-excluded code with a positive floor: nearest (k+1)/16, no rescale.
-#pragma unroll
-      for (int j = kPerLane / 2 - 1; j >= 0; --j) {
-        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
-        const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
-        const uint32_t k0 = max(__float_as_uint(t2.x) & 31u, 1u) - 1u;
-        const uint32_t k1 = max(__float_as_uint(t2.y) & 31u, 1u) - 1u;
-        const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? k1 : 0u;
-        const uint32_t c0 = (FULL || 2 * j < myn) ? k0 : 0u;
-        vco = (vco * 16u + c1) * 16u + c0;
-      }
-      vso = av;
-    } else {
-      // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
-      // code point, scale times ||x||^2 / max(<x,Q(x)>, 1e-12 s^2) on x = v/s.
-      float2 l1[kPerLane / 2];
-#pragma unroll
-      for (int j = 0; j < kPerLane / 2; ++j) {
-        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
-        const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
-        const float2 c2 = __fadd2_rn(t2, f2(-kMagic));             // rint(16x), exact
-        const float2 q2 = __fmul2_rn(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)),
-                                     f2(0.0625f));                 // (k+1)/16
-        const uint32_t k0 = max(__float_as_uint(t2.x) & 31u, 1u) - 1u;
-        const uint32_t k1 = max(__float_as_uint(t2.y) & 31u, 1u) - 1u;
-        float2 xx = __fmul2_rn(x2, x2);
-        float2 xq = __fmul2_rn(x2, q2);
-        if (!FULL) {
-          if (2 * j >= myn) { xx.x = 0.0f; xq.x = 0.0f; }
-          if (2 * j + 1 >= myn) { xx.y = 0.0f; xq.y = 0.0f; }
-        }
-        if (FULL || 2 * j < myn) vco |= k0 << (8 * j);
-        if (FULL || 2 * j + 1 < myn) vco |= k1 << (8 * j + 4);
-        // first tree level: (x0^2 + x1^2, x0 q0 + x1 q1)
-        l1[j] = __fadd2_rn(make_float2(xx.x, xq.x), make_float2(xx.y, xq.y));
-      }
-      const float2 l2a = __fadd2_rn(l1[0], l1[1]);
-      const float2 l2b = __fadd2_rn(l1[2], l1[3]);
-      const float2 s = hsum16_tree2(__fadd2_rn(l2a, l2b), hmask);    // (sum x^2, sum x q)
-      vso = __fmul_rn(av, __fdiv_rn(s.x, fmaxf(s.y, 1e-12f)));
-    }
-  }
-
-  *mcw = mco;
-  *vcw = vco;
-  if (lane == 0) {
-    *msp = mso;
-    *vsp = vso;
-  }
-}
-
-// Decode + moment update + weight update for 8 values of a 4-bit block.
-__device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, float decay,
-                                        float (&w)[kPerLane], const float (&g)[kPerLane],
-                                        uint32_t mc, uint32_t vc, float sm, float sv,
-                                        float (&m1)[kPerLane], float (&v1)[kPerLane],
-                                        float (&den)[kPerLane]) {
-#pragma unroll
-  for (int j = 0; j < kPerLane / 2; ++j) {
-    // one byte holds the codes of values 2j (low nibble) and 2j+1 (high nibble)
-    const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], f2(sm));
-    const float2 v0 = __fmul2_rn(S.vpair[__byte_perm(vc, 0, 0x4440 + j)], f2(sv));
-    const float2 gg = make_float2(g[2 * j], g[2 * j + 1]);
-    const float2 mm = __ffma2_rn(f2(a.b1), m0, __fmul2_rn(f2(a.omb1), gg));
-    const float2 vv = __ffma2_rn(f2(a.b2), v0, __fmul2_rn(f2(a.omb2), __fmul2_rn(gg, gg)));
-    const float2 dd = __ffma2_rn(make_float2(__fsqrt_rn(vv.x), __fsqrt_rn(vv.y)), f2(a.rs_bc2),
-                                 f2(a.eps));
-    const float2 qq = make_float2(__fdiv_rn(mm.x, dd.x), __fdiv_rn(mm.y, dd.y));
-    const float2 ww = __ffma2_rn(f2(-a.step_size), qq,
-                                 __fmul2_rn(make_float2(w[2 * j], w[2 * j + 1]), f2(decay)));
-    w[2 * j] = ww.x; w[2 * j + 1] = ww.y;
-    m1[2 * j] = mm.x; m1[2 * j + 1] = mm.y;
-    v1[2 * j] = vv.x; v1[2 * j + 1] = vv.y;
-    den[2 * j] = dd.x; den[2 * j + 1] = dd.y;
-  }
-}
-
-// Weight i of a lane's run, fp32 or (BF16W and flagged) bf16.
-template <bool BF16W>
-__device__ __forceinline__ float load_w(const float* wp, const uint16_t* wp16, bool wbf, int i) {
-  if (BF16W && wbf) return __uint_as_float((uint32_t)wp16[i] << 16);
-  return wp[i];
-}
-template <bool BF16W>
-__device__ __forceinline__ void store_w(float* wp, uint16_t* wp16, bool wbf, int i, float x) {
-  if (BF16W && wbf) wp16[i] = bf16_rn(x);
-  else wp[i] = x;
-}
-
-// A unit read straight from global memory: a ragged last 4-bit block or a
-// chunk of an fp32-state tensor.
-template <int VCODE, bool BF16W>
-__device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTables& S,
-                                            const StateArena& st, const UnitHeader* hdp,
-                                            int lane, unsigned hmask) {
-  const int my0 = lane * kPerLane;
-  const int myn = min(max(hdp->nvalid - my0, 0), kPerLane);
-  const uint32_t flags = hdp->flags;
-  const bool wbf = BF16W && (flags & kBf16W);
-  const float decay = hdp->decay;
-  const uint64_t state = hdp->state;
-  // the header's w is the unit's first weight, of either width
-  float* wp = wbf ? nullptr : hdp->w + my0;
-  uint16_t* wp16 = wbf ? reinterpret_cast<uint16_t*>(hdp->w) + my0 : nullptr;
-  const uint16_t* gp = hdp->g + my0;
-  float w[kPerLane], g[kPerLane];
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    w[i] = (i < myn) ? load_w<BF16W>(wp, wp16, wbf, i) : 0.0f;
-    g[i] = (i < myn) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
-  }
-  if (flags & kKindFp32) {
-    float* mp = st.fm + state + my0;
-    float* vp = st.fv + state + my0;
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i) {
-      if (i < myn) {
-        const float m1 = __fmaf_rn(a.b1, mp[i], __fmul_rn(a.omb1, g[i]));
-        const float v1 = __fmaf_rn(a.b2, vp[i], __fmul_rn(a.omb2, __fmul_rn(g[i], g[i])));
-        const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
-        store_w<BF16W>(wp, wp16, wbf, i,
-                       __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay)));
-        mp[i] = m1;
-        vp[i] = v1;
-      }
-    }
-    return;
-  }
-  const uint64_t blk = state;
-  uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
-  uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
-  float m1[kPerLane], v1[kPerLane], den[kPerLane];
-  update8(a, S, decay, w, g, *mcw, *vcw, st.mscale[blk], st.vscale[blk], m1, v1, den);
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i)
-    if (i < myn) store_w<BF16W>(wp, wp16, wbf, i, w[i]);
-  requant_store<VCODE, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask, m1, v1,
-                              den, mcw, vcw, st.mscale + blk, st.vscale + blk);
-}
-
-// ---------------------------------------------------------------------------
-// Producer: fills CTA-wide stages, one tile of kHalves consecutive units each.
-// Lane i handles unit i of the tile (header, scales); the lane that starts a
-// run of whole 4-bit blocks of one tensor issues that run's bulk copies.
-// ---------------------------------------------------------------------------
-template <bool BF16W>
-__device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t u_begin,
-                                        int64_t u_end, const StepArgs& a, const StateArena& st,
-                                        uint8_t* stages, uint32_t full0, uint32_t empty0,
-                                        int lane) {
-  constexpr unsigned kMask = (1u << kHalves) - 1u;
-  const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
-  int ti = -1;
-  int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0, t_eoff = 0;
-  float* t_param = nullptr;
-  const uint16_t* t_grad = nullptr;
-  uint32_t t_id = 0, t_flags = 0;
-  float t_decay = 1.0f;
-  const uint32_t stages_s = smem_addr(stages);
-  int s = 0;
-  uint32_t round = 0;
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const uint32_t full = full0 + 8u * s;
-    if (round > 0 && !__all_sync(kMask, wait_phase_napping(empty0 + 8u * s, (round - 1) & 1u,
-                                                           kWaitLimitNs))) {
-      // Leaving early: flag it, then wait (bounded) for the copies this warp
-      // issued into stages not yet handed back.  Stage j was last filled in
-      // this round if j < s, else in the previous one; its full barrier
-      // completes that fill's phase once the bytes have landed.
-      if (lane == 0) atomicOr(a.status, 1u);
-      for (int j = 0; j < kStages; ++j) {
-        const uint32_t last = (j < s) ? round : round - 1;
-        wait_phase_napping(full0 + 8u * j, last & 1u, kDrainLimitNs);
-      }
-      cp_async_wait_all();
-      return;
-    }
-    const int64_t u = u_begin + tile * kHalves + lane;
-    const bool has = u < u_end;
-    if (has && u >= t_end) {
-      do {
-        ++ti;
-        t_end = __ldg(&T[ti].unit_end);
-      } while (u >= t_end);
-      const DevTensor* d = &T[ti];
-      t_begin = __ldg(&d->unit_begin);
-      t_numel = __ldg(&d->numel);
-      t_soff = __ldg(&d->state_off);
-      t_eoff = (int64_t)__ldg(&d->block_offset) * kBlock;
-      t_param = d->param;
-      t_grad = d->grad;
-      t_id = __ldg(&d->tensor_id);
-      t_flags = __ldg(&d->flags);
-      t_decay = (float)(1.0 - (double)a.lr * (double)__ldg(&d->weight_decay));
-    }
-    const int64_t ub = u - t_begin;
-    const int64_t e0 = ub * kBlock;
-    const int nvalid = has ? (int)min((int64_t)kBlock, t_numel - e0) : 0;
-    const bool staged = has && !(t_flags & kKindFp32) && nvalid == kBlock;
-    const bool wbf = BF16W && (t_flags & kBf16W);       // bf16 weights: 256 B per unit
-    uint8_t* sp = stages + s * kStageBytes;
-    UnitHeader* hd = reinterpret_cast<UnitHeader*>(sp + kOffHdr) + lane;
-    hd->w = wbf ? reinterpret_cast<float*>(reinterpret_cast<uint16_t*>(t_param) + e0)
-                : t_param + e0;
-    hd->g = t_grad + e0;
-    hd->e0 = (uint64_t)(t_eoff + e0);   // keys the draws
-    hd->state = (t_flags & kKindFp32) ? (uint64_t)(t_soff + e0) : (uint64_t)(t_soff + ub);
-    hd->tensor_id = t_id;
-    hd->flags = has ? (t_flags | (staged ? kStaged : 0u)) : kNoUnit;
-    hd->decay = t_decay;
-    hd->nvalid = nvalid;
-    // Runs of whole blocks of one tensor are contiguous in global memory and
-    // in the stage: one bulk copy per array per run.
-    const unsigned staged_mask = __ballot_sync(kMask, staged);
-    const int prev_ti = __shfl_up_sync(kMask, ti, 1);
-    const bool cont = staged && lane > 0 && ((staged_mask >> (lane - 1)) & 1u) && prev_ti == ti;
-    const unsigned cont_mask = __ballot_sync(kMask, cont);
-    const uint32_t dst = stages_s + (uint32_t)(s * kStageBytes);
-    uint32_t tx = (uint32_t)__popc(staged_mask) * kUnitTx;
-    if (BF16W) tx -= (uint32_t)__popc(__ballot_sync(kMask, staged && wbf)) * 256u;
-    if (lane == 0) mbar_arrive_expect_tx(full, tx);
-    if (BF16W) {
-      // A run's weights land packed at the start of its own units' 512-B w
-      // slots: 512 B per unit for fp32, 256 B for bf16.  The run starts at the
-      // nearest lane at or below this one that does not continue a run.
-      const int start = 31 - __clz(~cont_mask & ((2u << lane) - 1u));
-      hd->w_soff = (uint32_t)(kOffW + start * 512 + (lane - start) * (wbf ? 256 : 512));
-    }
-    if (staged && !cont && !a.fault_stall) {
-      // this lane starts a run: it extends over the following lanes whose
-      // unit continues it
-      const unsigned rest = ~(cont_mask >> (lane + 1));
-      const int len = __ffs(rest);          // 1 + number of continuing lanes
-      const int64_t blk = t_soff + ub;
-      if (wbf)
-        bulk_g2s(dst + kOffW + lane * 512, reinterpret_cast<const uint16_t*>(t_param) + e0,
-                 256u * len, full);
-      else
-        bulk_g2s(dst + kOffW + lane * 512, t_param + e0, 512u * len, full);
-      bulk_g2s(dst + kOffG + lane * 256, t_grad + e0, 256u * len, full);
-      bulk_g2s(dst + kOffMC + lane * 64, st.mcodes + blk * (kBlock / 2), 64u * len, full);
-      bulk_g2s(dst + kOffVC + lane * 64, st.vcodes + blk * (kBlock / 2), 64u * len, full);
-    }
-    if (staged && !a.fault_stall) {
-      const int64_t blk = t_soff + ub;
-      cp_async4(dst + kOffMS + lane * 4, st.mscale + blk);
-      cp_async4(dst + kOffVS + lane * 4, st.vscale + blk);
-    }
-    cp_async_arrive_noinc(full);            // one arrival per lane, when its copies land
-    // (test hook: with the stall armed no bulk copy is issued, so the expected
-    // bytes never arrive and the consumers' waits run out)
-    if (++s == kStages) {
-      s = 0;
-      ++round;
-    }
-  }
-  cp_async_wait_all();
-}
-
-// ---------------------------------------------------------------------------
-// The step kernel
-// ---------------------------------------------------------------------------
-
-template <int VCODE, bool BF16W>
-__global__ void __launch_bounds__(kCtaThreads, 3)
-adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_end, StepArgs a,
-                   CodeTables tabs, StateArena st) {
-  extern __shared__ __align__(128) uint8_t s_stage[];
-  __shared__ __align__(8) uint64_t s_full[kStages];
-  __shared__ __align__(8) uint64_t s_empty[kStages];
-  __shared__ SmemTables S;
-
-  {
-    const int t = threadIdx.x;
-    if (t < 256) {
-      S.mpair[t] = make_float2(tabs.nf4[t & 15], tabs.nf4[t >> 4]);
-      const bool zx = (VCODE == kVZe || VCODE == kVZeFloor);   // zero-excluded code
-      const float lo = zx ? __fmul_rn((float)((t & 15) + 1), 0.0625f) : tabs.vz[t & 15];
-      const float hi = zx ? __fmul_rn((float)((t >> 4) + 1), 0.0625f) : tabs.vz[t >> 4];
-      S.vpair[t] = make_float2(lo, hi);
-    }
-    if (t < 128) S.rtn[t] = tabs.rtn[t];
-    if (t < 16) {
-      S.nf4[t] = tabs.nf4[t];
-      S.gap[t] = tabs.nf4_gap[t];
-      S.vz[t] = tabs.vz[t];
-      S.zip[t] = make_float4(t == 15 ? INFINITY : tabs.vz[t], tabs.vz_sqrt[max(t - 1, 0)],
-                             tabs.vz_sqrt[t], tabs.vz_sqrt[min(t + 1, 15)]);
-      S.vzp[t] = make_float2(tabs.vz[t], tabs.vz[min(t + 1, 15)]);
-      S.vzmid[t] = tabs.vz_mid[t];
-    }
-    if (t < kStages) {
-      // full: the producer's expect-tx arrive plus one cp.async arrive per
-      // producer lane; empty: one release per consumer half-warp
-      mbar_init(smem_addr(&s_full[t]), 1 + kHalves);
-      mbar_init(smem_addr(&s_empty[t]), kHalves);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  const uint32_t full0 = smem_addr(&s_full[0]);
-  const uint32_t empty0 = smem_addr(&s_empty[0]);
-  const int warp = threadIdx.x >> 5;
-  if (warp == kProducerWarp) {
-    const int lane = threadIdx.x & 31;
-    if (lane < kHalves) produce<BF16W>(T, u_begin, u_end, a, st, s_stage, full0, empty0, lane);
-    return;
-  }
-
-  // ---- consumers: half-warp `half` takes unit `half` of every tile ----
-  const int lane = threadIdx.x & 15;
-  const int half = threadIdx.x >> 4;
-  const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
-  const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
-  int s = 0;
-  uint32_t parity = 0;
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const uint32_t full = full0 + 8u * s;
-    const uint32_t empty = empty0 + 8u * s;
-    if (!__all_sync(hmask, wait_phase(full, parity, kWaitLimitNs))) {
-      if (lane == 0) atomicOr(a.status, 1u);
-      return;
-    }
-    const uint8_t* sp = s_stage + s * kStageBytes;
-    const UnitHeader* hdp = reinterpret_cast<const UnitHeader*>(sp + kOffHdr) + half;
-    const uint32_t flags = hdp->flags;
-    if (flags & kStaged) {
-      float w[kPerLane], g[kPerLane];
-      const bool wbf = BF16W && (flags & kBf16W);
-      {
-        const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
-        if (wbf) {
-          const uint4 wr = *reinterpret_cast<const uint4*>(sp + hdp->w_soff + lane * 16);
-          w[0] = bf16lo(wr.x); w[1] = bf16hi(wr.x); w[2] = bf16lo(wr.y); w[3] = bf16hi(wr.y);
-          w[4] = bf16lo(wr.z); w[5] = bf16hi(wr.z); w[6] = bf16lo(wr.w); w[7] = bf16hi(wr.w);
-        } else {
-          const uint8_t* wsrc = sp + kOffW + half * 512 + lane * 32;
-          const float4 wa = *reinterpret_cast<const float4*>(wsrc);
-          const float4 wb = *reinterpret_cast<const float4*>(wsrc + 16);
-          w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
-          w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
-        }
-        g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
-        g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
-      }
-      const uint32_t mc = *reinterpret_cast<const uint32_t*>(sp + kOffMC + half * 64 + lane * 4);
-      const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + half * 64 + lane * 4);
-      const float sm = *reinterpret_cast<const float*>(sp + kOffMS + half * 4);
-      const float sv = *reinterpret_cast<const float*>(sp + kOffVS + half * 4);
-
-      float m1[kPerLane], v1[kPerLane], den[kPerLane];
-      update8(a, S, hdp->decay, w, g, mc, vc, sm, sv, m1, v1, den);
-      if (wbf) {
-        uint16_t* wp = reinterpret_cast<uint16_t*>(hdp->w) + lane * kPerLane;
-        *reinterpret_cast<uint4*>(wp) = make_uint4(bf16x2_rn(w[0], w[1]), bf16x2_rn(w[2], w[3]),
-                                                   bf16x2_rn(w[4], w[5]), bf16x2_rn(w[6], w[7]));
-      } else {
-        float* wp = hdp->w + lane * kPerLane;
-        *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
-      }
-      const uint64_t blk = hdp->state;
-      uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
-      uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
-      requant_store<VCODE, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, kPerLane, hmask, m1,
-                                 v1, den, mcw, vcw, st.mscale + blk, st.vscale + blk);
-    } else if (!(flags & kNoUnit)) {
-      process_direct<VCODE, BF16W>(a, S, st, hdp, lane, hmask);
-    }
-    // every read of the stage (header included) is done: hand it back
-    fence_proxy_async_smem();
-    __syncwarp(hmask);
-    if (lane == 0) mbar_arrive(empty, 1);
-    if (++s == kStages) {
-      s = 0;
-      parity ^= 1u;
-    }
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Host side
@@ -1365,7 +499,14 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
   return ADAMW4_OK;
 }
 
+// NVTX range for the duration of one ABI call (tracing under nsys / ncu).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 extern "C" int adamw4_step(adamw4_handle* h, float lr, void* cuda_stream) {
+  NvtxRange nvtx("adamw4_step");
   if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
   if (!(lr >= 0.0f) || !std::isfinite(lr))
     return fail(h, ADAMW4_EINVAL, "lr must be finite and non-negative");
@@ -1381,6 +522,7 @@ extern "C" int adamw4_step(adamw4_handle* h, float lr, void* cuda_stream) {
 
 extern "C" int adamw4_step_host(adamw4_handle* h, float lr, const uint16_t* const* grads_host,
                                 float* const* params_host, void* cuda_stream) {
+  NvtxRange nvtx("adamw4_step_host");
   if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
   if (!(lr >= 0.0f) || !std::isfinite(lr))
     return fail(h, ADAMW4_EINVAL, "lr must be finite and non-negative");
