@@ -478,9 +478,7 @@ def run_zero1(args):
             "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
-    for s_ in opt.steppers:
-        if s_ is not None:
-            s_.close()
+    opt.close()
     dist.destroy_process_group()
     return 0
 

@@ -307,6 +307,13 @@ class ZeroAdamW4:
             blobs.update(p)
         return merge_state(self.layout, self.specs, blobs)
 
+    def close(self):
+        """Frees this rank's handles (also done when they are collected)."""
+        for s in self.steppers:
+            if s is not None and hasattr(s, "close"):
+                s.close()
+        self.steppers = [None] * len(self.steppers)
+
     def load_consolidated_state(self, blob: bytes):
         """Loads this rank's pieces from a whole-list blob (saved at any world
         size or chunk count) and takes its step counter."""

@@ -150,9 +150,8 @@ def test_zero1_over_nccl_one_rank(vcode):
         for i, p in enumerate(params):
             assert L2.tensor_view(fp2, i).cpu().numpy().tobytes() == p.cpu().numpy().tobytes()
         assert opt2.consolidated_state() == whole.state_dict_blob()
-        for s in opt.steppers + opt2.steppers:
-            if s is not None:
-                s.close()
+        opt.close()
+        opt2.close()
         whole.close()
     finally:
         dist.destroy_process_group()
