@@ -1,5 +1,5 @@
 """ZeRO-1 sharding on CPU: the flat layout, the checkpoint merge, the oracle on
-pieces, and the sharded step over gloo ranks (world size 2).
+pieces, and the sharded step over gloo ranks (world sizes 2 and 3).
 
 The invariant: the sharded step (reduce-scatter, step of each rank's pieces,
 all-gather) gives the same weights and state, bit for bit, as the oracle's
@@ -202,32 +202,35 @@ def _rank(rank, world, port, root, vcode, chunks, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("vcode,chunks", [(0, 1), (1, 2), (4, 3)])
-def test_two_gloo_ranks_equal_the_whole_step(vcode, chunks):
+@pytest.mark.parametrize("world,vcode,chunks", [(2, 0, 1), (2, 1, 2), (2, 4, 3), (3, 0, 2)])
+def test_gloo_ranks_equal_the_whole_step(world, vcode, chunks):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, root, vcode, chunks, q))
-             for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, root, vcode, chunks, q))
+             for r in range(world)]
     for p in procs:
         p.start()
-    res = dict((r[0], r[1:]) for r in (q.get(timeout=180), q.get(timeout=180)))
+    res = dict((r[0], r[1:]) for r in (q.get(timeout=180) for _ in range(world)))
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (red0, blob0, final0, w0, t0), (red1, blob1, final1, w1, t1) = res[0], res[1]
-    assert blob0 == blob1 and final0 == final1 and t0 == t1 == TOTAL_STEPS
-    for a, b in zip(w0, w1):
-        assert a.tobytes() == b.tobytes()
+    red0, blob0, final0, w0, t0 = res[0]
+    for r in range(1, world):
+        red, blob, final, w, t = res[r]
+        assert blob == blob0 and final == final0 and t == t0 == TOTAL_STEPS
+        for a, b in zip(w0, w):
+            assert a.tobytes() == b.tobytes()
+        for a, b in zip(red0, red):
+            assert a.tobytes() == b.tobytes()
     # the whole list on one process, on the reduced gradients
-    ws, _ = _inputs(2)
+    ws, _ = _inputs(world)
     full = oracle.OracleAdamW4(tensors=SPECS, vcode=vcode, seed=77, total_steps=TOTAL_STEPS)
     wf = [w.copy() for w in ws]
     for t in range(TOTAL_STEPS):
-        L = FlatLayout([s["numel"] for s in SPECS], 2, chunks if t < TOTAL_STEPS - 1
+        L = FlatLayout([s["numel"] for s in SPECS], world, chunks if t < TOTAL_STEPS - 1
                        else chunks + 1)
-        assert red0[t].tobytes() == red1[t].tobytes()
         g = [L.tensor_view(torch.from_numpy(red0[t]), i).numpy().view(np.uint16).copy()
              for i in range(len(SPECS))]
         full.step(wf, g)
