@@ -83,7 +83,7 @@ def assert_state_equal(blob_gpu, blob_ref, vcode, what=""):
                                        err_msg=tag + " v scales")
 
 
-class GpuRun:
+class CudaRun:
     """The CUDA path over a tensor list with host-provided inputs."""
 
     def __init__(self, ts, host_ws, vcode=0, seed=0, total_steps=0, lr=1e-3, beta1=0.9,
@@ -137,7 +137,7 @@ def run_both(ts, host_ws, grads_fn, steps, vcode=0, seed=0, total_steps=0, blob=
     """Steps the CUDA path and the oracle `steps` times from the same inputs
     and compares state and weights (after every step if asked, else at the
     end).  grads_fn(step) returns the host bf16 grads of that step."""
-    gpu = GpuRun(ts, host_ws, vcode=vcode, seed=seed, total_steps=total_steps, blob=blob, t0=t0)
+    gpu = CudaRun(ts, host_ws, vcode=vcode, seed=seed, total_steps=total_steps, blob=blob, t0=t0)
     ref = oracle_for(ts, vcode=vcode, seed=seed, total_steps=total_steps)
     if blob is not None:
         ref.import_state(blob)

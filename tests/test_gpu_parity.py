@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 import workloads
-from gpu_common import (GpuRun, assert_state_equal, assert_weights_close, binding, oracle_for,
+from gpu_common import (CudaRun, assert_state_equal, assert_weights_close, binding, oracle_for,
                         parse_blob, run_both)
 
 pytestmark = pytest.mark.gpu
@@ -96,7 +96,7 @@ def test_degenerate_values(vcode):
         return out
     run_both(ts, ws, grads, 6, vcode=vcode, check_every_step=True, what=f"degenerate v{vcode}")
     # lr = 0 leaves the weights unchanged (decay 1 - 0*wd = 1)
-    gpu = GpuRun(ts, ws, vcode=vcode)
+    gpu = CudaRun(ts, ws, vcode=vcode)
     try:
         gpu.step(grads(1), lr=0.0)
         for a, b in zip(gpu.weights(), ws):
@@ -124,17 +124,17 @@ def test_checkpoint_resume_bit_exact():
           for i, t in enumerate(ts)]
     gfn = lambda s: [workloads.bf16_bits((np.random.default_rng(50 + s).standard_normal(
         t["numel"]) * 1e-3).astype(np.float32)) for t in ts]
-    a = GpuRun(ts, ws)
+    a = CudaRun(ts, ws)
     for s in range(1, 7):
         a.step(gfn(s))
     wa, ba = a.weights(), a.blob()
     a.close()
-    b = GpuRun(ts, ws)
+    b = CudaRun(ts, ws)
     for s in range(1, 4):
         b.step(gfn(s))
     mid, wmid = b.blob(), b.weights()
     b.close()
-    c = GpuRun(ts, wmid, blob=mid)
+    c = CudaRun(ts, wmid, blob=mid)
     assert c.opt.t == 3
     for s in range(4, 7):
         c.step(gfn(s))
@@ -148,7 +148,7 @@ def test_state_bytes_match_layout():
     B = binding()
     ts = workloads.tensor_list("microlm-p4")
     ws = [np.zeros(t["numel"], np.float32) for t in ts]
-    g = GpuRun(ts, ws)
+    g = CudaRun(ts, ws)
     try:
         assert g.opt.state_bytes() == 157952
         assert g.opt.state_bytes() == oracle_for(ts).state_bytes()
@@ -167,11 +167,11 @@ def test_host_buffer_step_matches_device_step():
           for i, t in enumerate(ts)]
     gs = [workloads.bf16_bits((np.random.default_rng(9).standard_normal(t["numel"]) * 1e-3)
                               .astype(np.float32)) for t in ts]
-    a = GpuRun(ts, ws)
+    a = CudaRun(ts, ws)
     a.step(gs)
     wa = a.weights()
     a.close()
-    b = GpuRun(ts, ws)
+    b = CudaRun(ts, ws)
     hg = [torch.from_numpy(g.view(np.int16)).pin_memory() for g in gs]
     hp = [torch.empty(t["numel"], dtype=torch.float32).pin_memory() for t in ts]
     B.adamw4_step_host(b.opt.handle, 1e-3, [x.data_ptr() for x in hg], [x.data_ptr() for x in hp],
@@ -190,7 +190,7 @@ def test_pipeline_wait_timeout_is_reported_and_context_survives():
     B = binding()
     ts = workloads.tensor_list("single-65k")
     ws = workloads.host_weights("single-65k", ts)
-    g = GpuRun(ts, ws)
+    g = CudaRun(ts, ws)
     try:
         B.adamw4_inject_fault(g.opt.handle, B.ADAMW4_FAULT_STALL_PIPELINE)
         g.step(workloads.host_grads("single-65k", ts, 1))
