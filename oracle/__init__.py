@@ -255,7 +255,7 @@ def max_threads() -> int:
 
 
 # ----------------------------------------------------------------------------
-# Tensor-list driver with the C ABI's semantics.
+# The step over a tensor list, with the C ABI's semantics.
 # ----------------------------------------------------------------------------
 
 def is_fp32_state(numel: int, flags: int) -> bool:

@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 import test_oracle_bf16 as BF
-import test_oracle_driver as D
+import test_oracle_tensor_list as D
 import test_oracle_nf4 as N
 import test_oracle_philox as P
 import test_oracle_update as U

@@ -1,4 +1,4 @@
-"""The oracle's tensor-list driver: threads, partial blocks, checkpoints (CPU)."""
+"""The oracle over a tensor list: threads, partial blocks, checkpoints (CPU)."""
 import numpy as np
 import pytest
 
