@@ -22,7 +22,9 @@ __all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_V_ZI_RTN", "ADAMW4_V_ZI_
            "adamw4_state_buffers", "adamw4_step_noalloc", "ADAMW4_NOALLOC_MAX_TENSORS",
            "is_fp32_state", "LIB_PATH"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libadamw4.so")
+# ADAMW4_LIBRARY selects another build of the same library (the checked one)
+LIB_PATH = os.environ.get("ADAMW4_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libadamw4.so")
 
 ADAMW4_OK = 0
 ADAMW4_V_ZIPSR = 0
@@ -42,8 +44,10 @@ ADAMW4_ETIMEOUT = -7
 ADAMW4_NOALLOC_MAX_TENSORS = 1024
 ADAMW4_FAULT_STALL_PIPELINE = 1
 
+ADAMW4_ECHECK = -8
 STATUS = {0: "ADAMW4_OK", -1: "ADAMW4_EINVAL", -2: "ADAMW4_EALIGN", -3: "ADAMW4_ENOMEM",
-          -4: "ADAMW4_ECUDA", -5: "ADAMW4_ESTATE", -6: "ADAMW4_ERANGE", -7: "ADAMW4_ETIMEOUT"}
+          -4: "ADAMW4_ECUDA", -5: "ADAMW4_ESTATE", -6: "ADAMW4_ERANGE", -7: "ADAMW4_ETIMEOUT",
+          -8: "ADAMW4_ECHECK"}
 
 
 class AdamW4Error(RuntimeError):

@@ -30,20 +30,26 @@ def flags():
             "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "-shared", "-Xptxas", "-v"]
 
 
-def build(force=False, verbose=False):
-    if not force and os.path.exists(OUT) and all(
-            os.path.getmtime(OUT) >= os.path.getmtime(d) for d in DEPS):
-        return OUT
-    tmp = OUT + f".tmp{os.getpid()}"
-    cmd = [nvcc()] + flags() + [SRC, "-o", tmp]
+OUT_CHECKED = os.path.join(HERE, "libadamw4_checked.so")
+
+
+def build(force=False, verbose=False, checked=False):
+    """Builds libadamw4.so, or with checked=True libadamw4_checked.so, the
+    same library with device-side range checks (-DADAMW4_CHECKED)."""
+    out = OUT_CHECKED if checked else OUT
+    if not force and os.path.exists(out) and all(
+            os.path.getmtime(out) >= os.path.getmtime(d) for d in DEPS):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [nvcc()] + flags() + (["-DADAMW4_CHECKED"] if checked else []) + [SRC, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose:
         sys.stderr.write(r.stderr)
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv))

@@ -477,6 +477,8 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
   h->st.vscale = reinterpret_cast<float*>(base + o_vs);
   h->st.fm = reinterpret_cast<float*>(base + o_fm);
   h->st.fv = reinterpret_cast<float*>(base + o_fv);
+  h->st.nblocks4 = h->nblocks4;
+  h->st.n32 = h->nfp32;
   h->d_status = reinterpret_cast<uint32_t*>(base + o_st);
   if ((e = cudaMemset(h->d_arena, 0, h->arena_bytes)) != cudaSuccess ||
       (e = cudaMemcpy(h->d_tensors, dev.data(), sizeof(DevTensor) * dev.size(),
@@ -787,6 +789,10 @@ extern "C" int adamw4_sync(adamw4_handle* h, void* cuda_stream) {
   if (status != 0) {
     e = cudaMemset(h->d_status, 0, sizeof status);
     if (e != cudaSuccess) return cuda_fail(h, e, "clearing the status word");
+    if (status & 2u)
+      return fail(h, ADAMW4_ECHECK,
+                  "checked build: a unit's values or state lay outside its tensor or the arena; "
+                  "that unit was skipped");
     return fail(h, ADAMW4_ETIMEOUT,
                 "a stage wait in the step kernel ran out of time; the step is incomplete");
   }
@@ -945,6 +951,8 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   st.vscale = state->vscale;
   st.fm = state->m32;
   st.fv = state->v32;
+  st.nblocks4 = blocks4;
+  st.n32 = elems32;
   const int64_t need = (unit + kHalves - 1) / kHalves;
   launch_vcode(cfg->vcode, bf16w, (int)std::min<int64_t>(nd.grid[cfg->vcode][bf16w], need), s,
                table, 0, unit, a, tabs, st);

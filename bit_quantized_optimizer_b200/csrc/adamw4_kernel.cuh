@@ -140,6 +140,8 @@ struct StateArena {
   float* vscale;
   float* fm;         // fp32-state tensors
   float* fv;
+  int64_t nblocks4;  // blocks in the code and scale arrays (checked builds test against it)
+  int64_t n32;       // elements in fm and fv (likewise)
 };
 
 // What the producer tells the consumer about one unit (64 bytes).
@@ -689,7 +691,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
       return;
     }
     const int64_t u = u_begin + tile * kHalves + lane;
-    const bool has = u < u_end;
+    bool has = u < u_end;
     if (has && u >= t_end) {
       do {
         ++ti;
@@ -708,6 +710,21 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     }
     const int64_t ub = u - t_begin;
     const int64_t e0 = ub * kBlock;
+#ifdef ADAMW4_CHECKED
+    // Checked build: the unit's values lie inside its tensor and its state
+    // inside the arena; otherwise the status word gets bit 1 and the unit is
+    // dropped (no copy, no consumer work).
+    if (has) {
+      const int64_t nv = min((int64_t)kBlock, t_numel - e0);
+      const bool ok = ub >= 0 && nv > 0 && u < t_end &&
+                      ((t_flags & kKindFp32) ? (t_soff >= 0 && t_soff + e0 + nv <= st.n32)
+                                             : (t_soff >= 0 && t_soff + ub < st.nblocks4));
+      if (!ok) {
+        atomicOr(a.status, 2u);
+        has = false;
+      }
+    }
+#endif
     const int nvalid = has ? (int)min((int64_t)kBlock, t_numel - e0) : 0;
     const bool staged = has && !(t_flags & kKindFp32) && nvalid == kBlock;
     const bool wbf = BF16W && (t_flags & kBf16W);       // bf16 weights: 256 B per unit

@@ -58,7 +58,9 @@ typedef enum {
     ADAMW4_ECUDA = -4,      /* a CUDA runtime call or kernel launch failed     */
     ADAMW4_ESTATE = -5,     /* state blob does not match this handle           */
     ADAMW4_ERANGE = -6,     /* size above a stated maximum                     */
-    ADAMW4_ETIMEOUT = -7    /* a bounded wait inside the step kernel ran out   */
+    ADAMW4_ETIMEOUT = -7,   /* a bounded wait inside the step kernel ran out   */
+    ADAMW4_ECHECK = -8      /* library built with ADAMW4_CHECKED: a unit's values or
+                               state fell outside its tensor or the state arena */
 } adamw4_status;
 
 /* Faults adamw4_inject_fault can arm (test hooks; no GPU fault is raised). */
@@ -186,7 +188,11 @@ int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_ho
  * (about one second); when a wait runs out, the kernel records it in a device
  * status word and its half-warp stops, leaving that step incomplete.  This
  * call reads and clears the word: ADAMW4_ETIMEOUT if it was set, ADAMW4_ECUDA
- * on a CUDA error, else ADAMW4_OK.  The CUDA context stays usable. */
+ * on a CUDA error, else ADAMW4_OK.  The CUDA context stays usable.
+ * A library built with -DADAMW4_CHECKED (build.py --checked, a debugging aid
+ * in place of a memory checker) also tests every unit's element and state
+ * range on the device; a unit outside them is skipped and this call returns
+ * ADAMW4_ECHECK. */
 int adamw4_sync(adamw4_handle *h, void *cuda_stream);
 
 /* Test hook: arms `fault` (ADAMW4_FAULT_STALL_PIPELINE, or 0 to disarm) for
