@@ -165,7 +165,8 @@ def run_both(ts, host_ws, grads_fn, steps, vcode=0, seed=0, total_steps=0, blob=
 
 def sampled_blocks(ts, per_tensor=6, head_extra=192, seed=0):
     """Blocks to check per quantised tensor: the first, the last (the ragged
-    one if any) and a few random ones; more on the LM head."""
+    one if any) and a few random ones; more on the LM head; and, in a tensor
+    past 2^31 elements, the blocks on either side of element 2^31."""
     rng = np.random.default_rng(seed)
     out = {}
     for i, t in enumerate(ts):
@@ -174,6 +175,8 @@ def sampled_blocks(ts, per_tensor=6, head_extra=192, seed=0):
         nb = (t["numel"] + 127) // 128
         k = per_tensor + (head_extra if t["flags"] & workloads.T_LM_HEAD else 0)
         sel = {0, nb - 1} | set(rng.integers(0, nb, size=min(k, nb)).tolist())
+        if nb > (1 << 24) + 1:
+            sel |= {(1 << 24) - 1, 1 << 24, (1 << 24) + 1}
         out[i] = np.array(sorted(sel), np.int64)
     return out
 

@@ -60,3 +60,12 @@ def test_gpt_2p7b_sampled(vcode):
     for the two methods and the three state-space variants."""
     n = sampled_parity("gpt-2.7b", vcode=vcode, steps=2, t0=0, what=f"gpt-2.7b v{vcode}")
     assert n > 1500
+
+
+def test_tensor_past_2_31_elements():
+    """One 4-bit tensor of 2^31 + 300 values (element offsets and pointer
+    arithmetic past 32 bits, a ragged tail), with an LM head in its final-10%
+    phase and a norm tensor beside it; ZIP-SR, two steps, sampled blocks
+    including the two around element 2^31."""
+    n = sampled_parity("huge-2g", vcode=0, steps=2, t0=8, total_steps=10, what="huge-2g")
+    assert n > 100

@@ -155,3 +155,42 @@ def test_zero1_over_nccl_one_rank(vcode):
         whole.close()
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("vcode", [0, 1, 3])
+def test_pieces_at_large_element_offsets(vcode):
+    """Pieces far into their tensors: elem_offset 2^36 + 896 and 2^39 - 4096
+    (the largest allowed).  The Philox counter's high words are then in use
+    (element index / 4 >= 2^32); the kernel matches the oracle stepping the
+    same pieces by their blocks' indices in the whole tensor."""
+    import torch
+    B = binding()
+    from oracle_pieces import OraclePieces
+    Q = B.ADAMW4_T_QUANT_STATE
+    pspecs = [dict(numel=128 * 50 + 3, tensor_id=3, flags=Q, weight_decay=0.1,
+                   elem_offset=(1 << 36) + 896),
+              dict(numel=4096, tensor_id=4, flags=Q | B.ADAMW4_T_LM_HEAD, weight_decay=0.0,
+                   elem_offset=(1 << 39) - 4096)]
+    rng = np.random.default_rng(3)
+    ws = [(rng.standard_normal(s["numel"]) * 0.02).astype(np.float32) for s in pspecs]
+    params = [torch.from_numpy(w.copy()).cuda() for w in ws]
+    grads = [torch.zeros(s["numel"], dtype=torch.bfloat16, device="cuda") for s in pspecs]
+    opt = B.AdamW4(params, grads, pspecs, vcode=vcode, seed=99, total_steps=3)
+    cp = [torch.from_numpy(w.copy()) for w in ws]
+    cg = [torch.zeros(s["numel"], dtype=torch.bfloat16) for s in pspecs]
+    ref = OraclePieces(cp, cg, pspecs, vcode=vcode, seed=99, total_steps=3)
+    try:
+        for t in range(3):
+            for i, s in enumerate(pspecs):
+                hg = workloads.bf16_bits((np.random.default_rng(10 * t + i).standard_normal(
+                    s["numel"]) * 1e-3).astype(np.float32))
+                grads[i].view(torch.int16).copy_(torch.from_numpy(hg.view(np.int16)))
+                cg[i].view(torch.int16).copy_(torch.from_numpy(hg.view(np.int16)))
+            opt.step()
+            ref.step(1e-3)
+        torch.cuda.synchronize()
+        for p, c in zip(params, cp):
+            assert p.cpu().numpy().tobytes() == c.numpy().tobytes()
+        assert opt.state_dict_blob() == ref.state_dict_blob()
+    finally:
+        opt.close()

@@ -111,6 +111,9 @@ TENSOR_LISTS = {
     "microlm-p4": lambda: with_ids(gpt_tensors(2, 64, 256, 256, 64, tied=False)),
     "single-65k": lambda: with_ids([_t("w", 65536)]),
     "single-4m": lambda: with_ids([_t("w", 4194304)]),
+    # one 4-bit tensor past 2^31 elements (ragged tail), an LM head and a norm
+    "huge-2g": lambda: with_ids([_t("w", (1 << 31) + 300), _t("head", 128 * 4096, T_LM_HEAD),
+                                 _t("ln", 5000, T_NORM)]),
 }
 
 WORKLOADS = {
