@@ -231,7 +231,10 @@ int64_t adamw4_state_bytes(const adamw4_handle *h);
  * host_buf may be NULL to query).  adamw4_state_import reads such a blob into
  * a handle created over the same tensor list (same ids, kinds, numels,
  * vcode and seed, else ADAMW4_ESTATE) and sets t.  Both synchronise the device
- * and copy with the CUDA runtime. */
+ * and copy with the CUDA runtime.  The blob does not record elem_offset: a
+ * handle over pieces of tensors must be re-created over the same pieces, or
+ * the pieces' blobs merged into a whole-tensor blob and cut again for the new
+ * pieces (the Python zero1 module does both). */
 int adamw4_state_export(const adamw4_handle *h, void *host_buf, int64_t cap, int64_t *used);
 int adamw4_state_import(adamw4_handle *h, const void *host_buf, int64_t len);
 
