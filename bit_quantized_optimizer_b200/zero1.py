@@ -221,7 +221,8 @@ def split_state(layout: FlatLayout, specs, blob: bytes, rank: int, k: int) -> by
 class ZeroAdamW4:
     """ZeRO-1 AdamW4 over a process group.
 
-    ``flat_params`` (fp32) and ``flat_grads`` (bf16) are this rank's flat
+    ``flat_params`` (fp32, or bf16 for bf16 weights -- the all-gather then
+    moves half the bytes) and ``flat_grads`` (bf16) are this rank's flat
     buffers of ``layout.padded`` elements; the model's tensors are views
     ``layout.tensor_view(flat, i)``.  ``specs`` lists, per tensor, numel,
     tensor_id, flags and weight_decay.  Gradients are summed over the ranks
@@ -242,8 +243,9 @@ class ZeroAdamW4:
             raise ValueError("layout.world differs from the process group's size")
         if flat_params.numel() != layout.padded or flat_grads.numel() != layout.padded:
             raise ValueError("flat buffers must hold layout.padded elements")
-        if flat_params.dtype != torch.float32 or flat_grads.dtype != torch.bfloat16:
-            raise TypeError("flat params must be float32 and flat grads bfloat16")
+        if (flat_params.dtype not in (torch.float32, torch.bfloat16)
+                or flat_grads.dtype != torch.bfloat16):
+            raise TypeError("flat params must be float32 or bfloat16, flat grads bfloat16")
         if len(specs) != len(layout.numels) or any(
                 int(s["numel"]) != n for s, n in zip(specs, layout.numels)):
             raise ValueError("specs do not match the layout")

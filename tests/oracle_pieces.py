@@ -22,6 +22,10 @@ def _np_f32(t):
     return t.detach().numpy()
 
 
+def _is_bf16(t):
+    return t.dtype == torch.bfloat16
+
+
 def _np_u16(t):
     return t.detach().view(torch.int16).numpy().view(np.uint16)
 
@@ -54,11 +58,16 @@ class OraclePieces:
                                 np.float32(self.betas[1]), np.float32(self.eps), self.t,
                                 self.total_steps, self.seed)
         for p, g, spec, st in zip(self.params, self.grads, self.specs, self.state):
-            w, gb = _np_f32(p), _np_u16(g)
+            # bf16 weights: widened exactly, stepped in binary32, stored rounded
+            w = ((_np_u16(p).astype(np.uint32) << 16).view(np.float32) if _is_bf16(p)
+                 else _np_f32(p))
+            gb = _np_u16(g)
             n, e0 = spec["numel"], spec["elem_offset"]
             if st["kind"] == 1:
                 L.oracle_step_fp32(ctypes.byref(s), spec["weight_decay"], n, w, gb,
                                    st["m"], st["v"])
+                if _is_bf16(p):
+                    _np_u16(p)[:] = oracle.round_bf16(w)
                 continue
             nb = st["nb"]
             blocks = np.arange(e0 // 128, e0 // 128 + nb, dtype=np.int64)
@@ -71,7 +80,10 @@ class OraclePieces:
             L.oracle_step_blocks4(ctypes.byref(s), spec["weight_decay"], self.vcode, m_sr,
                                   spec["tensor_id"], e0 + n, nb, blocks, w_sel, g_sel,
                                   st["mcodes"], st["mscale"], st["vcodes"], st["vscale"])
-            w[:] = w_sel[:n]
+            if _is_bf16(p):
+                _np_u16(p)[:] = oracle.round_bf16(w_sel[:n])
+            else:
+                w[:] = w_sel[:n]
 
     def state_dict_blob(self) -> bytes:
         parts = []

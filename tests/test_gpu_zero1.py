@@ -194,3 +194,48 @@ def test_pieces_at_large_element_offsets(vcode):
         assert opt.state_dict_blob() == ref.state_dict_blob()
     finally:
         opt.close()
+
+
+@pytest.mark.parametrize("vcode", [0, 1])
+def test_emulated_shards_with_bf16_weights(vcode):
+    """The same emulation with bf16 weights in the flat buffer: the pieces'
+    handles keep bf16 weights and equal the whole-list handle bit for bit."""
+    import torch
+    B = binding()
+    from bit_quantized_optimizer_b200.zero1 import FlatLayout, merge_state, piece_spec
+    ws, gs = _host_inputs()
+    L = FlatLayout([s["numel"] for s in SPECS], 3, 2)
+    fp = torch.zeros(L.padded, dtype=torch.bfloat16, device="cuda")
+    fg = torch.zeros(L.padded, dtype=torch.bfloat16, device="cuda")
+    for i, w in enumerate(ws):
+        L.tensor_view(fp, i).copy_(torch.from_numpy(w))
+    handles = {}
+    for r in range(3):
+        for k in range(2):
+            ps = L.pieces(r, k)
+            if ps:
+                handles[(r, k)] = B.AdamW4([fp[p.flat:p.flat + p.numel] for p in ps],
+                                           [fg[p.flat:p.flat + p.numel] for p in ps],
+                                           [piece_spec(SPECS[p.tensor], p) for p in ps],
+                                           vcode=vcode, seed=21, total_steps=STEPS)
+    params = [torch.from_numpy(w).to(torch.bfloat16).cuda() for w in ws]
+    grads = [torch.zeros(s["numel"], dtype=torch.bfloat16, device="cuda") for s in SPECS]
+    whole = B.AdamW4(params, grads, SPECS, vcode=vcode, seed=21, total_steps=STEPS)
+    try:
+        for t in range(STEPS):
+            _flat_fill(torch, L, fg, gs[t])
+            for g, hg in zip(grads, gs[t]):
+                g.view(torch.int16).copy_(torch.from_numpy(hg.view(np.int16)))
+            for h in handles.values():
+                h.step()
+            whole.step()
+        torch.cuda.synchronize()
+        for i, p in enumerate(params):
+            a = L.tensor_view(fp, i).view(torch.int16).cpu().numpy()
+            assert a.tobytes() == p.view(torch.int16).cpu().numpy().tobytes(), f"tensor {i}"
+        merged = merge_state(L, SPECS, {rk: h.state_dict_blob() for rk, h in handles.items()})
+        assert merged == whole.state_dict_blob()
+    finally:
+        for h in handles.values():
+            h.close()
+        whole.close()

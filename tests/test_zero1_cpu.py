@@ -152,7 +152,13 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank(rank, world, port, root, vcode, chunks, out):
+def _wbits(t):
+    """Weights as comparable bytes: fp32, or bf16 bit patterns."""
+    return (t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16
+            else t.numpy()).copy()
+
+
+def _rank(rank, world, port, root, vcode, chunks, out, bf16=False):
     import sys
     sys.path.insert(0, root)
     sys.path.insert(0, os.path.join(root, "tests"))
@@ -167,7 +173,8 @@ def _rank(rank, world, port, root, vcode, chunks, out):
         cfg = dict(vcode=vcode, seed=77, total_steps=TOTAL_STEPS)
         ws, gs = _inputs(world)
         L = FlatLayout([s["numel"] for s in SPECS], world, chunks)
-        fp, fg = _flat(L, ws, torch.float32), torch.zeros(L.padded, dtype=torch.bfloat16)
+        wdt = torch.bfloat16 if bf16 else torch.float32
+        fp, fg = _flat(L, ws, wdt), torch.zeros(L.padded, dtype=torch.bfloat16)
 
         def make(p, g, s):
             return OraclePieces(p, g, s, **cfg)
@@ -184,8 +191,10 @@ def _rank(rank, world, port, root, vcode, chunks, out):
         blob = opt.consolidated_state()
         # resume the last step from the merged checkpoint in another layout
         L2 = FlatLayout([s["numel"] for s in SPECS], world, chunks + 1)
-        fp2, fg2 = _flat(L2, [L.tensor_view(fp, i).numpy() for i in range(len(SPECS))],
-                         torch.float32), torch.zeros(L2.padded, dtype=torch.bfloat16)
+        fp2 = torch.zeros(L2.padded, dtype=wdt)
+        for i in range(len(SPECS)):
+            L2.tensor_view(fp2, i).copy_(L.tensor_view(fp, i))
+        fg2 = torch.zeros(L2.padded, dtype=torch.bfloat16)
         opt2 = ZeroAdamW4(fp2, fg2, L2, SPECS, make_stepper=make, **cfg)
         opt2.load_consolidated_state(blob)
         fg2.copy_(_flat(L2, gs[-1][rank], torch.bfloat16))
@@ -196,19 +205,21 @@ def _rank(rank, world, port, root, vcode, chunks, out):
                                         opt2.grad_shard[k * L2.shard:(k + 1) * L2.shard])
         reduced.append(full_g.view(torch.int16).numpy().copy())
         final = opt2.consolidated_state()
-        weights = [L2.tensor_view(fp2, i).numpy().copy() for i in range(len(SPECS))]
+        weights = [_wbits(L2.tensor_view(fp2, i)) for i in range(len(SPECS))]
         out.put((rank, reduced, blob, final, weights, opt2.t))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,vcode,chunks", [(2, 0, 1), (2, 1, 2), (2, 4, 3), (3, 0, 2)])
-def test_gloo_ranks_equal_the_whole_step(world, vcode, chunks):
+@pytest.mark.parametrize("world,vcode,chunks,bf16", [(2, 0, 1, False), (2, 1, 2, False),
+                                                      (2, 4, 3, False), (3, 0, 2, False),
+                                                      (2, 0, 2, True)])
+def test_gloo_ranks_equal_the_whole_step(world, vcode, chunks, bf16):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, root, vcode, chunks, q))
+    procs = [ctx.Process(target=_rank, args=(r, world, port, root, vcode, chunks, q, bf16))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -226,8 +237,9 @@ def test_gloo_ranks_equal_the_whole_step(world, vcode, chunks):
             assert a.tobytes() == b.tobytes()
     # the whole list on one process, on the reduced gradients
     ws, _ = _inputs(world)
-    full = oracle.OracleAdamW4(tensors=SPECS, vcode=vcode, seed=77, total_steps=TOTAL_STEPS)
-    wf = [w.copy() for w in ws]
+    specs = [dict(s, flags=s["flags"] | (oracle.T_BF16_PARAM if bf16 else 0)) for s in SPECS]
+    full = oracle.OracleAdamW4(tensors=specs, vcode=vcode, seed=77, total_steps=TOTAL_STEPS)
+    wf = [oracle.round_bf16(w) if bf16 else w.copy() for w in ws]
     for t in range(TOTAL_STEPS):
         L = FlatLayout([s["numel"] for s in SPECS], world, chunks if t < TOTAL_STEPS - 1
                        else chunks + 1)
