@@ -425,7 +425,8 @@ def run_zero1(args):
     vcode = VCODES[args.vcode]
     ts = workloads.tensor_list(WORKLOAD)
     layout = FlatLayout([t["numel"] for t in ts], ws_, args.chunks)
-    fp = torch.empty(layout.padded, dtype=torch.float32, device="cuda")
+    wdt = torch.bfloat16 if args.bf16_params else torch.float32
+    fp = torch.zeros(layout.padded, dtype=wdt, device="cuda")
     fg = torch.zeros(layout.padded, dtype=torch.bfloat16, device="cuda")
     # the same weights on every rank, each rank's own gradients
     params, _ = workloads.device_inputs(WORKLOAD, ts, seed=0)
@@ -466,10 +467,11 @@ def run_zero1(args):
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "vcode": args.vcode, "params": nparams,
                        "tensors": len(ts), "parallelism": f"zero1 x{ws_}",
+                       "weights": "bf16" if args.bf16_params else "fp32",
                        "chunks": args.chunks, "shard_elems_per_chunk": layout.shard,
                        "reduce_scatter_bytes_per_rank": 2 * layout.padded,
-                       "all_gather_bytes_per_rank": 4 * layout.padded,
-                       "algorithmic_bytes_per_step": algorithmic_bytes(ts),
+                       "all_gather_bytes_per_rank": fp.element_size() * layout.padded,
+                       "algorithmic_bytes_per_step": algorithmic_bytes(ts, fp.element_size()),
                        "l2": "inputs 19.7 GB > 126 MB L2; no flush"},
             "roofline": None,
             "e2e": None,
