@@ -97,9 +97,12 @@ int main(int argc, char **argv)
 
     int64_t t = -1, used = 0;
     CHECK(adamw4_get_step(h, &t) == ADAMW4_OK && t == steps, "step counter");
-    CHECK(adamw4_state_export(h, NULL, 0, &used) == ADAMW4_ERANGE && used > 0, "export size");
+    CHECK(adamw4_state_export(h, NULL, 0, &used) == ADAMW4_OK && used > 40, "export size query");
     void *blob = malloc((size_t)used);
     CHECK(blob != NULL, "malloc");
+    int64_t used2 = 0;
+    CHECK(adamw4_state_export(h, blob, used - 1, &used2) == ADAMW4_ERANGE && used2 == used,
+          "a buffer one byte short must be refused");
     CHECK(adamw4_state_export(h, blob, used, &used) == ADAMW4_OK, "export");
 
     FILE *out = fopen(argv[2], "wb");
