@@ -1,7 +1,7 @@
 /*
  * c_client.c -- a plain C program that drives libadamw4 through its C ABI
  * only (include/adamw4.h), with the CUDA runtime for device memory.  Used by
- * tests/test_gpu_c_client.py: it reads a tensor list, weights and per-step
+ * tests/test_c_client.py: it reads a tensor list, weights and per-step
  * gradients from a file, runs the steps, and writes the weights and the
  * exported state blob back, for the test to compare with the oracle.
  *
