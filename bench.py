@@ -39,7 +39,7 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 WORKLOAD = "gpt-2.7b"        # the benchmark workload; --workload picks a profiling case
-VCODES = {"zipsr": 0, "zeeden": 1, "zi_rtn": 2, "zi_sr": 3, "ze_floor": 4}
+VCODES = {"zipsr": 0, "zeeden": 1, "zi_rtn": 2, "zi_sr": 3, "ze_floor": 4, "zipsr_u32": 5}
 METRIC = "fused 4-bit AdamW step Gparams/s; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
 # the device code of the step (the C ABI around it is in adamw4.cu)

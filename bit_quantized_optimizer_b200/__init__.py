@@ -13,7 +13,7 @@ import ctypes
 import os
 
 __all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_V_ZI_RTN", "ADAMW4_V_ZI_SR",
-           "ADAMW4_V_ZE_FLOOR", "ADAMW4_T_NORM", "ADAMW4_T_LM_HEAD",
+           "ADAMW4_V_ZE_FLOOR", "ADAMW4_V_ZIPSR_U32", "ADAMW4_T_NORM", "ADAMW4_T_LM_HEAD",
            "ADAMW4_T_FP32_STATE", "ADAMW4_T_QUANT_STATE", "ADAMW4_T_BF16_PARAM", "AdamW4Error", "adamw4_tensor", "adamw4_config", "lib",
            "adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
            "adamw4_get_step", "adamw4_set_step", "adamw4_state_bytes", "adamw4_state_export",
@@ -32,6 +32,7 @@ ADAMW4_V_ZEEDEN = 1
 ADAMW4_V_ZI_RTN = 2      # zero-inclusive code, state-space nearest
 ADAMW4_V_ZI_SR = 3       # zero-inclusive code, state-space stochastic rounding
 ADAMW4_V_ZE_FLOOR = 4    # zero-excluded code, nearest, no rescale
+ADAMW4_V_ZIPSR_U32 = 5   # ZIP-SR deciding on the whole 32-bit draw
 ADAMW4_T_NORM = 1
 ADAMW4_T_LM_HEAD = 2
 ADAMW4_T_FP32_STATE = 4

@@ -233,7 +233,7 @@ int validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n) {
     return fail(nullptr, ADAMW4_EINVAL, "eps must be positive and finite");
   if (!(cfg->lr >= 0.0f) || !std::isfinite(cfg->lr))
     return fail(nullptr, ADAMW4_EINVAL, "lr must be finite and non-negative");
-  if (cfg->vcode < ADAMW4_V_ZIPSR || cfg->vcode > ADAMW4_V_ZE_FLOOR)
+  if (cfg->vcode < ADAMW4_V_ZIPSR || cfg->vcode > ADAMW4_V_ZIPSR_U32)
     return fail(nullptr, ADAMW4_EINVAL, "vcode must be one of the adamw4_vcode values");
   if (cfg->total_steps < 0) return fail(nullptr, ADAMW4_EINVAL, "total_steps must be >= 0");
   if (n < 0 || (n > 0 && ts == nullptr))
@@ -304,6 +304,7 @@ int grid_for_w(int vcode, int device, int* grid) {
     case kVZiRtn: return occupancy_grid<kVZiRtn, BF16W>(device, grid);
     case kVZiSr: return occupancy_grid<kVZiSr, BF16W>(device, grid);
     case kVZeFloor: return occupancy_grid<kVZeFloor, BF16W>(device, grid);
+    case kVZip32: return occupancy_grid<kVZip32, BF16W>(device, grid);
     default: return (int)cudaErrorInvalidValue;
   }
 }
@@ -332,8 +333,11 @@ void launch_w(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t u
     case kVZiSr:
       adamw4_step_kernel<kVZiSr, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
       break;
-    default:
+    case kVZeFloor:
       adamw4_step_kernel<kVZeFloor, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
+      break;
+    default:
+      adamw4_step_kernel<kVZip32, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
       break;
   }
 }
@@ -844,7 +848,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 struct NoAllocDevice {
   bool ready;
   unsigned char* scratch;   // device address of g_noalloc_scratch on this device
-  int grid[ADAMW4_V_ZE_FLOOR + 1][2];   // per vcode, without / with bf16 weights
+  int grid[ADAMW4_V_ZIPSR_U32 + 1][2];  // per vcode, without / with bf16 weights
 };
 
 std::mutex g_noalloc_mu;
@@ -861,7 +865,7 @@ int na_validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n,
   if (!(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) || !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f))
     return ADAMW4_EINVAL;
   if (!(cfg->eps > 0.0f) || !std::isfinite(cfg->eps)) return ADAMW4_EINVAL;
-  if (cfg->vcode < ADAMW4_V_ZIPSR || cfg->vcode > ADAMW4_V_ZE_FLOOR) return ADAMW4_EINVAL;
+  if (cfg->vcode < ADAMW4_V_ZIPSR || cfg->vcode > ADAMW4_V_ZIPSR_U32) return ADAMW4_EINVAL;
   if (cfg->total_steps < 0 || t < 1) return ADAMW4_EINVAL;
   if (!(lr >= 0.0f) || !std::isfinite(lr)) return ADAMW4_EINVAL;
   if (n < 0 || (n > 0 && ts == nullptr)) return ADAMW4_EINVAL;
@@ -911,7 +915,7 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&nd.scratch), g_noalloc_scratch) !=
         cudaSuccess)
       return ADAMW4_ECUDA;
-    for (int vc = ADAMW4_V_ZIPSR; vc <= ADAMW4_V_ZE_FLOOR; ++vc)
+    for (int vc = ADAMW4_V_ZIPSR; vc <= ADAMW4_V_ZIPSR_U32; ++vc)
       for (int bw = 0; bw < 2; ++bw)
         if (grid_for(vc, bw != 0, device, &nd.grid[vc][bw]) != 0) return ADAMW4_ECUDA;
     nd.ready = true;

@@ -81,6 +81,7 @@ constexpr int kVZe = ADAMW4_V_ZEEDEN;
 constexpr int kVZiRtn = ADAMW4_V_ZI_RTN;
 constexpr int kVZiSr = ADAMW4_V_ZI_SR;
 constexpr int kVZeFloor = ADAMW4_V_ZE_FLOOR;
+constexpr int kVZip32 = ADAMW4_V_ZIPSR_U32;
 constexpr uint32_t kBf16W = ADAMW4_T_BF16_PARAM;  // weights stored as bf16
 constexpr uint32_t kKindFp32 = 1u << 16;          // internal flag: fp32-state tensor
 constexpr uint32_t kStaged = 1u << 17;            // internal flag: unit data is in the stage
@@ -374,7 +375,7 @@ struct SmemTables {
 // ZIP-SR codes of 8 values.  FLAT: also test for d(a) == d(b), which needs the
 // state-space fallback; callers skip it when the block's R makes that
 // impossible.
-template <bool FULL, bool FLAT>
+template <bool FULL, bool FLAT, bool U32>
 __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
                                                  const float (&v1)[kPerLane],
                                                  const float (&den)[kPerLane],
@@ -401,18 +402,31 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
     // fma(y, -1, x) rounds like x - y
     const float2 B = __fmul2_rn(__ffma2_rn(da, f2(-1.0f), db), dv);      // (db - da) * dv
     const float2 rhs = __fmul2_rn(__ffma2_rn(dv, f2(-1.0f), db), da);    // (db - dv) * da
-    const float2 f = make_float2(one_plus_u(rw[2 * j]), one_plus_u(rw[2 * j + 1]));
-    const float2 lhs = __ffma2_rn(f, B, make_float2(-B.x, -B.y));         // u * B
-    bool lowa = lhs.x < rhs.x, lowb = lhs.y < rhs.y;
+    bool lowa, lowb;
+    if (U32) {
+      // the whole word: (w 2^-32) * B rounded once in binary64, against rhs
+      lowa = __dmul_rn((double)rw[2 * j], (double)B.x * 0x1p-32) < (double)rhs.x;
+      lowb = __dmul_rn((double)rw[2 * j + 1], (double)B.y * 0x1p-32) < (double)rhs.y;
+    } else {
+      const float2 f = make_float2(one_plus_u(rw[2 * j]), one_plus_u(rw[2 * j + 1]));
+      const float2 lhs = __ffma2_rn(f, B, make_float2(-B.x, -B.y));       // u * B
+      lowa = lhs.x < rhs.x;
+      lowb = lhs.y < rhs.y;
+    }
     const uint32_t ka = k0a - (deca ? 1u : 0u), kb = k0b - (decb ? 1u : 0u);
     if (FLAT) {
       if (da.x == db.x) {
         const float2 z = S.vzp[ka];
-        lowa = __fmul_rn(__fsub_rn(f.x, 1.0f), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.x);
+        lowa = U32 ? __dmul_rn((double)rw[2 * j], (double)__fsub_rn(z.y, z.x) * 0x1p-32) <
+                         (double)__fsub_rn(z.y, x2.x)
+                   : __fmul_rn(uniform23(rw[2 * j]), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.x);
       }
       if (da.y == db.y) {
         const float2 z = S.vzp[kb];
-        lowb = __fmul_rn(__fsub_rn(f.y, 1.0f), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.y);
+        lowb = U32 ? __dmul_rn((double)rw[2 * j + 1], (double)__fsub_rn(z.y, z.x) * 0x1p-32) <
+                         (double)__fsub_rn(z.y, x2.y)
+                   : __fmul_rn(uniform23(rw[2 * j + 1]), __fsub_rn(z.y, z.x)) <
+                         __fsub_rn(z.y, x2.y);
       }
     }
     const uint32_t ca = (FULL || 2 * j < myn) ? ka + (lowa ? 0u : 1u) : 0u;
@@ -471,7 +485,7 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   float vso = 0.0f;
   if (av >= FLT_MIN) {
     const float inv = __fdiv_rn(1.0f, av);
-    if (VCODE == kVZip) {
+    if (VCODE == kVZip || VCODE == kVZip32) {
       // ZIP-SR ("ZIP-SR / ZE-EDEN", Core equation): keep the lower code point
       // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
       // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
@@ -481,9 +495,9 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       // d(a) == d(b) needs (sqrt(k+1/15) - sqrt(k/15)) R below two ulps of
       // R + eps; the smallest gap is 0.0339, so R > 1e-5 eps rules it out.
       if (R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN)
-        vco = zipsr_codes8<FULL, false>(a, S, v1, den, rw, inv, R, myn);
+        vco = zipsr_codes8<FULL, false, VCODE == kVZip32>(a, S, v1, den, rw, inv, R, myn);
       else
-        vco = zipsr_codes8<FULL, true>(a, S, v1, den, rw, inv, R, myn);
+        vco = zipsr_codes8<FULL, true, VCODE == kVZip32>(a, S, v1, den, rw, inv, R, myn);
       vso = av;
     } else if (VCODE == kVZiRtn || VCODE == kVZiSr) {
       // State-space rules on the zero-inclusive code: nearest code point, or

@@ -34,6 +34,7 @@ VCODE_ZEEDEN = 1
 VCODE_ZI_RTN = 2      # zero-inclusive code, state-space round-to-nearest
 VCODE_ZI_SR = 3       # zero-inclusive code, state-space stochastic rounding
 VCODE_ZE_FLOOR = 4    # zero-excluded code, no rescale
+VCODE_ZIPSR_U32 = 5   # ZIP-SR deciding on the whole 32-bit draw
 T_NORM = 1
 T_LM_HEAD = 2
 T_FP32_STATE = 4
@@ -103,6 +104,8 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_zi_sr.argtypes = [c.c_float, c.c_float]
     L.oracle_zipsr_decide.restype = c.c_int
     L.oracle_zipsr_decide.argtypes = [c.c_float] * 5
+    L.oracle_zipsr_decide_u32.restype = c.c_int
+    L.oracle_zipsr_decide_u32.argtypes = [c.c_float] * 4 + [c.c_uint32]
     L.oracle_zeeden_code.restype = c.c_int
     L.oracle_zeeden_code.argtypes = [c.c_float]
     L.oracle_zeeden_factor.restype = c.c_float
@@ -229,6 +232,10 @@ def zi_sr(x: float, u: float) -> int:
 
 def zipsr_decide(x: float, dv: float, R: float, eps: float, u: float) -> int:
     return int(lib().oracle_zipsr_decide(x, dv, R, eps, u))
+
+
+def zipsr_decide_u32(x: float, dv: float, R: float, eps: float, word: int) -> int:
+    return int(lib().oracle_zipsr_decide_u32(x, dv, R, eps, word))
 
 
 def zeeden_code(x: float) -> int:

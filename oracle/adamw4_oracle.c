@@ -51,6 +51,9 @@
 #define ORACLE_VCODE_ZI_RTN 2
 #define ORACLE_VCODE_ZI_SR 3
 #define ORACLE_VCODE_ZE_FLOOR 4
+/* ZIP-SR deciding on the whole 32-bit draw (the library's exact option: the
+ * probability is resolved to 2^-32 instead of the 23-bit uniform's 2^-23). */
+#define ORACLE_VCODE_ZIPSR_U32 5
 #define ORACLE_STREAM_V 0u        /* Philox stream for the v draw (ZIP-SR)        */
 #define ORACLE_STREAM_M 1u        /* Philox stream for the LM-head m draw         */
 
@@ -379,6 +382,30 @@ int oracle_zipsr_decide(float x, float dv, float R, float eps, float u)
     return lower ? k : k + 1;
 }
 
+/* The same decision taken on the whole 32-bit word w of the draw: with
+ * u = w 2^-32 (exact in binary64), the element goes low when the binary64
+ * product u * B, rounded once, is below rhs, where B = (db-da)*dv and
+ * rhs = (db-dv)*da are the binary32 values above (exact in binary64).  P(low)
+ * is then p rounded up to a multiple of 2^-32 instead of 2^-23.  The flat-h
+ * fallback takes its state-space rule in the same way. */
+int oracle_zipsr_decide_u32(float x, float dv, float R, float eps, uint32_t w)
+{
+    build_tables();
+    int k = oracle_zipsr_bracket(x);
+    float da = fmaf(g_vz_sqrt[k], R, eps);
+    float db = fmaf(g_vz_sqrt[k + 1], R, eps);
+    double u = (double)w * 0x1p-32;
+    int lower;
+    if (da == db) {
+        lower = u * (double)(g_vz[k + 1] - g_vz[k]) < (double)(g_vz[k + 1] - x);
+    } else {
+        float B = (db - da) * dv;
+        float rhs = (db - dv) * da;
+        lower = u * (double)B < (double)rhs;
+    }
+    return lower ? k : k + 1;
+}
+
 /* ZE-EDEN nearest zero-excluded code point (k+1)/16, ties to even on 16x. */
 int oracle_zeeden_code(float x)
 {
@@ -466,13 +493,16 @@ void oracle_block4(const oracle_scalars *s, float decay, int vcode, int m_sr, ui
         return;
     }
     float inv = 1.0f / av;
-    if (vcode == ORACLE_VCODE_ZIPSR) {
+    if (vcode == ORACLE_VCODE_ZIPSR || vcode == ORACLE_VCODE_ZIPSR_U32) {
         float R = sqrtf(av) * s->rs_bc2;
         for (int i = 0; i < nvalid; ++i) {
             float x = v1[i] * inv;
-            float u = oracle_uniform(oracle_draw_word(s->seed, s->t, tensor_id, ORACLE_STREAM_V,
-                                                      elem0 + (uint64_t)i));
-            set_nibble(vcodes, i, oracle_zipsr_decide(x, den[i], R, s->eps, u));
+            uint32_t w = oracle_draw_word(s->seed, s->t, tensor_id, ORACLE_STREAM_V,
+                                          elem0 + (uint64_t)i);
+            int c = (vcode == ORACLE_VCODE_ZIPSR)
+                        ? oracle_zipsr_decide(x, den[i], R, s->eps, oracle_uniform(w))
+                        : oracle_zipsr_decide_u32(x, den[i], R, s->eps, w);
+            set_nibble(vcodes, i, c);
         }
         *vscale = av;
     } else if (vcode == ORACLE_VCODE_ZI_RTN || vcode == ORACLE_VCODE_ZI_SR) {

@@ -53,7 +53,7 @@ P0 = 0x7F0000000000   # fake, aligned device addresses: validation never derefer
 
 
 @pytest.mark.parametrize("kw,code", [(dict(beta1=1.0), -1), (dict(beta2=-0.1), -1),
-                                     (dict(eps=0.0), -1), (dict(vcode=5), -1), (dict(vcode=-1), -1),
+                                     (dict(eps=0.0), -1), (dict(vcode=6), -1), (dict(vcode=-1), -1),
                                      (dict(total_steps=-1), -1), (dict(lr=float("nan")), -1)])
 def test_bad_config(L, kw, code):
     rc, _ = _create(_cfg(**kw), [B.adamw4_tensor(P0, P0 + (1 << 30), 4096, 0, 0, 0.0)])

@@ -50,7 +50,7 @@ def _host(torch, p):
     return p.cpu().numpy()
 
 
-@pytest.mark.parametrize("vcode", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("vcode", [0, 1, 2, 3, 4, 5])
 def test_bf16_weights_match_the_oracle(vcode):
     import torch
     B = binding()

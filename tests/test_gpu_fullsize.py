@@ -54,7 +54,7 @@ def test_llama_1p1b_zeeden_lm_head_phase_sampled():
     assert n > 1000
 
 
-@pytest.mark.parametrize("vcode", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("vcode", [0, 1, 2, 3, 4, 5])
 def test_gpt_2p7b_sampled(vcode):
     """GPT-style 2.7B list (the benchmark workload), two steps from zero state,
     for the two methods and the three state-space variants."""

@@ -24,7 +24,7 @@ def test_single_65k_zipsr_10_steps():
              what="single-65k")
 
 
-@pytest.mark.parametrize("vcode", [2, 3, 4])
+@pytest.mark.parametrize("vcode", [2, 3, 4, 5])
 def test_single_65k_state_space_variants_10_steps(vcode):
     """The state-space variants (zero-inclusive nearest and stochastic
     rounding, zero-excluded floor without rescale) on the 65,536-element
@@ -46,7 +46,8 @@ def test_single_4m_zeeden_20_steps():
 RAGGED = [1, 7, 100, 4095, 4096, 4097, 4096 + 5, 4096 + 37, 4096 + 120, 128 * 37 + 64, 8192]
 
 
-ALL_VCODES = [0, 1, 2, 3, 4]   # ZIP-SR, ZE-EDEN, and the three state-space variants
+# ZIP-SR, ZE-EDEN, the three state-space variants, and ZIP-SR on 32-bit draws
+ALL_VCODES = [0, 1, 2, 3, 4, 5]
 
 
 @pytest.mark.parametrize("vcode", ALL_VCODES)

@@ -49,7 +49,7 @@ def _whole(torch, B, ws, vcode):
     return params, grads, opt
 
 
-@pytest.mark.parametrize("vcode", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("vcode", [0, 1, 2, 3, 4, 5])
 @pytest.mark.parametrize("world,chunks", [(2, 1), (3, 2), (8, 3)])
 def test_emulated_shards_equal_the_whole_list(vcode, world, chunks):
     import torch
@@ -157,7 +157,7 @@ def test_zero1_over_nccl_one_rank(vcode):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("vcode", [0, 1, 3])
+@pytest.mark.parametrize("vcode", [0, 1, 3, 5])
 def test_pieces_at_large_element_offsets(vcode):
     """Pieces far into their tensors: elem_offset 2^36 + 896 and 2^39 - 4096
     (the largest allowed).  The Philox counter's high words are then in use

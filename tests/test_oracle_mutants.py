@@ -36,6 +36,9 @@ def pins(golden):
         ("ZIP-SR expectation", lambda: [Z.test_exact_expectation_of_h(*c) for c in Z.CASES[::7]]),
         ("ZIP-SR ends", Z.test_zero_and_top_are_deterministic),
         ("ZIP-SR bracket", Z.test_bracket_at_and_below_code_points),
+        ("ZIP-SR 32-bit expectation", lambda: [Z.test_u32_decision_exact_expectation(*c)
+                                               for c in Z.CASES[::9]]),
+        ("ZIP-SR 32-bit bias", Z.test_u32_decision_removes_the_23_bit_bias),
         ("ZE-EDEN codes", E.test_codes_are_nearest_zero_excluded_points),
         ("ZE-EDEN hand", E.test_factor_hand_computed_two_elements),
         ("ZE-EDEN grid", E.test_factor_is_one_on_the_grid),
@@ -91,11 +94,17 @@ MUTANTS = [
     ("floor code rescaled", "oracle_zeeden_code(v1[i] * inv));\n        *vscale = av;",
      "oracle_zeeden_code(v1[i] * inv));\n        *vscale = av * 1.01f;"),
     ("ZIP-SR a and b swapped",
-     "float da = fmaf(g_vz_sqrt[k], R, eps);\n    float db = fmaf(g_vz_sqrt[k + 1], R, eps);",
-     "float db = fmaf(g_vz_sqrt[k], R, eps);\n    float da = fmaf(g_vz_sqrt[k + 1], R, eps);"),
+     "float da = fmaf(g_vz_sqrt[k], R, eps);\n    float db = fmaf(g_vz_sqrt[k + 1], R, eps);"
+     "\n    int lower;",
+     "float db = fmaf(g_vz_sqrt[k], R, eps);\n    float da = fmaf(g_vz_sqrt[k + 1], R, eps);"
+     "\n    int lower;"),
     ("ZIP-SR probability in state space",
      "float lhs = u * ((db - da) * dv);\n        float rhs = (db - dv) * da;",
      "float lhs = u * (g_vz[k + 1] - g_vz[k]);\n        float rhs = g_vz[k + 1] - x;"),
+    ("32-bit draw scaled by 2^-31", "double u = (double)w * 0x1p-32;",
+     "double u = (double)w * 0x1p-31;"),
+    ("32-bit decision sides swapped", "lower = u * (double)B < (double)rhs;",
+     "lower = u * (double)B >= (double)rhs;"),
     ("ZIP-SR bracket excludes its lower end", "if (g_vz[i] <= x) k = i;",
      "if (g_vz[i] < x) k = i;"),
     ("ZE-EDEN code includes zero", "int k = (int)c - 1;", "int k = (int)c;"),

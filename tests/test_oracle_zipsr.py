@@ -195,3 +195,90 @@ def test_bracket_at_and_below_code_points():
         below = float(np.nextafter(vz[k], np.float32(-1)))
         assert oracle.zipsr_bracket(below) == k - 1
     assert oracle.zipsr_bracket(0.0) == 0
+
+
+# ---------------------------------------------------------------------------
+# ZIP-SR deciding on the whole 32-bit draw (v code 5)
+# ---------------------------------------------------------------------------
+
+W_STEP = 2.0 ** -32
+
+
+def p_low_exact_u32(x, dv, R, eps):
+    """Fraction of the 2^32 draw words for which the 32-bit decision keeps the
+    lower code point (the decision is monotone in the word; bisection)."""
+    k_lo = oracle.zipsr_decide_u32(x, dv, R, eps, 0)
+    k_hi = oracle.zipsr_decide_u32(x, dv, R, eps, 0xFFFFFFFF)
+    if k_lo == k_hi:
+        return (1.0 if k_lo == oracle.zipsr_bracket(x) else 0.0), k_lo
+    lo, hi = 0, 1 << 32
+    while lo < hi:
+        j = (lo + hi) // 2
+        if oracle.zipsr_decide_u32(x, dv, R, eps, j) == k_lo:
+            lo = j + 1
+        else:
+            hi = j
+    return lo * W_STEP, k_lo
+
+
+@pytest.mark.parametrize("s,xv,rs_bc2", CASES[::3])
+def test_u32_decision_exact_expectation(s, xv, rs_bc2):
+    """Over all 2^32 words the 32-bit decision's probability equals the pages'
+    formula in binary64 within 2^-32 plus the binary32 conditioning of the
+    cell, so E[h(Q)] = h(v) to that resolution."""
+    eps = f32(1e-8)
+    s = f32(s)
+    rs_bc2 = f32(rs_bc2)
+    _, _, vz, vzs = oracle.tables()
+    v = f32(np.float32(xv) * np.float32(s))
+    x = f32(np.float32(v) * (np.float32(1.0) / np.float32(s)))
+    R = f32(np.sqrt(np.float32(s)) * np.float32(rs_bc2))
+    dv = f32(np.float32(np.sqrt(np.float32(v))) * np.float32(rs_bc2) + np.float32(eps))
+    k = oracle.zipsr_bracket(x)
+    p, _ = p_low_exact_u32(x, dv, R, eps)
+    da = float(vzs[k]) * R + eps
+    db = float(vzs[k + 1]) * R + eps
+    if db == da:
+        return
+    p_ref = min(max((1 / dv - 1 / db) / (1 / da - 1 / db), 0.0), 1.0)
+    cond = 4 * 2.0 ** -24 * db / (db - da)
+    assert abs(p - p_ref) < 1e-6 * cond + W_STEP + cond
+    # the binary32 terms B and rhs fix the probability to binary32 precision:
+    # p is rhs/B rounded up to a multiple of 2^-32
+    B = f32(np.float32(np.float32(db) - np.float32(da)) * np.float32(dv))
+    rhs = f32(np.float32(np.float32(db) - np.float32(dv)) * np.float32(da))
+    if B > 0 and 0 <= rhs < B:
+        assert p == pytest.approx(np.ceil(rhs / B * 2.0 ** 32) * W_STEP, abs=2 * W_STEP)
+
+
+def test_u32_decision_removes_the_23_bit_bias():
+    """A value in the cell next to zero where the pages' probability is below
+    2^-23 (v = 1e-2, b = 2e-2, eps = 1e-8, no bias correction): the 23-bit
+    decision keeps zero with probability 2^-23, four times too often, and
+    E[h] is nearly twice h(v); the 32-bit decision is within 2^-32."""
+    eps = f32(1e-8)
+    s = f32(15 * 2e-2)                              # b = s/15 = 2e-2
+    v = f32(1e-2)
+    x = f32(np.float32(v) * (np.float32(1.0) / np.float32(s)))
+    R = f32(np.sqrt(np.float32(s)))
+    dv = f32(np.float32(np.sqrt(np.float32(v))) + np.float32(eps))
+    assert oracle.zipsr_bracket(x) == 0
+    _, _, vz, vzs = oracle.tables()
+    da, db = float(vzs[0]) * R + eps, float(vzs[1]) * R + eps
+    p_ref = (1 / dv - 1 / db) / (1 / da - 1 / db)
+    assert p_ref < 2.0 ** -23
+    p23, _ = p_low_exact(x, dv, R, eps)
+    p32, _ = p_low_exact_u32(x, dv, R, eps)
+    assert p23 == U_STEP                            # rounded up to one granule
+    assert abs(p32 - p_ref) < 2 * W_STEP + 1e-6 * p_ref
+    e_h = lambda p: p / da + (1 - p) / db          # noqa: E731
+    assert e_h(p23) > 1.8 / dv
+    assert abs(e_h(p32) - 1 / dv) < 1e-3 / dv
+
+
+def test_u32_decision_ends_are_deterministic():
+    eps = f32(1e-8)
+    R = f32(np.sqrt(np.float32(1e-6)))
+    for w in (0, 0x12345678, 0xFFFFFFFF):
+        assert oracle.zipsr_decide_u32(0.0, eps, R, eps, w) == 0
+        assert oracle.zipsr_decide_u32(1.0, R + eps, R, eps, w) == 15

@@ -114,7 +114,7 @@ def _flat(layout, arrays, dtype):
     return f
 
 
-@pytest.mark.parametrize("vcode", [0, 1, 3])
+@pytest.mark.parametrize("vcode", [0, 1, 3, 5])
 def test_oracle_pieces_equal_the_whole_step(vcode):
     """No collectives: the pieces of an 8 x 3 layout stepped one by one give the
     whole step's bits (weights and merged state)."""
