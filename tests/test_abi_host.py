@@ -156,3 +156,34 @@ def test_bf16_params_span_two_bytes_per_weight(L):
     finally:
         del os.environ["ADAMW4_FAIL_ALLOC"]
     assert rc == -3 and "injected" in B.adamw4_last_error()
+
+
+def _header_enums():
+    txt = open(os.path.join(ROOT, "include", "adamw4.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    vals = {}
+    for name, val in re.findall(r"\b(ADAMW4_[A-Z0-9_]+)\s*=\s*(-?[0-9]+)u?\b", txt):
+        vals[name] = int(val)
+    for name, val in re.findall(r"#define\s+(ADAMW4_[A-Z0-9_]+)\s+([0-9]+)", txt):
+        vals[name] = int(val)
+    return vals
+
+
+def test_binding_constants_match_the_header():
+    """Every status code, v code, flag and size the header defines has the same
+    value in the Python binding, and every status code has a name there."""
+    vals = _header_enums()
+    assert len(vals) >= 20
+    for name, v in vals.items():
+        if hasattr(B, name):
+            assert getattr(B, name) == v, name
+    for name in ("ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_V_ZI_RTN", "ADAMW4_V_ZI_SR",
+                 "ADAMW4_V_ZE_FLOOR", "ADAMW4_V_ZIPSR_U32", "ADAMW4_T_NORM", "ADAMW4_T_LM_HEAD",
+                 "ADAMW4_T_FP32_STATE", "ADAMW4_T_QUANT_STATE", "ADAMW4_T_BF16_PARAM",
+                 "ADAMW4_NOALLOC_MAX_TENSORS", "ADAMW4_ETIMEOUT", "ADAMW4_ECHECK"):
+        assert name in vals and getattr(B, name) == vals[name], name
+    codes = {v for n, v in vals.items() if n in (
+        "ADAMW4_OK", "ADAMW4_EINVAL", "ADAMW4_EALIGN", "ADAMW4_ENOMEM", "ADAMW4_ECUDA",
+        "ADAMW4_ESTATE", "ADAMW4_ERANGE", "ADAMW4_ETIMEOUT", "ADAMW4_ECHECK")}
+    assert codes == set(B.STATUS)
+    assert B.MIN_QUANT_NUMEL == vals["ADAMW4_MIN_QUANT_NUMEL"] and B.BLOCK == vals["ADAMW4_BLOCK"]
