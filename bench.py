@@ -485,6 +485,48 @@ def run_zero1(args):
     return 0
 
 
+def run_sweep(args):
+    """Single tensors of 4 K to 256 M values: the step's time per launch with
+    L2 flushed before every timed launch (a 256 MB write between launches,
+    outside the timed interval), for the v code chosen.  One JSON line per
+    size; a profiling aid beside the headline line, not the headline."""
+    import torch
+    import bit_quantized_optimizer_b200 as B
+    torch.cuda.set_device(0)
+    B.lib()
+    vcode = VCODES[args.vcode]
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for n in (1 << 12, 1 << 16, 1 << 20, 1 << 24, 1 << 28):
+        ts = [dict(numel=n, tensor_id=0, flags=0, weight_decay=0.1)]
+        gen = torch.Generator(device="cuda").manual_seed(n)
+        w = torch.empty(n, device="cuda").normal_(0.0, 0.02, generator=gen)
+        g = torch.empty(n, device="cuda").normal_(0.0, 1e-3, generator=gen).to(torch.bfloat16)
+        opt = B.AdamW4([w], [g], ts, vcode=vcode)
+        for _ in range(args.warmup):
+            opt.step()
+        times = []
+        for _ in range(max(args.steps // 10, 5)):
+            flush.fill_(1.0)                       # evict the tensor's data from L2
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            opt.step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = float(np.median(times))
+        alg = algorithmic_bytes(ts)
+        peak, _ = peaks()
+        print(json.dumps({"sweep": args.vcode, "numel": n, "ms_per_launch": ms,
+                          "gparams": n / (ms * 1e-3) / 1e9, "hbm_gbs": alg / (ms * 1e-3) / 1e9,
+                          "frac": alg / (ms * 1e-3) / 1e9 / peak, "l2": "flushed before each launch"}),
+              flush=True)
+        opt.close()
+        del w, g
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -499,6 +541,8 @@ def main():
                     help="keep every tensor's weights in bf16 (ADAMW4_T_BF16_PARAM)")
     ap.add_argument("--zero1", action="store_true",
                     help="time the ZeRO-1 sharded step (reduce-scatter, step, all-gather)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time single tensors of 4K..256M values (L2 flushed per launch)")
     ap.add_argument("--chunks", type=int, default=4,
                     help="ZeRO-1 pipeline chunks (collectives of one overlap the step of another)")
     ap.add_argument("--workload", default=WORKLOAD, choices=["gpt-2.7b", "llama-1.1b", "gpt-130m"],
@@ -510,6 +554,8 @@ def main():
         return run_reference(args)
     if args.zero1:
         return run_zero1(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 
