@@ -1,5 +1,5 @@
 """ZeRO-1 sharding on CPU: the flat layout, the checkpoint merge, the oracle on
-pieces, and the sharded step over gloo ranks (world sizes 2 and 3).
+pieces, and the sharded step over gloo ranks (world sizes 2, 3 and 4).
 
 The invariant: the sharded step (reduce-scatter, step of each rank's pieces,
 all-gather) gives the same weights and state, bit for bit, as the oracle's
@@ -213,7 +213,7 @@ def _rank(rank, world, port, root, vcode, chunks, out, bf16=False):
 
 @pytest.mark.parametrize("world,vcode,chunks,bf16", [(2, 0, 1, False), (2, 1, 2, False),
                                                       (2, 4, 3, False), (3, 0, 2, False),
-                                                      (2, 0, 2, True)])
+                                                      (4, 5, 2, False), (2, 0, 2, True)])
 def test_gloo_ranks_equal_the_whole_step(world, vcode, chunks, bf16):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
