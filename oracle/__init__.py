@@ -82,6 +82,8 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_draw_word.argtypes = [c.c_uint64, c.c_int64, c.c_uint32, c.c_uint32, c.c_uint64]
     L.oracle_uniform.restype = c.c_float
     L.oracle_uniform.argtypes = [c.c_uint32]
+    L.oracle_uniform32.restype = c.c_float
+    L.oracle_uniform32.argtypes = [c.c_uint32]
     L.oracle_nf4_levels_f64.argtypes = [_f64p]
     L.oracle_tables.argtypes = [_f32p, _f32p, _f32p, _f32p]
     L.oracle_make_scalars.argtypes = [c.c_float, c.c_float, c.c_float, c.c_float,
@@ -187,6 +189,11 @@ def draw_word(seed: int, t: int, tensor_id: int, stream: int, e: int) -> int:
 
 def uniform(word: int) -> float:
     return float(lib().oracle_uniform(word))
+
+
+def uniform32(word: int) -> float:
+    """The ZIP-SR uniform: the whole word rounded to binary32, times 2^-32."""
+    return float(lib().oracle_uniform32(word))
 
 
 def nf4_levels_f64() -> np.ndarray:

@@ -51,8 +51,8 @@
 #define ORACLE_VCODE_ZI_RTN 2
 #define ORACLE_VCODE_ZI_SR 3
 #define ORACLE_VCODE_ZE_FLOOR 4
-/* ZIP-SR deciding on the whole 32-bit draw (the library's exact option: the
- * probability is resolved to 2^-32 instead of the 23-bit uniform's 2^-23). */
+/* ZIP-SR deciding on the whole 32-bit draw with one binary64 multiply (the
+ * library's option beside the binary32 decision of ZIP-SR itself). */
 #define ORACLE_VCODE_ZIPSR_U32 5
 #define ORACLE_STREAM_V 0u        /* Philox stream for the v draw (ZIP-SR)        */
 #define ORACLE_STREAM_M 1u        /* Philox stream for the LM-head m draw         */
@@ -110,10 +110,26 @@ uint32_t oracle_draw_word(uint64_t seed, int64_t t, uint32_t tensor_id, uint32_t
 }
 
 /* Uniform in [0,1) with 2^-23 granularity: the low 23 bits of the word,
- * scaled by 2^-23 (exact in binary32). */
+ * scaled by 2^-23 (exact in binary32).  The LM-head first-moment draw and
+ * the state-space variants use it. */
 float oracle_uniform(uint32_t word)
 {
     return (float)(word & 0x7FFFFFu) * 0x1p-23f;
+}
+
+/* Uniform in [0,1] from the whole 32-bit word, for the ZIP-SR decision: the
+ * word rounded to the nearest binary32, times 2^-32 (exact).  Small words are
+ * exact (granularity 2^-32 near zero, where the cell next to zero needs it);
+ * above 2^24 the rounding is relative, 2^-24.  So the keep probability
+ * p = [h(v)-h(b)]/[h(a)-h(b)] of "ZIP-SR / ZE-EDEN" (Core equation) is
+ * realised to within 2^-32 + 2^-23 p, and E[h] to within
+ * 2^-32 (h(a)-h(b)) + 2^-23 h(v): unbiased in preconditioner space at the
+ * binary32 level, also where h(a) = 1/eps is large ("ZIP-SR 4-bit AdamW --
+ * Preconditioner-space stochastic rounding", car / stochastic rounding
+ * paragraph: the average multiplier is exact at storage time). */
+float oracle_uniform32(uint32_t word)
+{
+    return (float)word * 0x1p-32f;
 }
 
 /* ------------------------------------------------------------------------- */
@@ -360,7 +376,7 @@ int oracle_zi_sr(float x, float u)
 /* ZIP-SR decision for one element [D, Core equation]: the lower code point a
  * is kept with probability [h(v)-h(b)]/[h(a)-h(b)], h(y) = 1/(sqrt(y)*rs_bc2
  * + eps).  With d = 1/h this is (db - dv)*da / ((db - da)*dv); the element
- * goes low when u*((db-da)*dv) < (db-dv)*da.  x = v/s, dv = 1/h(v) as used in
+ * goes low when u*((db-da)*dv) < (db-dv)*da, u = oracle_uniform32(word).  x = v/s, dv = 1/h(v) as used in
  * the weight update, R = sqrt(s)*rs_bc2, so d at code point k is
  * sqrt(k/15)*R + eps.  If da == db in binary32 (h flat across the cell) the
  * preconditioner is the same either way and the rule falls back to state
@@ -500,7 +516,7 @@ void oracle_block4(const oracle_scalars *s, float decay, int vcode, int m_sr, ui
             uint32_t w = oracle_draw_word(s->seed, s->t, tensor_id, ORACLE_STREAM_V,
                                           elem0 + (uint64_t)i);
             int c = (vcode == ORACLE_VCODE_ZIPSR)
-                        ? oracle_zipsr_decide(x, den[i], R, s->eps, oracle_uniform(w))
+                        ? oracle_zipsr_decide(x, den[i], R, s->eps, oracle_uniform32(w))
                         : oracle_zipsr_decide_u32(x, den[i], R, s->eps, w);
             set_nibble(vcodes, i, c);
         }

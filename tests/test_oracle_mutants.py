@@ -38,7 +38,10 @@ def pins(golden):
         ("ZIP-SR bracket", Z.test_bracket_at_and_below_code_points),
         ("ZIP-SR 32-bit expectation", lambda: [Z.test_u32_decision_exact_expectation(*c)
                                                for c in Z.CASES[::9]]),
-        ("ZIP-SR 32-bit bias", Z.test_u32_decision_removes_the_23_bit_bias),
+        ("ZIP-SR zero-cell bias", lambda: [Z.test_zero_cell_has_no_23_bit_bias(v)
+                                           for v in (1e-2, 1e-3)]),
+        ("ZIP-SR block decisions", Z.test_block_decisions_follow_the_page_probability_on_the_word),
+        ("uniform32", P.test_uniform32_rounds_the_whole_word),
         ("ZE-EDEN codes", E.test_codes_are_nearest_zero_excluded_points),
         ("ZE-EDEN hand", E.test_factor_hand_computed_two_elements),
         ("ZE-EDEN grid", E.test_factor_is_one_on_the_grid),
@@ -70,6 +73,13 @@ MUTANTS = [
      "tensor_id * 2u + stream,\n                       (uint32_t)t}"),
     ("uniform takes 24 bits", "(float)(word & 0x7FFFFFu) * 0x1p-23f",
      "(float)(word & 0xFFFFFFu) * 0x1p-23f"),
+    ("ZIP-SR uniform scaled by 2^-31", "return (float)word * 0x1p-32f;",
+     "return (float)word * 0x1p-31f;"),
+    ("ZIP-SR uniform from the low 23 bits", "return (float)word * 0x1p-32f;",
+     "return (float)(word & 0x7FFFFFu) * 0x1p-23f;"),
+    ("ZIP-SR block step on the 23-bit uniform",
+     "oracle_zipsr_decide(x, den[i], R, s->eps, oracle_uniform32(w))",
+     "oracle_zipsr_decide(x, den[i], R, s->eps, oracle_uniform(w))"),
     ("NF4 offset", "const double offset = 0.9677083;", "const double offset = 0.96;"),
     ("NF4 negatives not normalised", "out[i] = neg[i] / top;", "out[i] = neg[i] / (top * 1.0001);"),
     ("first bias correction dropped", "s->step_size = (float)((double)lr / bc1);",

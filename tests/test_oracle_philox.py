@@ -55,12 +55,39 @@ def test_uniform_range_and_granularity():
     assert oracle.uniform(0x12345678) == (0x12345678 & 0x7FFFFF) * 2.0 ** -23
 
 
+def test_uniform32_rounds_the_whole_word():
+    """ZIP-SR's uniform is the whole word rounded to the nearest binary32
+    (ties to even), times 2^-32: exact below 2^24, relative rounding above."""
+    assert oracle.uniform32(0) == 0.0
+    assert oracle.uniform32(1) == 2.0 ** -32
+    assert oracle.uniform32(12345) == 12345 * 2.0 ** -32
+    assert oracle.uniform32((1 << 24) - 1) == ((1 << 24) - 1) * 2.0 ** -32
+    assert oracle.uniform32((1 << 24) + 1) == 2.0 ** -8           # tie to even: down
+    assert oracle.uniform32((1 << 24) + 3) == ((1 << 24) + 4) * 2.0 ** -32   # tie: up to even
+    assert oracle.uniform32(0x80000000) == 0.5
+    assert oracle.uniform32(0x80000080) == 0.5                    # 2^31 + 2^7: tie, even
+    assert oracle.uniform32(0x80000081) == 0.5 + 2.0 ** -24
+    assert oracle.uniform32(0xFFFFFFFF) == 1.0                    # rounds up to 2^32
+    assert oracle.uniform32(0xFFFFFF7F) == 1.0 - 2.0 ** -24
+    rng = np.random.default_rng(5)
+    for w in rng.integers(0, 1 << 32, 2000, dtype=np.uint64):
+        w = int(w)
+        u = oracle.uniform32(w)
+        # the nearest binary32 to w: no binary32 is closer
+        f = np.float32(u * 2.0 ** 32)
+        assert float(f) == u * 2.0 ** 32
+        assert abs(float(f) - w) <= abs(float(np.nextafter(f, np.float32(np.inf))) - w)
+        assert abs(float(f) - w) <= abs(float(np.nextafter(f, np.float32(0))) - w)
+
+
 def test_uniform_moments():
     # 2^16 draws: mean 1/2 and variance 1/12 within 5 sigma.
     n = 1 << 16
-    u = np.array([oracle.uniform(oracle.draw_word(1, 1, 0, 0, e)) for e in range(n)])
-    assert abs(u.mean() - 0.5) < 5 * np.sqrt(1 / 12 / n)
-    assert abs(u.var() - 1 / 12) < 5 * np.sqrt(1 / 180 / n)
+    words = [oracle.draw_word(1, 1, 0, 0, e) for e in range(n)]
+    for u in (np.array([oracle.uniform(w) for w in words]),
+              np.array([oracle.uniform32(w) for w in words])):
+        assert abs(u.mean() - 0.5) < 5 * np.sqrt(1 / 12 / n)
+        assert abs(u.var() - 1 / 12) < 5 * np.sqrt(1 / 180 / n)
 
 
 def _curand():

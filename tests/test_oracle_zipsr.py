@@ -14,6 +14,7 @@ import oracle
 
 U_STEP = 2.0 ** -23
 N_U = 1 << 23
+W_STEP = 2.0 ** -32
 
 
 def f32(x):
@@ -21,8 +22,26 @@ def f32(x):
 
 
 def p_low_exact(x, dv, R, eps):
-    """Fraction of the 2^23 uniforms for which the oracle keeps the lower code
-    point.  The decision is monotone in u; bisection finds the threshold."""
+    """Fraction of the 2^32 draw words for which ZIP-SR keeps the lower code
+    point, with the uniform ZIP-SR draws from a word (oracle.uniform32).  The
+    decision is monotone in the word; bisection finds the threshold."""
+    k_lo = oracle.zipsr_decide(x, dv, R, eps, oracle.uniform32(0))
+    k_hi = oracle.zipsr_decide(x, dv, R, eps, oracle.uniform32(0xFFFFFFFF))
+    if k_lo == k_hi:
+        return (1.0 if k_lo == oracle.zipsr_bracket(x) else 0.0), k_lo
+    lo, hi = 0, 1 << 32
+    while lo < hi:
+        j = (lo + hi) // 2
+        if oracle.zipsr_decide(x, dv, R, eps, oracle.uniform32(j)) == k_lo:
+            lo = j + 1
+        else:
+            hi = j
+    return lo * W_STEP, k_lo
+
+
+def p_low_exact_u23(x, dv, R, eps):
+    """The same fraction for a 23-bit uniform (j 2^-23, j < 2^23): the
+    granularity the ZIP-SR draw had before it took the whole word."""
     k_lo = oracle.zipsr_decide(x, dv, R, eps, 0.0)
     k_hi = oracle.zipsr_decide(x, dv, R, eps, 1.0 - U_STEP)
     if k_lo == k_hi:
@@ -104,9 +123,9 @@ for s in [6e-11, 1e-8, 3e-7, 1e-4, 2.5e-2]:
 
 @pytest.mark.parametrize("s,xv,rs_bc2", CASES)
 def test_exact_expectation_of_h(s, xv, rs_bc2):
-    """Enumerating every uniform: the oracle's canonical binary32 probability
-    equals the pages' formula in binary64 within 1e-6 plus the binary32
-    conditioning of the cell, and the expected preconditioner
+    """Enumerating every draw word: the oracle's canonical binary32
+    probability equals the pages' formula in binary64 within 1e-6 plus the
+    binary32 conditioning of the cell, and the expected preconditioner
     equals h(v) (the preconditioner-space unbiasedness ZIP-SR is built on)."""
     eps = f32(1e-8)
     s = f32(s)
@@ -130,10 +149,12 @@ def test_exact_expectation_of_h(s, xv, rs_bc2):
     # binary32 conditioning: da and db are each rounded once (half an ulp of
     # d); p moves by that over (db - da).  Plus the draw granularity.
     cond = 4 * 2.0 ** -24 * db / (db - da)
-    assert abs(p - p_ref) < 1e-6 + U_STEP + cond
+    # the draw: 2^-32 granularity near zero, 2^-23 relative above 2^-8
+    grain = W_STEP + 2.0 ** -22 * p_ref
+    assert abs(p - p_ref) < 1e-6 * p_ref + grain + cond
     # E[h(Q)] = h(v): with d-values of the code points, in binary64
     e_h = p * (1 / da) + (1 - p) * (1 / db)
-    assert abs(e_h - 1 / dv) <= (1e-6 + U_STEP + cond) * abs(1 / da - 1 / db) + 1e-12 / dv
+    assert abs(e_h - 1 / dv) <= (1e-6 * p_ref + grain + cond) * abs(1 / da - 1 / db) + 1e-12 / dv
 
 
 def test_zero_and_top_are_deterministic():
@@ -251,14 +272,18 @@ def test_u32_decision_exact_expectation(s, xv, rs_bc2):
         assert p == pytest.approx(np.ceil(rhs / B * 2.0 ** 32) * W_STEP, abs=2 * W_STEP)
 
 
-def test_u32_decision_removes_the_23_bit_bias():
-    """A value in the cell next to zero where the pages' probability is below
-    2^-23 (v = 1e-2, b = 2e-2, eps = 1e-8, no bias correction): the 23-bit
-    decision keeps zero with probability 2^-23, four times too often, and
-    E[h] is nearly twice h(v); the 32-bit decision is within 2^-32."""
+@pytest.mark.parametrize("v_hat", [1e-2, 3e-3, 1e-3])
+def test_zero_cell_has_no_23_bit_bias(v_hat):
+    """Values in the cell next to zero where the pages' probability of zero
+    is below 2^-23 (b = 2 v, eps = 1e-8, no bias correction).  A 23-bit
+    uniform keeps zero with probability 2^-23 at least, several times too
+    often, and pushes E[h] far above h(v) (h(0) = 1/eps is huge); ZIP-SR's
+    draw from the whole word and the binary64 option (v code 5) both realise
+    the probability to within 2^-32 plus 2^-22 relative, so
+    |E[h] - h(v)| <= 2^-32 (h(0) - h(b)) + the cell's binary32 conditioning."""
     eps = f32(1e-8)
-    s = f32(15 * 2e-2)                              # b = s/15 = 2e-2
-    v = f32(1e-2)
+    s = f32(15 * 2 * v_hat)                         # b = s/15 = 2 v
+    v = f32(v_hat)
     x = f32(np.float32(v) * (np.float32(1.0) / np.float32(s)))
     R = f32(np.sqrt(np.float32(s)))
     dv = f32(np.float32(np.sqrt(np.float32(v))) + np.float32(eps))
@@ -267,13 +292,69 @@ def test_u32_decision_removes_the_23_bit_bias():
     da, db = float(vzs[0]) * R + eps, float(vzs[1]) * R + eps
     p_ref = (1 / dv - 1 / db) / (1 / da - 1 / db)
     assert p_ref < 2.0 ** -23
-    p23, _ = p_low_exact(x, dv, R, eps)
-    p32, _ = p_low_exact_u32(x, dv, R, eps)
+    p23, _ = p_low_exact_u23(x, dv, R, eps)
+    p0, _ = p_low_exact(x, dv, R, eps)              # ZIP-SR (v code 0)
+    p5, _ = p_low_exact_u32(x, dv, R, eps)          # binary64 option (v code 5)
     assert p23 == U_STEP                            # rounded up to one granule
-    assert abs(p32 - p_ref) < 2 * W_STEP + 1e-6 * p_ref
+    cond = 4 * 2.0 ** -24 * db / (db - da) * p_ref
+    for p in (p0, p5):
+        assert abs(p - p_ref) < 2 * W_STEP + 2.0 ** -22 * p_ref + cond
     e_h = lambda p: p / da + (1 - p) / db          # noqa: E731
-    assert e_h(p23) > 1.8 / dv
-    assert abs(e_h(p32) - 1 / dv) < 1e-3 / dv
+    assert e_h(p23) - 1 / dv > 0.5 * (U_STEP - p_ref) * (1 / da - 1 / db)
+    for p in (p0, p5):
+        assert abs(e_h(p) - 1 / dv) <= (2 * W_STEP + 2.0 ** -22 * p_ref + cond) * (1 / da - 1 / db)
+    assert abs(e_h(p0) - 1 / dv) < 1e-3 / dv
+
+
+def test_block_decisions_follow_the_page_probability_on_the_word():
+    """The block step's ZIP-SR codes, element by element: with the draw word
+    w of each element (Philox, pinned by its known answers) and the pages'
+    keep probability p computed in binary64 from the block's binary32
+    quantities, an element whose w 2^-32 lies clearly below p keeps the lower
+    code point and one clearly above takes the upper; near-ties (within the
+    binary32 conditioning) are skipped.  A decision taken on other bits of
+    the word, or on a mis-scaled uniform, fails this."""
+    from workloads import bf16_bits, bf16_to_f32
+    _, _, vz, vzs = oracle.tables()
+    b1, b2, eps = np.float32(0.9), np.float32(0.999), np.float32(1e-8)
+    rng = np.random.default_rng(7)
+    decisive = 0
+    for rep in range(40):
+        g = (rng.standard_normal(128) * 1e-3 * np.exp(rng.uniform(-3, 0, 128))).astype(np.float32)
+        gb = bf16_bits(g)
+        gf = bf16_to_f32(gb)
+        seed, tid = 1000 + rep, 3
+        sc = oracle.make_scalars(1e-3, b1, b2, eps, t=1, seed=seed)
+        w = np.zeros(128, np.float32)
+        mc, vc = np.zeros(64, np.uint8), np.zeros(64, np.uint8)
+        ms, vs = np.zeros(1, np.float32), np.zeros(1, np.float32)
+        oracle.lib().oracle_block4(sc, np.float32(1.0), 0, 0, tid, 0, 128, w, gb, mc, ms, vc, vs)
+        codes = np.empty(128, np.int64)
+        codes[0::2] = vc & 15
+        codes[1::2] = vc >> 4
+        # the canonical binary32 quantities of the block (zero prior state)
+        omb2 = np.float32(1.0) - b2
+        v1 = (omb2 * (gf * gf)).astype(np.float32)
+        av = np.float32(v1.max())
+        inv = np.float32(1.0) / av
+        rs = np.float32(sc.rs_bc2)
+        R = np.float32(np.sqrt(av) * rs)
+        for i in range(128):
+            x = np.float32(v1[i] * inv)
+            dv = np.float32(np.float32(np.sqrt(v1[i]) * rs) + eps)
+            k = oracle.zipsr_bracket(float(x))
+            da = float(np.float32(np.float32(vzs[k]) * R + eps))   # fma: exact enough here
+            db = float(np.float32(np.float32(vzs[k + 1]) * R + eps))
+            if db == da:
+                continue
+            p = min(max((1 / float(dv) - 1 / db) / (1 / da - 1 / db), 0.0), 1.0)
+            u = oracle.draw_word(seed, 1, tid, 0, i) * 2.0 ** -32
+            tol = 1e-5 * db / (db - da) + 2.0 ** -22
+            if abs(u - p) <= tol:
+                continue
+            decisive += 1
+            assert codes[i] == (k if u < p else k + 1), (rep, i, u, p, k, codes[i])
+    assert decisive > 3000
 
 
 def test_u32_decision_ends_are_deterministic():
