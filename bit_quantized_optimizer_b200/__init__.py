@@ -19,8 +19,9 @@ __all__ = ["ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_V_ZI_RTN", "ADAMW4_V_ZI_
            "adamw4_get_step", "adamw4_set_step", "adamw4_state_bytes", "adamw4_state_export",
            "adamw4_state_import", "adamw4_launch_info", "adamw4_last_error", "adamw4_sync",
            "adamw4_inject_fault", "ADAMW4_ETIMEOUT", "ADAMW4_FAULT_STALL_PIPELINE", "AdamW4",
-           "adamw4_state_buffers", "adamw4_step_noalloc", "ADAMW4_NOALLOC_MAX_TENSORS",
-           "is_fp32_state", "LIB_PATH"]
+           "adamw4_state_buffers", "adamw4_step_noalloc", "adamw4_noalloc_sync",
+           "ADAMW4_NOALLOC_MAX_TENSORS", "ADAMW4_ENONFINITE", "ADAMW4_ERANGE", "ADAMW4_ECHECK",
+           "is_fp32_state", "adamw4_tensor_state_kind", "LIB_PATH"]
 
 # ADAMW4_LIBRARY selects another build of the same library (the checked one)
 LIB_PATH = os.environ.get("ADAMW4_LIBRARY") or os.path.join(
@@ -41,14 +42,16 @@ ADAMW4_T_BF16_PARAM = 16   # bf16 weights (rounded to nearest even after each up
 MIN_QUANT_NUMEL = 4096
 BLOCK = 128
 
+ADAMW4_ENONFINITE = -6
 ADAMW4_ETIMEOUT = -7
+ADAMW4_ECHECK = -8
+ADAMW4_ERANGE = -9
 ADAMW4_NOALLOC_MAX_TENSORS = 1024
 ADAMW4_FAULT_STALL_PIPELINE = 1
 
-ADAMW4_ECHECK = -8
 STATUS = {0: "ADAMW4_OK", -1: "ADAMW4_EINVAL", -2: "ADAMW4_EALIGN", -3: "ADAMW4_ENOMEM",
-          -4: "ADAMW4_ECUDA", -5: "ADAMW4_ESTATE", -6: "ADAMW4_ERANGE", -7: "ADAMW4_ETIMEOUT",
-          -8: "ADAMW4_ECHECK"}
+          -4: "ADAMW4_ECUDA", -5: "ADAMW4_ESTATE", -6: "ADAMW4_ENONFINITE",
+          -7: "ADAMW4_ETIMEOUT", -8: "ADAMW4_ECHECK", -9: "ADAMW4_ERANGE"}
 
 
 class AdamW4Error(RuntimeError):
@@ -108,12 +111,15 @@ def lib() -> ctypes.CDLL:
         L.adamw4_step_noalloc.argtypes = [c.POINTER(adamw4_config), c.POINTER(adamw4_tensor),
                                           c.c_int, c.POINTER(adamw4_state_buffers), c.c_int64,
                                           c.c_float, c.c_int, c.c_void_p]
+        L.adamw4_noalloc_sync.argtypes = [c.c_int, c.c_void_p]
+        L.adamw4_tensor_state_kind.argtypes = [c.POINTER(adamw4_tensor)]
+        L.adamw4_tensor_state_kind.restype = c.c_int
         L.adamw4_last_error.argtypes = [H]
         L.adamw4_last_error.restype = c.c_char_p
         for f in ("adamw4_create", "adamw4_step", "adamw4_step_host", "adamw4_destroy",
                   "adamw4_get_step", "adamw4_set_step", "adamw4_state_export",
                   "adamw4_state_import", "adamw4_launch_info", "adamw4_sync",
-                  "adamw4_inject_fault", "adamw4_step_noalloc"):
+                  "adamw4_inject_fault", "adamw4_step_noalloc", "adamw4_noalloc_sync"):
             getattr(L, f).restype = c.c_int
         _lib = L
     return _lib
@@ -184,6 +190,8 @@ def adamw4_sync(h, stream=None):
 
 
 def adamw4_inject_fault(h, fault: int):
+    """Arms a test fault for the next step of handle h (h None: for the next
+    adamw4_step_noalloc call)."""
     _check(lib().adamw4_inject_fault(h, fault), h)
 
 
@@ -198,18 +206,35 @@ def adamw4_step_noalloc(cfg: adamw4_config, tensors, state: adamw4_state_buffers
         raise AdamW4Error(rc, "adamw4_step_noalloc failed")
 
 
+def adamw4_noalloc_sync(device: int = 0, stream=None):
+    """Waits for the stream and reads and clears the allocation-free step's
+    status word on the device; raises AdamW4Error(ADAMW4_ETIMEOUT /
+    ADAMW4_ENONFINITE) when a call reported a failure."""
+    rc = lib().adamw4_noalloc_sync(device, stream)
+    if rc != ADAMW4_OK:
+        raise AdamW4Error(rc, "adamw4_noalloc_sync: status word set")
+
+
 def adamw4_launch_info(h):
     g, b, u = ctypes.c_int(), ctypes.c_int(), ctypes.c_int64()
     _check(lib().adamw4_launch_info(h, ctypes.byref(g), ctypes.byref(b), ctypes.byref(u)), h)
     return g.value, b.value, u.value
 
 
+def adamw4_tensor_state_kind(numel: int, flags: int, elem_offset: int = 0) -> int:
+    """The library's state class of a descriptor: 1 fp32 state, 0 4-bit."""
+    t = adamw4_tensor(1, 1, numel, 0, flags, 0.0, elem_offset)
+    k = lib().adamw4_tensor_state_kind(ctypes.byref(t))
+    if k < 0:
+        raise AdamW4Error(k, "invalid descriptor (numel, flags or elem_offset)")
+    return k
+
+
 def is_fp32_state(numel: int, flags: int) -> bool:
-    """The library's classification rule: fp32 state for NORM / FP32_STATE
-    tensors, and below 4096 elements unless flagged QUANT_STATE."""
-    if flags & (ADAMW4_T_NORM | ADAMW4_T_FP32_STATE):
-        return True
-    return numel < MIN_QUANT_NUMEL and not flags & ADAMW4_T_QUANT_STATE
+    """Whether the library keeps fp32 state for such a tensor (asked of the
+    library: fp32 for NORM / FP32_STATE tensors, and below 4096 elements
+    unless flagged QUANT_STATE)."""
+    return adamw4_tensor_state_kind(numel, flags) == 1
 
 
 class AdamW4:
@@ -257,7 +282,8 @@ class AdamW4:
 
     def sync(self, stream=None):
         """Waits for the stream; raises AdamW4Error(ADAMW4_ETIMEOUT) if a step
-        kernel on it stopped on a pipeline wait."""
+        kernel on it stopped on a pipeline wait, AdamW4Error(ADAMW4_ENONFINITE)
+        if a step produced a non-finite weight."""
         import torch
         s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
         adamw4_sync(self.handle, s)

@@ -8,6 +8,7 @@
 #include <nvtx3/nvToolsExt.h>   // header-only; ranges show up under a profiler
 
 #include <algorithm>
+#include <atomic>
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
@@ -58,7 +59,6 @@ struct adamw4_handle {
   cudaStream_t s_out = nullptr;   // adamw4_step_host: device-to-host copies
   std::vector<cudaEvent_t> events;
   int fault_stall = 0;            // test hook for the next step
-  CodeTables tabs{};
   std::string err;
 };
 
@@ -140,6 +140,48 @@ void build_tables(CodeTables* T) {
   }
 }
 
+// The shared-memory tables of one code family (zero_excluded: the ZE codes
+// (k+1)/16, else the zero-inclusive k/15), as each CTA of the step kernel
+// holds them.
+void fill_smem_tables(const CodeTables& T, bool zero_excluded, SmemTables* S) {
+  for (int t = 0; t < 256; ++t) {
+    S->mpair[t] = make_float2(T.nf4[t & 15], T.nf4[t >> 4]);
+    const float lo = zero_excluded ? (float)((t & 15) + 1) * 0.0625f : T.vz[t & 15];
+    const float hi = zero_excluded ? (float)((t >> 4) + 1) * 0.0625f : T.vz[t >> 4];
+    S->vpair[t] = make_float2(lo, hi);
+  }
+  for (int t = 0; t < 128; ++t) S->rtn[t] = T.rtn[t];
+  for (int t = 0; t < 16; ++t) {
+    S->nf4[t] = T.nf4[t];
+    S->gap[t] = T.nf4_gap[t];
+    S->vz[t] = T.vz[t];
+    S->zip[t] = make_float4(t == 15 ? INFINITY : T.vz[t], T.vz_sqrt[std::max(t - 1, 0)],
+                            T.vz_sqrt[t], T.vz_sqrt[std::min(t + 1, 15)]);
+    S->vzp[t] = make_float2(T.vz[t], T.vz[std::min(t + 1, 15)]);
+    S->vzmid[t] = T.vz_mid[t];
+  }
+}
+
+// Writes the code tables into the device's g_code_tables once per device
+// (cudaMemcpyToSymbol; no allocation).  The caller has the device current.
+std::mutex g_tables_mu;
+bool g_tables_ready[64];
+
+cudaError_t upload_tables(int device) {
+  if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_tables_mu);
+  if (g_tables_ready[device]) return cudaSuccess;
+  CodeTables T;
+  build_tables(&T);
+  static SmemTables host[2];
+  fill_smem_tables(T, false, &host[0]);
+  fill_smem_tables(T, true, &host[1]);
+  const cudaError_t e = cudaMemcpyToSymbol(g_code_tables, host, sizeof host, 0,
+                                           cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) g_tables_ready[device] = true;
+  return e;
+}
+
 bool tables_ok(const CodeTables& T) {
   int seen[65] = {0};
   for (int j = 0; j < 15; ++j) {
@@ -166,6 +208,21 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.omb2 = (float)(1.0 - (double)c.beta2);
   a.eps = c.eps;
   a.lr = lr;
+  a.nb2 = -a.b2;
+  a.nomb2 = -a.omb2;
+  a.neps = -a.eps;
+  a.nstep = -a.step_size;
+  // Ranges of the kernel's fast square root and division (exact_math.cuh):
+  // v1 in [2^-100, 2^64] keeps sqrt(v1) rs_bc2 + eps within [eps, 2^53) when
+  // rs_bc2 <= 2^20; |m1| >= 2^-60 keeps the quotient at or above 2^-113 and
+  // its remainder exact; |m1| <= 2^100 eps keeps it at or below 2^100.  With
+  // eps outside [2^-60, 2^10] or rs_bc2 above 2^20 every lane takes the IEEE
+  // operations instead (m_hi < 0).
+  a.m_lo = 0x1p-60f;
+  a.v_lo = 0x1p-100f;
+  a.v_hi = 0x1p64f;
+  const bool fast_ok = a.eps >= 0x1p-60f && a.eps <= 0x1p10f && a.rs_bc2 <= 0x1p20f;
+  a.m_hi = fast_ok ? std::min(std::ldexp(a.eps, 100), 0x1p100f) : -1.0f;
   // Philox round keys: round r uses the seed words plus r times the Weyl
   // constants (mod 2^32).
   for (int r = 0; r < 10; ++r) {
@@ -317,27 +374,27 @@ int grid_for(int vcode, bool bf16w, int device, int* grid) {
 
 template <bool BF16W>
 void launch_w(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t u0, int64_t u1,
-              const StepArgs& a, const CodeTables& tabs, const StateArena& st) {
+              const StepArgs& a, const StateArena& st) {
   const int n = kCtaThreads;
   const int smem = kSmemStages;
   switch (vcode) {
     case kVZip:
-      adamw4_step_kernel<kVZip, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
+      adamw4_step_kernel<kVZip, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, st);
       break;
     case kVZe:
-      adamw4_step_kernel<kVZe, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
+      adamw4_step_kernel<kVZe, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, st);
       break;
     case kVZiRtn:
-      adamw4_step_kernel<kVZiRtn, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
+      adamw4_step_kernel<kVZiRtn, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, st);
       break;
     case kVZiSr:
-      adamw4_step_kernel<kVZiSr, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
+      adamw4_step_kernel<kVZiSr, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, st);
       break;
     case kVZeFloor:
-      adamw4_step_kernel<kVZeFloor, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
+      adamw4_step_kernel<kVZeFloor, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, st);
       break;
     default:
-      adamw4_step_kernel<kVZip32, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, tabs, st);
+      adamw4_step_kernel<kVZip32, BF16W><<<grid, n, smem, s>>>(T, u0, u1, a, st);
       break;
   }
 }
@@ -346,10 +403,9 @@ void launch_w(int vcode, int grid, cudaStream_t s, const DevTensor* T, int64_t u
 // table; bf16w selects the instantiation that reads and writes bf16 weights
 // where a tensor asks for it.
 void launch_vcode(int vcode, bool bf16w, int grid, cudaStream_t s, const DevTensor* T,
-                  int64_t u0, int64_t u1, const StepArgs& a, const CodeTables& tabs,
-                  const StateArena& st) {
-  if (bf16w) launch_w<true>(vcode, grid, s, T, u0, u1, a, tabs, st);
-  else launch_w<false>(vcode, grid, s, T, u0, u1, a, tabs, st);
+                  int64_t u0, int64_t u1, const StepArgs& a, const StateArena& st) {
+  if (bf16w) launch_w<true>(vcode, grid, s, T, u0, u1, a, st);
+  else launch_w<false>(vcode, grid, s, T, u0, u1, a, st);
 }
 
 // One launch over units [u0, u1) of the handle's list.
@@ -360,7 +416,7 @@ int launch(adamw4_handle* h, StepArgs a, cudaStream_t s, int64_t u0, int64_t u1)
   a.status = h->d_status;
   a.fault_stall = h->fault_stall;
   h->fault_stall = 0;
-  launch_vcode(h->cfg.vcode, h->bf16w, grid, s, h->d_tensors, u0, u1, a, h->tabs, h->st);
+  launch_vcode(h->cfg.vcode, h->bf16w, grid, s, h->d_tensors, u0, u1, a, h->st);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(h, e, "step kernel launch");
   return ADAMW4_OK;
@@ -408,10 +464,13 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
   if (h == nullptr) return fail(nullptr, ADAMW4_ENOMEM, "host allocation failed");
   h->device = device;
   h->cfg = *cfg;
-  build_tables(&h->tabs);
-  if (!tables_ok(h->tabs)) {
-    delete h;
-    return fail(nullptr, ADAMW4_EINVAL, "NF4 bucket table has two midpoints in one bucket");
+  {
+    CodeTables tabs;
+    build_tables(&tabs);
+    if (!tables_ok(tabs)) {
+      delete h;
+      return fail(nullptr, ADAMW4_EINVAL, "NF4 bucket table has two midpoints in one bucket");
+    }
   }
 
   // Classify and lay out the state.
@@ -483,6 +542,7 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
   h->st.fv = reinterpret_cast<float*>(base + o_fv);
   h->st.nblocks4 = h->nblocks4;
   h->st.n32 = h->nfp32;
+  h->st.vs_minus_ms = h->st.vscale - h->st.mscale;
   h->d_status = reinterpret_cast<uint32_t*>(base + o_st);
   if ((e = cudaMemset(h->d_arena, 0, h->arena_bytes)) != cudaSuccess ||
       (e = cudaMemcpy(h->d_tensors, dev.data(), sizeof(DevTensor) * dev.size(),
@@ -490,6 +550,11 @@ extern "C" int adamw4_create(const adamw4_config* cfg, const adamw4_tensor* tens
     release(h);
     delete h;
     return cuda_fail(nullptr, e, "initialising the state");
+  }
+  if ((e = upload_tables(device)) != cudaSuccess) {
+    release(h);
+    delete h;
+    return cuda_fail(nullptr, e, "writing the code tables");
   }
   int ge = grid_for(cfg->vcode, h->bf16w, device, &h->grid);
   if (ge != 0) {
@@ -780,6 +845,25 @@ extern "C" int adamw4_state_import(adamw4_handle* h, const void* host_buf, int64
   return ADAMW4_OK;
 }
 
+namespace {
+
+// The status code (and message) of a non-zero device status word: a wait
+// that ran out first, since it leaves the step incomplete.
+int status_error(adamw4_handle* h, uint32_t status) {
+  if (status & 1u)
+    return fail(h, ADAMW4_ETIMEOUT,
+                "a stage wait in the step kernel ran out of time; the step is incomplete");
+  if (status & 2u)
+    return fail(h, ADAMW4_ECHECK,
+                "checked build: a unit's values or state lay outside its tensor or the arena; "
+                "that unit was skipped");
+  return fail(h, ADAMW4_ENONFINITE,
+              "a step produced a non-finite weight (a NaN or infinite grad or weight, or an "
+              "overflow); the step ran to the end");
+}
+
+}  // namespace
+
 extern "C" int adamw4_sync(adamw4_handle* h, void* cuda_stream) {
   if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
   DeviceGuard dg(h->device);
@@ -793,22 +877,30 @@ extern "C" int adamw4_sync(adamw4_handle* h, void* cuda_stream) {
   if (status != 0) {
     e = cudaMemset(h->d_status, 0, sizeof status);
     if (e != cudaSuccess) return cuda_fail(h, e, "clearing the status word");
-    if (status & 2u)
-      return fail(h, ADAMW4_ECHECK,
-                  "checked build: a unit's values or state lay outside its tensor or the arena; "
-                  "that unit was skipped");
-    return fail(h, ADAMW4_ETIMEOUT,
-                "a stage wait in the step kernel ran out of time; the step is incomplete");
+    return status_error(h, status);
   }
   return ADAMW4_OK;
 }
 
+namespace {
+std::atomic<int> g_noalloc_fault_stall{0};   // test hook for the next noalloc call
+}  // namespace
+
 extern "C" int adamw4_inject_fault(adamw4_handle* h, int fault) {
-  if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
   if (fault != 0 && fault != ADAMW4_FAULT_STALL_PIPELINE)
-    return fail(h, ADAMW4_EINVAL, "unknown fault");
+    return fail(live(h) ? h : nullptr, ADAMW4_EINVAL, "unknown fault");
+  if (h == nullptr) {   // the next adamw4_step_noalloc call
+    g_noalloc_fault_stall.store(fault == ADAMW4_FAULT_STALL_PIPELINE ? 1 : 0);
+    return ADAMW4_OK;
+  }
+  if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
   h->fault_stall = (fault == ADAMW4_FAULT_STALL_PIPELINE);
   return ADAMW4_OK;
+}
+
+extern "C" int adamw4_tensor_state_kind(const adamw4_tensor* t) {
+  if (t == nullptr || t->numel <= 0 || piece_error(*t) != nullptr) return ADAMW4_EINVAL;
+  return fp32_state(*t) ? 1 : 0;
 }
 
 extern "C" int adamw4_launch_info(const adamw4_handle* h, int* grid, int* block, int64_t* units) {
@@ -873,12 +965,14 @@ int na_validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n,
   if (!na_aligned(sb->mcodes, 16) || !na_aligned(sb->vcodes, 16) || !na_aligned(sb->mscale, 4) ||
       !na_aligned(sb->vscale, 4) || !na_aligned(sb->m32, 16) || !na_aligned(sb->v32, 16))
     return ADAMW4_EALIGN;
+  int64_t blocks4 = 0, elems32 = 0;   // what the list needs of each state buffer
   for (int i = 0; i < n; ++i) {
     const adamw4_tensor& x = ts[i];
     if (x.param == nullptr || x.grad_bf16 == nullptr || x.numel <= 0 ||
         x.numel > ((int64_t)1 << 40) || !std::isfinite(x.weight_decay) || piece_error(x) != nullptr)
       return ADAMW4_EINVAL;
     if (!na_aligned(x.param, 16) || !na_aligned(x.grad_bf16, 16)) return ADAMW4_EALIGN;
+    if (fp32_state(x)) elems32 += x.numel; else blocks4 += (x.numel + kBlock - 1) / kBlock;
     const uintptr_t p0 = reinterpret_cast<uintptr_t>(x.param),
                     p1 = p0 + (uintptr_t)x.numel * param_bytes(x);
     const uintptr_t g0 = reinterpret_cast<uintptr_t>(x.grad_bf16), g1 = g0 + (uintptr_t)x.numel * 2u;
@@ -893,6 +987,11 @@ int na_validate(const adamw4_config* cfg, const adamw4_tensor* ts, int n,
         return ADAMW4_EINVAL;                                     // a param overlaps
     }
   }
+  // the state buffers the list uses must be given (a NULL one would be read)
+  if (blocks4 > 0 && (sb->mcodes == nullptr || sb->vcodes == nullptr || sb->mscale == nullptr ||
+                      sb->vscale == nullptr))
+    return ADAMW4_EINVAL;
+  if (elems32 > 0 && (sb->m32 == nullptr || sb->v32 == nullptr)) return ADAMW4_EINVAL;
   return ADAMW4_OK;
 }
 
@@ -918,6 +1017,7 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
     for (int vc = ADAMW4_V_ZIPSR; vc <= ADAMW4_V_ZIPSR_U32; ++vc)
       for (int bw = 0; bw < 2; ++bw)
         if (grid_for(vc, bw != 0, device, &nd.grid[vc][bw]) != 0) return ADAMW4_ECUDA;
+    if (upload_tables(device) != cudaSuccess) return ADAMW4_ECUDA;
     nd.ready = true;
   }
   // The table adamw4_create would build, in the same order and layout.
@@ -936,18 +1036,16 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   uint32_t* status = reinterpret_cast<uint32_t*>(nd.scratch);
   DevTensor* table = reinterpret_cast<DevTensor*>(nd.scratch + kNoAllocStatusBytes);
-  // The array keeps the previous call's contents: clear the status word and
-  // overwrite the table.  The copy is from pageable memory, so the staging
-  // buffer is free again when the call returns.
-  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return ADAMW4_ECUDA;
+  // The array keeps the previous call's contents: overwrite the table (the
+  // status word accumulates until adamw4_noalloc_sync reads and clears it).
+  // The copy is from pageable memory, so the staging buffer is free again when
+  // the call returns.
   if (cudaMemcpyAsync(table, g_noalloc_table, sizeof(DevTensor) * (size_t)n,
                       cudaMemcpyHostToDevice, s) != cudaSuccess)
     return ADAMW4_ECUDA;
-  CodeTables tabs;
-  build_tables(&tabs);
   StepArgs a = make_args(*cfg, lr, t);
   a.status = status;
-  a.fault_stall = 0;
+  a.fault_stall = g_noalloc_fault_stall.exchange(0);
   StateArena st;
   st.mcodes = state->mcodes;
   st.vcodes = state->vcodes;
@@ -957,8 +1055,31 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   st.fv = state->v32;
   st.nblocks4 = blocks4;
   st.n32 = elems32;
+  st.vs_minus_ms = st.vscale - st.mscale;
   const int64_t need = (unit + kHalves - 1) / kHalves;
   launch_vcode(cfg->vcode, bf16w, (int)std::min<int64_t>(nd.grid[cfg->vcode][bf16w], need), s,
-               table, 0, unit, a, tabs, st);
+               table, 0, unit, a, st);
   return cudaGetLastError() == cudaSuccess ? ADAMW4_OK : ADAMW4_ECUDA;
+}
+
+extern "C" int adamw4_noalloc_sync(int device, void* cuda_stream) {
+  if (device < 0 || device >= kNoAllocMaxDevices) return ADAMW4_EINVAL;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_dev[device].ready) return ADAMW4_EINVAL;
+  DeviceGuard dg(device);
+  if (!dg.ok) return ADAMW4_ECUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return ADAMW4_ECUDA;
+  uint32_t status = 0;
+  if (cudaMemcpyFromSymbol(&status, g_noalloc_scratch, sizeof status, 0,
+                           cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ADAMW4_ECUDA;
+  if (status == 0) return ADAMW4_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_noalloc_scratch, &zero, sizeof zero, 0, cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return ADAMW4_ECUDA;
+  if (status & 1u) return ADAMW4_ETIMEOUT;
+  if (status & 2u) return ADAMW4_ECHECK;
+  return ADAMW4_ENONFINITE;
 }

@@ -49,6 +49,7 @@
 #include <cstdint>
 
 #include "../../include/adamw4.h"
+#include "exact_math.cuh"
 
 namespace {
 
@@ -117,14 +118,23 @@ struct StepArgs {
   float step_size;   // lr / (1 - b1^t)
   float rs_bc2;      // 1 / sqrt(1 - b2^t)
   float b1, omb1, b2, omb2, eps, lr;
+  float nb2, nomb2, neps, nstep;  // -b2, -(1 - b2), -eps, -step_size
+  // Operand ranges of the fast division and square root (exact_math.cuh):
+  // a lane takes them when all its |m1| lie in [m_lo, m_hi] and all its v1
+  // in [v_lo, v_hi]; otherwise it uses the IEEE operations.  m_hi < 0
+  // switches the fast path off (eps or rs_bc2 outside the range it needs).
+  float m_lo, m_hi, v_lo, v_hi;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
   int lm_sr_active;      // final-10% LM-head phase
-  uint32_t* status;      // device status word (bit 0: a pipeline wait timed out)
+  uint32_t* status;      // device status word (bit 0: a pipeline wait timed out;
+                         // bit 1: checked build, unit out of range; bit 2: a
+                         // non-finite updated weight)
   int fault_stall;       // test hook: mark stages filled without filling them
 };
 
-// Code tables, passed by value and staged in shared memory by each CTA.
+// The code tables' source values, formed on the host (the shared-memory
+// tables SmemTables below are built from them).
 struct CodeTables {
   float nf4[16];        // NF4 levels, ascending
   float nf4_gap[16];    // nf4[j+1] - nf4[j]
@@ -143,20 +153,24 @@ struct StateArena {
   float* fv;
   int64_t nblocks4;  // blocks in the code and scale arrays (checked builds test against it)
   int64_t n32;       // elements in fm and fv (likewise)
+  int64_t vs_minus_ms;  // vscale - mscale, in floats
 };
 
 // What the producer tells the consumer about one unit (64 bytes).
+// The addresses are formed by the producer (one lane per unit) so that the
+// consumers' sixteen lanes do not each recompute them.
 struct __align__(16) UnitHeader {
-  float* w;              // the unit's first weight
-  const uint16_t* g;     // its first gradient
-  uint64_t e0;           // index of that element within its (logical) tensor
-  uint64_t state;        // 4-bit: block index in the code arena; fp32: element index
+  float* w;              // the unit's first weight (fp32, or bf16 bit patterns)
+  uint32_t* mc;          // 4-bit: the block's m code words; fp32 state: its first m
+  uint32_t* vc;          // 4-bit: the block's v code words; fp32 state: its first v
+  float* ms;             // 4-bit: the block's m scale (its v scale: ms + vs_minus_ms)
+  uint64_t e0;           // index of the unit's first element within its (logical) tensor
   uint32_t tensor_id;
   uint32_t flags;        // ADAMW4_T_* | kKindFp32 | kStaged
   float decay;           // 1 - lr * weight_decay of the tensor
-  int32_t nvalid;        // values in the unit (1..128)
-  uint32_t w_soff;       // bf16-weight units: stage offset of the unit's weights
-  uint32_t pad_[3];
+  uint32_t nv_soff;      // values in the unit (bits 0-7: 1..128) | bf16-weight units:
+                         // stage offset of the unit's weights << 8
+  const uint16_t* g;     // its first gradient (read from global memory by direct units)
 };
 static_assert(sizeof(UnitHeader) == 64, "UnitHeader layout");
 
@@ -319,6 +333,35 @@ __device__ __forceinline__ uint16_t bf16_rn(float x) {
 }
 __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
+// Three-input maximum and minimum (one instruction each on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// Largest and smallest |x| over a lane's eight values (four pairs).
+__device__ __forceinline__ float absmax8(const float2 (&x)[4]) {
+  const float r = max3f(fabsf(x[0].x), fabsf(x[0].y), fabsf(x[1].x));
+  const float q = max3f(r, fabsf(x[1].y), fabsf(x[2].x));
+  return max3f(q, fabsf(x[2].y), fmaxf(fabsf(x[3].x), fabsf(x[3].y)));
+}
+__device__ __forceinline__ float absmin8(const float2 (&x)[4]) {
+  const float r = min3f(fabsf(x[0].x), fabsf(x[0].y), fabsf(x[1].x));
+  const float q = min3f(r, fabsf(x[1].y), fabsf(x[2].x));
+  return min3f(q, fabsf(x[2].y), fminf(fabsf(x[3].x), fabsf(x[3].y)));
+}
+
+// The ZIP-SR uniforms of two draw words: each word rounded to the nearest
+// binary32 (ties to even) and scaled by 2^-32, exactly.
+__device__ __forceinline__ float2 uniform32x2(uint32_t w0, uint32_t w1) {
+  return __fmul2_rn(make_float2(__uint2float_rn(w0), __uint2float_rn(w1)), f2(0x1p-32f));
+}
+
 // Max of non-negative binary32 values over a half-warp: their bit patterns
 // order like the values, so an integer reduction gives the exact maximum.
 __device__ __forceinline__ float hmax16_nonneg(float v, unsigned mask) {
@@ -366,27 +409,35 @@ struct SmemTables {
   float2 vzp[16];      // {k/15, (k+1)/15}
   float vzmid[16];     // thresholds between adjacent k/15 code points
 };
+static_assert(sizeof(SmemTables) % 16 == 0, "tables are copied in 16-byte pieces");
+
+// The shared tables of both code families (0: zero-inclusive v codes, 1:
+// zero-excluded), written once per device by the host (cudaMemcpyToSymbol)
+// before the first launch; each CTA copies its family's into shared memory.
+static __device__ __align__(16) SmemTables g_code_tables[2];
 
 // ---------------------------------------------------------------------------
 // Requantisation of one 4-bit block held by a half-warp (8 values per lane).
 // FULL: all 128 values valid.  Otherwise `myn` values of this lane are valid.
 // ---------------------------------------------------------------------------
 
-// ZIP-SR codes of 8 values.  FLAT: also test for d(a) == d(b), which needs the
-// state-space fallback; callers skip it when the block's R makes that
-// impossible.
+// ZIP-SR codes of 8 values, from nv = -v1 and ndv = -d(v1) (d = 1/h, the
+// update's denominator) in pairs, and ninv = -1/s of the block.  FLAT: also
+// test for d(a) == d(b), which needs the state-space fallback; callers skip
+// it when the block's R makes that impossible.  U32: the binary64 decision of
+// v code 5; else the binary32 one with the whole-word uniform.
 template <bool FULL, bool FLAT, bool U32>
 __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
-                                                 const float (&v1)[kPerLane],
-                                                 const float (&den)[kPerLane],
-                                                 const uint32_t (&rw)[kPerLane], float inv,
+                                                 const float2 (&nv)[kPerLane / 2],
+                                                 const float2 (&ndv)[kPerLane / 2],
+                                                 const uint32_t (&rw)[kPerLane], float ninv,
                                                  float R, int myn) {
   // two values at a time; from the last pair to the first, so that element i
   // ends in bits 4i..4i+3
   uint32_t vco = 0;
 #pragma unroll
   for (int j = kPerLane / 2 - 1; j >= 0; --j) {
-    const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+    const float2 x2 = __fmul2_rn(nv[j], f2(ninv));                  // v1 / s
     const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
     // k0, the nearest integer to 15x, is the bracket or one above it (the top
     // entry's threshold is +inf: its bracket is always 14)
@@ -398,20 +449,19 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
     const float2 sb = make_float2(deca ? ea.z : ea.w, decb ? eb.z : eb.w);
     const float2 da = __ffma2_rn(sa, f2(R), f2(a.eps));
     const float2 db = __ffma2_rn(sb, f2(R), f2(a.eps));
-    const float2 dv = make_float2(den[2 * j], den[2 * j + 1]);
-    // fma(y, -1, x) rounds like x - y
-    const float2 B = __fmul2_rn(__ffma2_rn(da, f2(-1.0f), db), dv);      // (db - da) * dv
-    const float2 rhs = __fmul2_rn(__ffma2_rn(dv, f2(-1.0f), db), da);    // (db - dv) * da
+    // fma(y, -1, x) rounds like x - y; nB = -(db - da) dv, rhs = (db - dv) da
+    const float2 nB = __fmul2_rn(__ffma2_rn(da, f2(-1.0f), db), ndv[j]);
+    const float2 rhs = __fmul2_rn(__fadd2_rn(db, ndv[j]), da);
     bool lowa, lowb;
     if (U32) {
       // the whole word: (w 2^-32) * B rounded once in binary64, against rhs
-      lowa = __dmul_rn((double)rw[2 * j], (double)B.x * 0x1p-32) < (double)rhs.x;
-      lowb = __dmul_rn((double)rw[2 * j + 1], (double)B.y * 0x1p-32) < (double)rhs.y;
+      lowa = __dmul_rn((double)rw[2 * j], -(double)nB.x * 0x1p-32) < (double)rhs.x;
+      lowb = __dmul_rn((double)rw[2 * j + 1], -(double)nB.y * 0x1p-32) < (double)rhs.y;
     } else {
-      const float2 f = make_float2(one_plus_u(rw[2 * j]), one_plus_u(rw[2 * j + 1]));
-      const float2 lhs = __ffma2_rn(f, B, make_float2(-B.x, -B.y));       // u * B
-      lowa = lhs.x < rhs.x;
-      lowb = lhs.y < rhs.y;
+      // u * B < rhs, with -(u * B) = u * nB rounded once
+      const float2 nlhs = __fmul2_rn(uniform32x2(rw[2 * j], rw[2 * j + 1]), nB);
+      lowa = -nlhs.x < rhs.x;
+      lowb = -nlhs.y < rhs.y;
     }
     const uint32_t ka = k0a - (deca ? 1u : 0u), kb = k0b - (decb ? 1u : 0u);
     if (FLAT) {
@@ -419,14 +469,15 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
         const float2 z = S.vzp[ka];
         lowa = U32 ? __dmul_rn((double)rw[2 * j], (double)__fsub_rn(z.y, z.x) * 0x1p-32) <
                          (double)__fsub_rn(z.y, x2.x)
-                   : __fmul_rn(uniform23(rw[2 * j]), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.x);
+                   : __fmul_rn(__fmul_rn(__uint2float_rn(rw[2 * j]), 0x1p-32f),
+                               __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.x);
       }
       if (da.y == db.y) {
         const float2 z = S.vzp[kb];
         lowb = U32 ? __dmul_rn((double)rw[2 * j + 1], (double)__fsub_rn(z.y, z.x) * 0x1p-32) <
                          (double)__fsub_rn(z.y, x2.y)
-                   : __fmul_rn(uniform23(rw[2 * j + 1]), __fsub_rn(z.y, z.x)) <
-                         __fsub_rn(z.y, x2.y);
+                   : __fmul_rn(__fmul_rn(__uint2float_rn(rw[2 * j + 1]), 0x1p-32f),
+                               __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x2.y);
       }
     }
     const uint32_t ca = (FULL || 2 * j < myn) ? ka + (lowa ? 0u : 1u) : 0u;
@@ -436,41 +487,68 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
   return vco;
 }
 
+// The codes k of a pair of zero-excluded values from cm = (k + 1) as exact
+// binary32 integers in [1, 16]: cm + (kMagic - 1) is exact, and its bit
+// pattern is kMagic's (low byte 0) plus k.  The low byte of the result holds
+// k of the first value in bits 0-3 and of the second in bits 4-7.
+__device__ __forceinline__ uint32_t ze_code_pair(float2 cm) {
+  const float2 kb = __fadd2_rn(cm, f2(kMagic - 1.0f));
+  return __float_as_uint(kb.x) + 16u * __float_as_uint(kb.y);
+}
+
+// The low bytes of four code pairs as one 32-bit word of eight nibbles
+// (value i in bits 4i..4i+3), with the nibbles of values at or past `nvalid`
+// cleared.
+__device__ __forceinline__ uint32_t pack_code_pairs(const uint32_t (&P)[kPerLane / 2],
+                                                    int nvalid) {
+  const uint32_t w = __byte_perm(__byte_perm(P[0], P[1], 0x0040), __byte_perm(P[2], P[3], 0x0040),
+                                 0x5410);
+  return nvalid >= kPerLane ? w : w & ((1u << (4 * nvalid)) - 1u);
+}
+
+// Value i of a lane's eight, held as four pairs.
+__device__ __forceinline__ float el(const float2 (&x)[kPerLane / 2], int i) {
+  return (i & 1) ? x[i >> 1].y : x[i >> 1].x;
+}
+
+// RN(1/d) for a block scale d >= FLT_MIN: the fast sequence inside its range,
+// else the IEEE division (the branch is uniform over the half-warp).
+__device__ __forceinline__ float block_rcp(float d) {
+  if (d >= exact::kRcpLo && d <= exact::kRcpHi) return exact::rcp_rn(d);
+  return __fdiv_rn(1.0f, d);
+}
+
+// Requantises one block held by a half-warp: m1 and nv = -v1 in pairs, ndv =
+// -d(v1) (ZIP-SR), lam / lav = the lane's largest |m1| and v1 (over its valid
+// values).  Writes this lane's code words and, from lane 0, the two scales.
 template <int VCODE, bool FULL>
 __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTables& S,
                                               uint32_t tensor_id, uint32_t flags, uint64_t e0,
                                               int lane, int myn, unsigned hmask,
-                                              const float (&m1)[kPerLane],
-                                              const float (&v1)[kPerLane],
-                                              const float (&den)[kPerLane], uint32_t* mcw,
-                                              uint32_t* vcw, float* msp, float* vsp) {
-  float am = 0.0f, av = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    if (FULL || i < myn) {
-      am = fmaxf(am, fabsf(m1[i]));
-      av = fmaxf(av, fabsf(v1[i]));
-    }
-  }
-  am = hmax16_nonneg(am, hmask);
-  av = hmax16_nonneg(av, hmask);
+                                              const float2 (&m1)[kPerLane / 2],
+                                              const float2 (&nv)[kPerLane / 2],
+                                              const float2 (&ndv)[kPerLane / 2], float lam,
+                                              float lav, uint32_t* mcw, uint32_t* vcw, float* msp,
+                                              float* vsp) {
+  const float am = hmax16_nonneg(lam, hmask);
+  const float av = hmax16_nonneg(lav, hmask);
 
   // ---- first moment: absmax scale, NF4 codes ----
   uint32_t mco = 0;
   float mso = 0.0f;
   if (am >= FLT_MIN) {
-    const float inv = __fdiv_rn(1.0f, am);
+    const float inv = block_rcp(am);
     if ((flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
       uint32_t rw[kPerLane];
       words8(a, tensor_id, kStreamM, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
 #pragma unroll
       for (int i = 0; i < kPerLane; ++i)
         if (FULL || i < myn)
-          mco |= nf4_sr(__fmul_rn(m1[i], inv), uniform23(rw[i]), S.nf4, S.gap) << (4 * i);
+          mco |= nf4_sr(__fmul_rn(el(m1, i), inv), uniform23(rw[i]), S.nf4, S.gap) << (4 * i);
     } else {
 #pragma unroll
       for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
-        const float2 x = __fmul2_rn(make_float2(m1[2 * j], m1[2 * j + 1]), f2(inv));
+        const float2 x = __fmul2_rn(m1[j], f2(inv));
         const float2 b = __ffma2_rn(x, f2(32.0f), f2(kMagic + 32.0f));
         const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? nf4_rtn_bucket(x.y, b.y, S.rtn) : 0u;
         const uint32_t c0 = (FULL || 2 * j < myn) ? nf4_rtn_bucket(x.x, b.x, S.rtn) : 0u;
@@ -484,20 +562,23 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   uint32_t vco = 0;
   float vso = 0.0f;
   if (av >= FLT_MIN) {
-    const float inv = __fdiv_rn(1.0f, av);
+    // -1/s: x = v1/s is then nv * ninv, the same binary32 product
+    const float ninv = -block_rcp(av);
     if (VCODE == kVZip || VCODE == kVZip32) {
       // ZIP-SR ("ZIP-SR / ZE-EDEN", Core equation): keep the lower code point
       // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
       // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
-      const float R = __fmul_rn(__fsqrt_rn(av), a.rs_bc2);
+      const float rs = (av >= exact::kSqrtLo && av <= exact::kSqrtHi) ? exact::sqrt_rn(av)
+                                                                       : __fsqrt_rn(av);
+      const float R = __fmul_rn(rs, a.rs_bc2);
       uint32_t rw[kPerLane];
       words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
       // d(a) == d(b) needs (sqrt(k+1/15) - sqrt(k/15)) R below two ulps of
       // R + eps; the smallest gap is 0.0339, so R > 1e-5 eps rules it out.
       if (R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN)
-        vco = zipsr_codes8<FULL, false, VCODE == kVZip32>(a, S, v1, den, rw, inv, R, myn);
+        vco = zipsr_codes8<FULL, false, VCODE == kVZip32>(a, S, nv, ndv, rw, ninv, R, myn);
       else
-        vco = zipsr_codes8<FULL, true, VCODE == kVZip32>(a, S, v1, den, rw, inv, R, myn);
+        vco = zipsr_codes8<FULL, true, VCODE == kVZip32>(a, S, nv, ndv, rw, ninv, R, myn);
       vso = av;
     } else if (VCODE == kVZiRtn || VCODE == kVZiSr) {
       // State-space rules on the zero-inclusive code: nearest code point, or
@@ -506,7 +587,7 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       if (VCODE == kVZiSr) words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
 #pragma unroll
       for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
-        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+        const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
         const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
 #pragma unroll
         for (int h = 1; h >= 0; --h) {
@@ -528,45 +609,49 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       vso = av;
     } else if (VCODE == kVZeFloor) {
       // Zero-excluded code with a positive floor: nearest (k+1)/16, no rescale.
+      uint32_t P[kPerLane / 2];
 #pragma unroll
-      for (int j = kPerLane / 2 - 1; j >= 0; --j) {
-        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+      for (int j = 0; j < kPerLane / 2; ++j) {
+        const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
         const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
-        const uint32_t k0 = max(__float_as_uint(t2.x) & 31u, 1u) - 1u;
-        const uint32_t k1 = max(__float_as_uint(t2.y) & 31u, 1u) - 1u;
-        const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? k1 : 0u;
-        const uint32_t c0 = (FULL || 2 * j < myn) ? k0 : 0u;
-        vco = (vco * 16u + c1) * 16u + c0;
+        const float2 c2 = __fadd2_rn(t2, f2(-kMagic));             // rint(16x), exact
+        P[j] = ze_code_pair(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)));
       }
+      vco = pack_code_pairs(P, FULL ? kPerLane : myn);
       vso = av;
     } else {
       // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
       // code point, scale times ||x||^2 / max(<x,Q(x)>, 1e-12 s^2) on x = v/s.
       float2 l1[kPerLane / 2];
+      uint32_t P[kPerLane / 2];
 #pragma unroll
       for (int j = 0; j < kPerLane / 2; ++j) {
-        const float2 x2 = __fmul2_rn(make_float2(v1[2 * j], v1[2 * j + 1]), f2(inv));
+        const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
         const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
         const float2 c2 = __fadd2_rn(t2, f2(-kMagic));             // rint(16x), exact
-        const float2 q2 = __fmul2_rn(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)),
-                                     f2(0.0625f));                 // (k+1)/16
-        const uint32_t k0 = max(__float_as_uint(t2.x) & 31u, 1u) - 1u;
-        const uint32_t k1 = max(__float_as_uint(t2.y) & 31u, 1u) - 1u;
+        const float2 cm = make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f));   // k + 1
+        const float2 q2 = __fmul2_rn(cm, f2(0.0625f));             // (k+1)/16
+        P[j] = ze_code_pair(cm);
         float2 xx = __fmul2_rn(x2, x2);
         float2 xq = __fmul2_rn(x2, q2);
         if (!FULL) {
           if (2 * j >= myn) { xx.x = 0.0f; xq.x = 0.0f; }
           if (2 * j + 1 >= myn) { xx.y = 0.0f; xq.y = 0.0f; }
         }
-        if (FULL || 2 * j < myn) vco |= k0 << (8 * j);
-        if (FULL || 2 * j + 1 < myn) vco |= k1 << (8 * j + 4);
         // first tree level: (x0^2 + x1^2, x0 q0 + x1 q1)
         l1[j] = __fadd2_rn(make_float2(xx.x, xq.x), make_float2(xx.y, xq.y));
       }
+      vco = pack_code_pairs(P, FULL ? kPerLane : myn);
       const float2 l2a = __fadd2_rn(l1[0], l1[1]);
       const float2 l2b = __fadd2_rn(l1[2], l1[3]);
       const float2 s = hsum16_tree2(__fadd2_rn(l2a, l2b), hmask);    // (sum x^2, sum x q)
-      vso = __fmul_rn(av, __fdiv_rn(s.x, fmaxf(s.y, 1e-12f)));
+      const float den = fmaxf(s.y, 1e-12f);
+      // s.x >= 1 - 2^-22 (the block's largest x rounds to 1) and den <= 129:
+      // the fast quotient's range holds unless the inputs were not finite
+      const float c = (s.x >= 0x1p-60f && s.x <= 0x1p60f && den <= 0x1p60f)
+                          ? exact::div_rn(s.x, den)
+                          : __fdiv_rn(s.x, den);
+      vso = __fmul_rn(av, c);
     }
   }
 
@@ -578,29 +663,80 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   }
 }
 
-// Decode + moment update + weight update for 8 values of a 4-bit block.
+// Decode + moment update + weight update for 8 values of a 4-bit block
+// ("ZIP-SR / ZE-EDEN", Method flowchart: decode the prior moments, update
+// them, update the weights -- with the unquantised moments, Core equation).
+// Out: m1 and nv = -v1 in pairs, ndv = -d(v1) = -(sqrt(v1) rs_bc2 + eps) in
+// pairs (KEEP_DV), lam / lav = the lane's largest |m1| and v1 over its valid
+// values, and nfacc += 0 * w (NaN once an updated weight is not finite).
+// A lane whose |m1| and v1 all lie in the fast ranges takes the square root
+// and the division from exact_math.cuh (the IEEE results, without branches);
+// any other lane, and every ragged block (FULL false: `myn` valid values),
+// calls the IEEE operations per value.
+template <bool FULL, bool KEEP_DV>
 __device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, float decay,
                                         float (&w)[kPerLane], const float (&g)[kPerLane],
-                                        uint32_t mc, uint32_t vc, float sm, float sv,
-                                        float (&m1)[kPerLane], float (&v1)[kPerLane],
-                                        float (&den)[kPerLane]) {
+                                        uint32_t mc, uint32_t vc, float sm, float sv, int myn,
+                                        float2 (&m1)[kPerLane / 2], float2 (&nv)[kPerLane / 2],
+                                        float2 (&ndv)[kPerLane / 2], float& lam, float& lav,
+                                        float2& nfacc) {
 #pragma unroll
   for (int j = 0; j < kPerLane / 2; ++j) {
     // one byte holds the codes of values 2j (low nibble) and 2j+1 (high nibble)
     const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], f2(sm));
     const float2 v0 = __fmul2_rn(S.vpair[__byte_perm(vc, 0, 0x4440 + j)], f2(sv));
     const float2 gg = make_float2(g[2 * j], g[2 * j + 1]);
-    const float2 mm = __ffma2_rn(f2(a.b1), m0, __fmul2_rn(f2(a.omb1), gg));
-    const float2 vv = __ffma2_rn(f2(a.b2), v0, __fmul2_rn(f2(a.omb2), __fmul2_rn(gg, gg)));
-    const float2 dd = __ffma2_rn(make_float2(__fsqrt_rn(vv.x), __fsqrt_rn(vv.y)), f2(a.rs_bc2),
-                                 f2(a.eps));
-    const float2 qq = make_float2(__fdiv_rn(mm.x, dd.x), __fdiv_rn(mm.y, dd.y));
-    const float2 ww = __ffma2_rn(f2(-a.step_size), qq,
-                                 __fmul2_rn(make_float2(w[2 * j], w[2 * j + 1]), f2(decay)));
-    w[2 * j] = ww.x; w[2 * j + 1] = ww.y;
-    m1[2 * j] = mm.x; m1[2 * j + 1] = mm.y;
-    v1[2 * j] = vv.x; v1[2 * j + 1] = vv.y;
-    den[2 * j] = dd.x; den[2 * j + 1] = dd.y;
+    m1[j] = __ffma2_rn(f2(a.b1), m0, __fmul2_rn(f2(a.omb1), gg));
+    // -v1 = fma(-b2, v0, -(1-b2) g^2), the negation of the canonical v1 exactly
+    nv[j] = __ffma2_rn(f2(a.nb2), v0, __fmul2_rn(f2(a.nomb2), __fmul2_rn(gg, gg)));
+  }
+  bool fast;
+  if (FULL) {
+    lam = absmax8(m1);
+    lav = absmax8(nv);
+    fast = absmin8(m1) >= a.m_lo && lam <= a.m_hi && absmin8(nv) >= a.v_lo && lav <= a.v_hi;
+  } else {
+    lam = 0.0f;
+    lav = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kPerLane / 2; ++j) ndv[j] = f2(-1.0f);   // (slots past myn)
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      if (i < myn) {
+        lam = fmaxf(lam, fabsf(el(m1, i)));
+        lav = fmaxf(lav, fabsf(el(nv, i)));
+      }
+    }
+    fast = false;
+  }
+  if (fast) {
+#pragma unroll
+    for (int j = 0; j < kPerLane / 2; ++j) {
+      const float2 ns = exact::neg_sqrt2_rn(nv[j]);                   // -sqrt(v1)
+      const float2 nd = __ffma2_rn(ns, f2(a.rs_bc2), f2(a.neps));     // -(sqrt(v1) rs + eps)
+      const float2 q = exact::div2_rn_neg(m1[j], nd);                 // m1 / den
+      const float2 ww = __ffma2_rn(f2(a.nstep), q,
+                                   __fmul2_rn(make_float2(w[2 * j], w[2 * j + 1]), f2(decay)));
+      if (KEEP_DV) ndv[j] = nd;
+      w[2 * j] = ww.x;
+      w[2 * j + 1] = ww.y;
+      nfacc = __ffma2_rn(ww, f2(0.0f), nfacc);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      if (FULL || i < myn) {
+        const float v1 = -el(nv, i);
+        const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
+        const float wi = __fmaf_rn(a.nstep, __fdiv_rn(el(m1, i), den), __fmul_rn(w[i], decay));
+        w[i] = wi;
+        if (KEEP_DV) {
+          if (i & 1) ndv[i >> 1].y = -den;
+          else ndv[i >> 1].x = -den;
+        }
+        nfacc.x = __fmaf_rn(wi, 0.0f, nfacc.x);
+      }
+    }
   }
 }
 
@@ -621,13 +757,12 @@ __device__ __forceinline__ void store_w(float* wp, uint16_t* wp16, bool wbf, int
 template <int VCODE, bool BF16W>
 __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTables& S,
                                             const StateArena& st, const UnitHeader* hdp,
-                                            int lane, unsigned hmask) {
+                                            int lane, unsigned hmask, float2& nfacc) {
   const int my0 = lane * kPerLane;
-  const int myn = min(max(hdp->nvalid - my0, 0), kPerLane);
+  const int myn = min(max((int)(hdp->nv_soff & 255u) - my0, 0), kPerLane);
   const uint32_t flags = hdp->flags;
   const bool wbf = BF16W && (flags & kBf16W);
   const float decay = hdp->decay;
-  const uint64_t state = hdp->state;
   // the header's w is the unit's first weight, of either width
   float* wp = wbf ? nullptr : hdp->w + my0;
   uint16_t* wp16 = wbf ? reinterpret_cast<uint16_t*>(hdp->w) + my0 : nullptr;
@@ -639,32 +774,37 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
     g[i] = (i < myn) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
   }
   if (flags & kKindFp32) {
-    float* mp = st.fm + state + my0;
-    float* vp = st.fv + state + my0;
+    float* mp = reinterpret_cast<float*>(hdp->mc) + my0;
+    float* vp = reinterpret_cast<float*>(hdp->vc) + my0;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
       if (i < myn) {
         const float m1 = __fmaf_rn(a.b1, mp[i], __fmul_rn(a.omb1, g[i]));
         const float v1 = __fmaf_rn(a.b2, vp[i], __fmul_rn(a.omb2, __fmul_rn(g[i], g[i])));
         const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
-        store_w<BF16W>(wp, wp16, wbf, i,
-                       __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay)));
+        const float wi = __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay));
+        store_w<BF16W>(wp, wp16, wbf, i, wi);
+        nfacc.x = __fmaf_rn(wi, 0.0f, nfacc.x);
         mp[i] = m1;
         vp[i] = v1;
       }
     }
     return;
   }
-  const uint64_t blk = state;
-  uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
-  uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
-  float m1[kPerLane], v1[kPerLane], den[kPerLane];
-  update8(a, S, decay, w, g, *mcw, *vcw, st.mscale[blk], st.vscale[blk], m1, v1, den);
+  uint32_t* mcw = hdp->mc + lane;
+  uint32_t* vcw = hdp->vc + lane;
+  float* msp = hdp->ms;
+  float* vsp = msp + st.vs_minus_ms;
+  constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
+  float2 m1[kPerLane / 2], nv[kPerLane / 2], ndv[kPerLane / 2];
+  float lam, lav;
+  update8<false, kKeepDv>(a, S, decay, w, g, *mcw, *vcw, *msp, *vsp, myn, m1, nv, ndv, lam, lav,
+                          nfacc);
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i)
     if (i < myn) store_w<BF16W>(wp, wp16, wbf, i, w[i]);
-  requant_store<VCODE, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask, m1, v1,
-                              den, mcw, vcw, st.mscale + blk, st.vscale + blk);
+  requant_store<VCODE, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask, m1, nv,
+                              ndv, lam, lav, mcw, vcw, msp, vsp);
 }
 
 // ---------------------------------------------------------------------------
@@ -748,11 +888,19 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
                 : t_param + e0;
     hd->g = t_grad + e0;
     hd->e0 = (uint64_t)(t_eoff + e0);   // keys the draws
-    hd->state = (t_flags & kKindFp32) ? (uint64_t)(t_soff + e0) : (uint64_t)(t_soff + ub);
+    if (t_flags & kKindFp32) {
+      hd->mc = reinterpret_cast<uint32_t*>(st.fm + t_soff + e0);
+      hd->vc = reinterpret_cast<uint32_t*>(st.fv + t_soff + e0);
+      hd->ms = nullptr;
+    } else {
+      const int64_t blk = t_soff + ub;
+      hd->mc = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2));
+      hd->vc = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2));
+      hd->ms = st.mscale + blk;
+    }
     hd->tensor_id = t_id;
     hd->flags = has ? (t_flags | (staged ? kStaged : 0u)) : kNoUnit;
     hd->decay = t_decay;
-    hd->nvalid = nvalid;
     // Runs of whole blocks of one tensor are contiguous in global memory and
     // in the stage: one bulk copy per array per run.
     const unsigned staged_mask = __ballot_sync(kMask, staged);
@@ -762,14 +910,20 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     const uint32_t dst = stages_s + (uint32_t)(s * kStageBytes);
     uint32_t tx = (uint32_t)__popc(staged_mask) * kUnitTx;
     if (BF16W) tx -= (uint32_t)__popc(__ballot_sync(kMask, staged && wbf)) * 256u;
-    if (lane == 0) mbar_arrive_expect_tx(full, tx);
+    uint32_t w_soff = 0;
     if (BF16W) {
       // A run's weights land packed at the start of its own units' 512-B w
       // slots: 512 B per unit for fp32, 256 B for bf16.  The run starts at the
       // nearest lane at or below this one that does not continue a run.
       const int start = 31 - __clz(~cont_mask & ((2u << lane) - 1u));
-      hd->w_soff = (uint32_t)(kOffW + start * 512 + (lane - start) * (wbf ? 256 : 512));
+      w_soff = (uint32_t)(kOffW + start * 512 + (lane - start) * (wbf ? 256 : 512));
     }
+    hd->nv_soff = (uint32_t)nvalid | (w_soff << 8);
+    // Publish the headers: the warp barrier orders every lane's header stores
+    // before lane 0's arrive, whose release (mbarrier.arrive is a release at
+    // CTA scope) the consumers' acquiring wait on the phase then covers.
+    __syncwarp(kMask);
+    if (lane == 0) mbar_arrive_expect_tx(full, tx);
     if (staged && !cont && !a.fault_stall) {
       // this lane starts a run: it extends over the following lanes whose
       // unit continues it
@@ -808,7 +962,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
 template <int VCODE, bool BF16W>
 __global__ void __launch_bounds__(kCtaThreads, 3)
 adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_end, StepArgs a,
-                   CodeTables tabs, StateArena st) {
+                   StateArena st) {
   extern __shared__ __align__(128) uint8_t s_stage[];
   __shared__ __align__(8) uint64_t s_full[kStages];
   __shared__ __align__(8) uint64_t s_empty[kStages];
@@ -816,23 +970,11 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
 
   {
     const int t = threadIdx.x;
-    if (t < 256) {
-      S.mpair[t] = make_float2(tabs.nf4[t & 15], tabs.nf4[t >> 4]);
-      const bool zx = (VCODE == kVZe || VCODE == kVZeFloor);   // zero-excluded code
-      const float lo = zx ? __fmul_rn((float)((t & 15) + 1), 0.0625f) : tabs.vz[t & 15];
-      const float hi = zx ? __fmul_rn((float)((t >> 4) + 1), 0.0625f) : tabs.vz[t >> 4];
-      S.vpair[t] = make_float2(lo, hi);
-    }
-    if (t < 128) S.rtn[t] = tabs.rtn[t];
-    if (t < 16) {
-      S.nf4[t] = tabs.nf4[t];
-      S.gap[t] = tabs.nf4_gap[t];
-      S.vz[t] = tabs.vz[t];
-      S.zip[t] = make_float4(t == 15 ? INFINITY : tabs.vz[t], tabs.vz_sqrt[max(t - 1, 0)],
-                             tabs.vz_sqrt[t], tabs.vz_sqrt[min(t + 1, 15)]);
-      S.vzp[t] = make_float2(tabs.vz[t], tabs.vz[min(t + 1, 15)]);
-      S.vzmid[t] = tabs.vz_mid[t];
-    }
+    constexpr int kFamily = (VCODE == kVZe || VCODE == kVZeFloor) ? 1 : 0;   // zero-excluded
+    const uint4* src = reinterpret_cast<const uint4*>(&g_code_tables[kFamily]);
+    uint4* dst = reinterpret_cast<uint4*>(&S);
+#pragma unroll 1
+    for (int i = t; i < (int)(sizeof(SmemTables) / 16); i += kCtaThreads) dst[i] = src[i];
     if (t < kStages) {
       // full: the producer's expect-tx arrive plus one cp.async arrive per
       // producer lane; empty: one release per consumer half-warp
@@ -857,8 +999,10 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
   const int half = threadIdx.x >> 4;
   const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
   const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
+  constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
   int s = 0;
   uint32_t parity = 0;
+  float2 nfacc = make_float2(0.0f, 0.0f);   // NaN once an updated weight is not finite
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const uint32_t full = full0 + 8u * s;
     const uint32_t empty = empty0 + 8u * s;
@@ -875,7 +1019,7 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
       {
         const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
         if (wbf) {
-          const uint4 wr = *reinterpret_cast<const uint4*>(sp + hdp->w_soff + lane * 16);
+          const uint4 wr = *reinterpret_cast<const uint4*>(sp + (hdp->nv_soff >> 8) + lane * 16);
           w[0] = bf16lo(wr.x); w[1] = bf16hi(wr.x); w[2] = bf16lo(wr.y); w[3] = bf16hi(wr.y);
           w[4] = bf16lo(wr.z); w[5] = bf16hi(wr.z); w[6] = bf16lo(wr.w); w[7] = bf16hi(wr.w);
         } else {
@@ -893,8 +1037,10 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
       const float sm = *reinterpret_cast<const float*>(sp + kOffMS + half * 4);
       const float sv = *reinterpret_cast<const float*>(sp + kOffVS + half * 4);
 
-      float m1[kPerLane], v1[kPerLane], den[kPerLane];
-      update8(a, S, hdp->decay, w, g, mc, vc, sm, sv, m1, v1, den);
+      float2 m1[kPerLane / 2], nv[kPerLane / 2], ndv[kPerLane / 2];
+      float lam, lav;
+      update8<true, kKeepDv>(a, S, hdp->decay, w, g, mc, vc, sm, sv, kPerLane, m1, nv, ndv, lam,
+                             lav, nfacc);
       if (wbf) {
         uint16_t* wp = reinterpret_cast<uint16_t*>(hdp->w) + lane * kPerLane;
         *reinterpret_cast<uint4*>(wp) = make_uint4(bf16x2_rn(w[0], w[1]), bf16x2_rn(w[2], w[3]),
@@ -904,13 +1050,12 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
         *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
       }
-      const uint64_t blk = hdp->state;
-      uint32_t* mcw = reinterpret_cast<uint32_t*>(st.mcodes + blk * (kBlock / 2)) + lane;
-      uint32_t* vcw = reinterpret_cast<uint32_t*>(st.vcodes + blk * (kBlock / 2)) + lane;
+      float* msp = hdp->ms;
       requant_store<VCODE, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, kPerLane, hmask, m1,
-                                 v1, den, mcw, vcw, st.mscale + blk, st.vscale + blk);
+                                 nv, ndv, lam, lav, hdp->mc + lane, hdp->vc + lane, msp,
+                                 msp + st.vs_minus_ms);
     } else if (!(flags & kNoUnit)) {
-      process_direct<VCODE, BF16W>(a, S, st, hdp, lane, hmask);
+      process_direct<VCODE, BF16W>(a, S, st, hdp, lane, hmask, nfacc);
     }
     // every read of the stage (header included) is done: hand it back
     fence_proxy_async_smem();
@@ -921,6 +1066,7 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
       parity ^= 1u;
     }
   }
+  if (nfacc.x != nfacc.x || nfacc.y != nfacc.y) atomicOr(a.status, 4u);
 }
 
 }  // namespace

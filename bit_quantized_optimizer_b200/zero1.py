@@ -258,6 +258,7 @@ class ZeroAdamW4:
         self.grad_shard = torch.zeros(layout.chunks * S, dtype=flat_grads.dtype,
                                       device=flat_grads.device)
         self._gchunk, self._gshard, self._pchunk, self._pshard = [], [], [], []
+        self.kernel_events = None   # a list to collect (start, end) events of each step launch
         self.steppers = []
         for k in range(layout.chunks):
             c0, c1 = layout.chunk_range(k)
@@ -286,7 +287,16 @@ class ZeroAdamW4:
         for k, stepper in enumerate(self.steppers):
             rs[k].wait()
             if stepper is not None:
-                stepper.step(self.lr if lr is None else lr)
+                if self.kernel_events is not None:      # timing hook (CUDA events)
+                    import torch
+                    e0, e1 = (torch.cuda.Event(enable_timing=True),
+                              torch.cuda.Event(enable_timing=True))
+                    e0.record()
+                    stepper.step(self.lr if lr is None else lr)
+                    e1.record()
+                    self.kernel_events.append((e0, e1))
+                else:
+                    stepper.step(self.lr if lr is None else lr)
             ag.append(dist.all_gather_into_tensor(self._pchunk[k], self._pshard[k],
                                                   group=self.group, async_op=True))
         for w in ag:

@@ -57,10 +57,13 @@ typedef enum {
     ADAMW4_ENOMEM = -3,     /* device or host allocation failed                */
     ADAMW4_ECUDA = -4,      /* a CUDA runtime call or kernel launch failed     */
     ADAMW4_ESTATE = -5,     /* state blob does not match this handle           */
-    ADAMW4_ERANGE = -6,     /* size above a stated maximum                     */
+    ADAMW4_ENONFINITE = -6, /* a step produced a non-finite weight (NaN or +-inf:
+                               from a non-finite grad or weight, or an overflow);
+                               reported by adamw4_sync, the step still ran      */
     ADAMW4_ETIMEOUT = -7,   /* a bounded wait inside the step kernel ran out   */
-    ADAMW4_ECHECK = -8      /* library built with ADAMW4_CHECKED: a unit's values or
+    ADAMW4_ECHECK = -8,     /* library built with ADAMW4_CHECKED: a unit's values or
                                state fell outside its tensor or the state arena */
+    ADAMW4_ERANGE = -9      /* size above a stated maximum, or a buffer too small */
 } adamw4_status;
 
 /* Faults adamw4_inject_fault can arm (test hooks; no GPU fault is raised). */
@@ -78,11 +81,11 @@ typedef enum {
     ADAMW4_V_ZI_RTN = 2,    /* zero-inclusive code, state-space nearest        */
     ADAMW4_V_ZI_SR = 3,     /* zero-inclusive code, state-space SR             */
     ADAMW4_V_ZE_FLOOR = 4,  /* zero-excluded code, nearest, no rescale         */
-    ADAMW4_V_ZIPSR_U32 = 5  /* ZIP-SR deciding on the whole 32-bit draw: lower iff
-                               (word * 2^-32) * B < rhs in one binary64 multiply, so
-                               the keep probability is resolved to 2^-32 instead of
-                               the 23-bit uniform's 2^-23 (whose rounding biases
-                               E[h] upward by up to 2^-23/eps); about 4% slower */
+    ADAMW4_V_ZIPSR_U32 = 5  /* ZIP-SR with the decision taken in binary64: lower
+                               iff (word * 2^-32) * B < rhs in one binary64 multiply
+                               (ZIP-SR itself rounds the word and the product to
+                               binary32; both resolve the keep probability to
+                               2^-32 near zero) */
 } adamw4_vcode;
 
 /* Per-tensor flags. */
@@ -153,6 +156,11 @@ typedef struct {
 typedef struct adamw4_handle adamw4_handle;
 
 /* Creates an optimizer over n tensors on CUDA device `device`.
+ * State layout from "ZIP-SR 4-bit AdamW -- Preconditioner-space stochastic
+ * rounding" (learnaivisually.com), memory paragraph (128-value blocks, one
+ * fp32 scale each, norm layers in fp32), and "ZIP-SR / ZE-EDEN: 4-bit AdamW
+ * state quantization" (daiwk.github.io), Local reproduction notes (uint8
+ * nibble pairs, fp32 state below 4096 elements).
  * Validates every descriptor on the host (non-NULL pointers, 16-byte
  * alignment, numel > 0, unique tensor_id, known flags, elem_offset), classifies
  * each tensor (fp32 state when flagged NORM/FP32_STATE, or when numel < 4096
@@ -167,9 +175,17 @@ int adamw4_create(const adamw4_config *cfg, const adamw4_tensor *tensors, int n,
 /* One optimizer step over every tensor: t <- t + 1, then for each weight
  * decode (m, v), m <- b1 m + (1-b1) g, v <- b2 v + (1-b2) g^2,
  * w <- w (1 - lr wd) - lr/(1-b1^t) * m / (sqrt(v)/sqrt(1-b2^t) + eps),
- * then requantise and pack m and v.  A single kernel launch on `cuda_stream`;
- * the call returns without waiting.  Reads the grads, updates the params and
- * the state in place. */
+ * then requantise and pack m and v: m to NF4 (nearest, or state-space
+ * stochastic rounding for the LM head in the final 10%), v by the handle's
+ * vcode.  Implements "ZIP-SR / ZE-EDEN: 4-bit AdamW state quantization"
+ * (daiwk.github.io), Method flowchart and Core equation (the weights use the
+ * unquantised moments; the ZIP-SR probability and the ZE-EDEN scale), with
+ * the AdamW form of "A New Approach to 4-bit AdamW Optimizer Quantization"
+ * (kongchang.com), AdamW and optimizer states.  lr must be finite and >= 0
+ * (else ADAMW4_EINVAL, nothing enqueued).  A single kernel launch on
+ * `cuda_stream`; the call returns without waiting.  Reads the grads, updates
+ * the params and the state in place; device-side failures (a timed-out wait,
+ * a non-finite updated weight) are reported by adamw4_sync. */
 int adamw4_step(adamw4_handle *h, float lr, void *cuda_stream);
 
 /* The same step with host buffers: for each tensor i, copies grads_host[i]
@@ -191,9 +207,13 @@ int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_ho
 /* Waits for `cuda_stream` and reports whether the steps enqueued on it so far
  * completed.  The step kernel bounds every wait on its shared-memory pipeline
  * (about one second); when a wait runs out, the kernel records it in a device
- * status word and its half-warp stops, leaving that step incomplete.  This
- * call reads and clears the word: ADAMW4_ETIMEOUT if it was set, ADAMW4_ECUDA
- * on a CUDA error, else ADAMW4_OK.  The CUDA context stays usable.
+ * status word and its half-warp stops, leaving that step incomplete.  The
+ * kernel also records an updated weight that is not finite (a NaN or infinite
+ * grad or weight leads to one; the pages leave non-finite inputs undefined, so
+ * the step itself goes on).  This call reads and clears the word:
+ * ADAMW4_ETIMEOUT if a wait ran out, else ADAMW4_ENONFINITE if a weight was
+ * not finite, ADAMW4_ECUDA on a CUDA error, else ADAMW4_OK.  The CUDA context
+ * stays usable.
  * A library built with -DADAMW4_CHECKED (build.py --checked, a debugging aid
  * in place of a memory checker) also tests every unit's element and state
  * range on the device; a unit outside them is skipped and this call returns
@@ -201,7 +221,8 @@ int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_ho
 int adamw4_sync(adamw4_handle *h, void *cuda_stream);
 
 /* Test hook: arms `fault` (ADAMW4_FAULT_STALL_PIPELINE, or 0 to disarm) for
- * the next adamw4_step only.  With the stall armed the kernel marks its
+ * the next adamw4_step only (with h = NULL: for the next adamw4_step_noalloc
+ * call of this process instead).  With the stall armed the kernel marks its
  * pipeline stages as filled without issuing the copies, so every stage wait
  * runs out after its time limit and adamw4_sync then returns ADAMW4_ETIMEOUT.
  * Nothing faults; the handle's state after that step is unspecified. */
@@ -243,18 +264,29 @@ int64_t adamw4_state_bytes(const adamw4_handle *h);
 int adamw4_state_export(const adamw4_handle *h, void *host_buf, int64_t cap, int64_t *used);
 int adamw4_state_import(adamw4_handle *h, const void *host_buf, int64_t len);
 
+/* The state class the library gives one descriptor (host only; its pointers
+ * are not looked at): 1 when it keeps fp32 m and v (flagged NORM or
+ * FP32_STATE, or numel < ADAMW4_MIN_QUANT_NUMEL and not flagged
+ * QUANT_STATE), 0 when it keeps 4-bit codes and block scales, ADAMW4_EINVAL
+ * for a NULL pointer, numel <= 0, unknown flag bits, QUANT_STATE with NORM or
+ * FP32_STATE, or a bad elem_offset.  The classification follows "ZIP-SR
+ * 4-bit AdamW -- Preconditioner-space stochastic rounding" (learnaivisually.com),
+ * memory paragraph (normalisation layers in fp32), and "ZIP-SR / ZE-EDEN:
+ * 4-bit AdamW state quantization" (daiwk.github.io), Local reproduction
+ * notes (tensors below 4096 elements in fp32). */
+int adamw4_tensor_state_kind(const adamw4_tensor *t);
+
 /* Launch geometry used by adamw4_step (filled at create): CUDA blocks, threads
  * per block, and 128-value work units (4-bit blocks plus fp32 chunks). */
 int adamw4_launch_info(const adamw4_handle *h, int *grid, int *block, int64_t *units);
 
 /* ---------------------------------------------------------------------------
  * Allocation-free step.  The paper has no counterpart: this entry point exists
- * for callers that must not allocate device memory.  Examples are code running
- * while a CUDA graph is being captured, where an allocation would be refused or
- * frozen into the graph; programs whose device memory belongs to a pooling
- * allocator or a fixed arena sized at start-up, which has to account for every
- * byte; and tight training loops, where cudaMalloc and cudaFree can
- * synchronise the device and stall other streams.
+ * for callers that must not allocate device memory.  Examples are programs
+ * whose device memory belongs to a pooling allocator or a fixed arena sized at
+ * start-up, which has to account for every byte, and tight training loops,
+ * where cudaMalloc and cudaFree can synchronise the device and stall other
+ * streams.
  *
  * It runs the same step as adamw4_step, without a handle.  The caller passes
  * the tensors, the packed state buffers below, the step number t (1-based)
@@ -267,14 +299,17 @@ int adamw4_launch_info(const adamw4_handle *h, int *grid, int *block, int64_t *u
  *     The status code is the whole report: this call records no message for
  *     adamw4_last_error.
  *   - The first call on a device looks up the array's device address and the
- *     launch geometry for that device; make that first call before any stream
- *     capture.
+ *     launch geometry for that device.
  *   - All calls share the one array and each overwrites it: calls whose work
  *     overlaps on the GPU (different streams, or different host threads without
  *     ordering) race.  Calls on one stream are ordered and safe.
- *   - A pipeline wait that runs out ends the kernel early like in adamw4_step;
- *     this entry point has no handle to report it, so only launch errors are
- *     returned (ADAMW4_ECUDA).
+ *   - The descriptor table is copied from a host staging array of this library
+ *     with a pageable cudaMemcpyAsync, which the call's return leaves free for
+ *     the next call.
+ *   - Device-side failures (a pipeline wait that ran out, which ends the kernel
+ *     early like in adamw4_step, or a non-finite updated weight) go to the
+ *     status word in the array; adamw4_noalloc_sync reads and clears it.  The
+ *     call itself returns only host-side and launch errors.
  * Results equal adamw4_step's for the same inputs, state and t.
  * ------------------------------------------------------------------------- */
 #define ADAMW4_NOALLOC_MAX_TENSORS 1024
@@ -297,6 +332,15 @@ typedef struct {
 int adamw4_step_noalloc(const adamw4_config *cfg, const adamw4_tensor *tensors, int n,
                         const adamw4_state_buffers *state, int64_t t, float lr, int device,
                         void *cuda_stream);
+
+/* Waits for `cuda_stream` and reads and clears the allocation-free step's
+ * status word on `device` (with cudaMemcpyFromSymbol / cudaMemcpyToSymbol, no
+ * allocation): ADAMW4_ETIMEOUT if a stage wait of a call on that device ran
+ * out, else ADAMW4_ENONFINITE if a call produced a non-finite weight,
+ * ADAMW4_ECUDA on a CUDA error, else ADAMW4_OK.  The word is shared by every
+ * call on the device, so it reports all of them since the last read.
+ * ADAMW4_EINVAL for a device no call has used yet. */
+int adamw4_noalloc_sync(int device, void *cuda_stream);
 
 /* Message of the last failed call on this handle, or of the last failed call
  * on this thread when h is NULL.  Never NULL; valid until the next call. */

@@ -55,7 +55,9 @@ def assert_weights_close(w_gpu, w_ref, w_old, what=""):
     w_gpu = np.asarray(w_gpu, np.float64)
     w_ref = np.asarray(w_ref, np.float64)
     scale = np.maximum(np.abs(w_ref), np.abs(np.asarray(w_old, np.float64)))
-    bad = np.abs(w_gpu - w_ref) > 1e-6 * scale
+    with np.errstate(invalid="ignore"):            # equal infinities subtract to NaN
+        same = (w_gpu == w_ref) | (np.isnan(w_gpu) & np.isnan(w_ref))
+        bad = ~same & ~(np.abs(w_gpu - w_ref) <= 1e-6 * scale)
     assert not bad.any(), (f"{what}: {bad.sum()} weights differ beyond 1e-6, first at "
                            f"{np.argmax(bad)}: gpu {w_gpu[bad][0]!r} oracle {w_ref[bad][0]!r}")
 
@@ -276,6 +278,87 @@ def sampled_parity(name, vcode, steps, t0=0, total_steps=0, prewarm=False, seed=
             np.testing.assert_allclose(got["tensors"][i]["m"], st.m, rtol=1e-6, atol=0)
             np.testing.assert_allclose(got["tensors"][i]["v"], st.v, rtol=1e-6, atol=0)
         return checked
+    finally:
+        opt.close()
+        del params, grads
+        torch.cuda.empty_cache()
+
+
+def teacher_forced_parity(name, vcode, steps, seed=0, what=""):
+    """Runs the CUDA path for `steps` steps over a full-size list (device
+    inputs, one seeded grad set reused every step, zero initial state), then
+    checks the last step teacher-forced: the state and weights the GPU holds
+    after step `steps` - 1 are given to the oracle, which computes step
+    `steps` on sampled blocks of every 4-bit tensor and on every fp32-state
+    tensor; the GPU's own step `steps` must match it.  Returns (blocks
+    checked, share of the sampled v codes that are 0 after step `steps` - 1)."""
+    import torch
+    ts = workloads.tensor_list(name)
+    params, grads = workloads.device_inputs(name, ts, seed=seed)
+    sel = sampled_blocks(ts, seed=seed + 1)
+    fp_idx = [i for i, t in enumerate(ts) if oracle.is_fp32_state(t["numel"], t["flags"])]
+    B_ = binding()
+    opt = B_.AdamW4(params, grads, ts, lr=1e-3, vcode=vcode, seed=0)
+    try:
+        for _ in range(steps - 1):
+            opt.step()
+        torch.cuda.synchronize()
+        before = parse_blob(opt.state_dict_blob())
+        assert before["t"] == steps - 1
+        ref = oracle_for(ts, vcode=vcode, seed=0)
+        ref.t = steps - 1
+        d_in = {}
+        zero_codes, n_codes = 0, 0
+        for i, blocks in sel.items():
+            w, valid = _gather_blocks(params[i], ts[i]["numel"], blocks, np.float32)
+            g, _ = _gather_blocks(grads[i], ts[i]["numel"], blocks, np.uint16)
+            tb = before["tensors"][i]
+            vc = np.concatenate([tb["vcodes"][b * 64:(b + 1) * 64] for b in blocks]).copy()
+            nib = np.stack([vc & 15, vc >> 4], axis=1).reshape(-1)[:valid.size][valid]
+            zero_codes += int((nib == 0).sum())
+            n_codes += nib.size
+            d_in[i] = dict(blocks=blocks, w=w, w0=w.copy(), g=g, valid=valid,
+                           mc=np.concatenate([tb["mcodes"][b * 64:(b + 1) * 64] for b in blocks]).copy(),
+                           vc=vc, ms=tb["mscale"][blocks].copy(), vs=tb["vscale"][blocks].copy())
+        fp_w = {i: params[i].cpu().numpy().copy() for i in fp_idx}
+        fp_g = {i: grads[i].view(torch.int16).cpu().numpy().view(np.uint16).copy() for i in fp_idx}
+        for i in fp_idx:
+            st = ref.tensors[i]
+            st.m = before["tensors"][i]["m"].copy()
+            st.v = before["tensors"][i]["v"].copy()
+        del before
+        # step `steps`: the GPU, and the oracle from the GPU's state
+        opt.step()
+        ref.t = steps
+        for i, d in d_in.items():
+            ref.step_blocks(i, d["blocks"], d["w"], d["g"], d["mc"], d["ms"], d["vc"], d["vs"],
+                            advance=False)
+        old_fp = {i: fp_w[i].copy() for i in fp_idx}
+        ref.step([fp_w[i] for i in fp_idx], [fp_g[i] for i in fp_idx], only=fp_idx, advance=False)
+        torch.cuda.synchronize()
+        after = parse_blob(opt.state_dict_blob())
+        checked = 0
+        for i, d in d_in.items():
+            wg, valid = _gather_blocks(params[i], ts[i]["numel"], d["blocks"], np.float32)
+            assert_weights_close(wg[valid], d["w"][valid], d["w0"][valid], f"{what} tensor {i}")
+            tb = after["tensors"][i]
+            for j, b in enumerate(d["blocks"]):
+                for key, arr in (("mcodes", d["mc"]), ("vcodes", d["vc"])):
+                    assert np.array_equal(tb[key][b * 64:(b + 1) * 64], arr[j * 64:(j + 1) * 64]), \
+                        f"{what} tensor {i} block {b} {key}"
+                assert tb["mscale"][b] == d["ms"][j], f"{what} tensor {i} block {b} m scale"
+                if vcode != 1:
+                    assert tb["vscale"][b] == d["vs"][j], f"{what} tensor {i} block {b} v scale"
+                else:
+                    assert abs(tb["vscale"][b] - d["vs"][j]) <= 1e-6 * abs(d["vs"][j]), \
+                        f"{what} tensor {i} block {b} v scale"
+                checked += 1
+        for i in fp_idx:
+            st = ref.tensors[i]
+            assert_weights_close(params[i].cpu().numpy(), fp_w[i], old_fp[i], f"{what} fp32 {i}")
+            np.testing.assert_allclose(after["tensors"][i]["m"], st.m, rtol=1e-6, atol=0)
+            np.testing.assert_allclose(after["tensors"][i]["v"], st.v, rtol=1e-6, atol=0)
+        return checked, zero_codes / max(n_codes, 1)
     finally:
         opt.close()
         del params, grads

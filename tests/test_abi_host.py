@@ -180,10 +180,73 @@ def test_binding_constants_match_the_header():
     for name in ("ADAMW4_V_ZIPSR", "ADAMW4_V_ZEEDEN", "ADAMW4_V_ZI_RTN", "ADAMW4_V_ZI_SR",
                  "ADAMW4_V_ZE_FLOOR", "ADAMW4_V_ZIPSR_U32", "ADAMW4_T_NORM", "ADAMW4_T_LM_HEAD",
                  "ADAMW4_T_FP32_STATE", "ADAMW4_T_QUANT_STATE", "ADAMW4_T_BF16_PARAM",
-                 "ADAMW4_NOALLOC_MAX_TENSORS", "ADAMW4_ETIMEOUT", "ADAMW4_ECHECK"):
+                 "ADAMW4_NOALLOC_MAX_TENSORS", "ADAMW4_ETIMEOUT", "ADAMW4_ECHECK",
+                 "ADAMW4_ENONFINITE", "ADAMW4_ERANGE"):
         assert name in vals and getattr(B, name) == vals[name], name
     codes = {v for n, v in vals.items() if n in (
         "ADAMW4_OK", "ADAMW4_EINVAL", "ADAMW4_EALIGN", "ADAMW4_ENOMEM", "ADAMW4_ECUDA",
-        "ADAMW4_ESTATE", "ADAMW4_ERANGE", "ADAMW4_ETIMEOUT", "ADAMW4_ECHECK")}
+        "ADAMW4_ESTATE", "ADAMW4_ENONFINITE", "ADAMW4_ERANGE", "ADAMW4_ETIMEOUT",
+        "ADAMW4_ECHECK")}
     assert codes == set(B.STATUS)
     assert B.MIN_QUANT_NUMEL == vals["ADAMW4_MIN_QUANT_NUMEL"] and B.BLOCK == vals["ADAMW4_BLOCK"]
+
+
+def _noalloc(L, ts, sb, n=None):
+    arr = (B.adamw4_tensor * max(len(ts), 1))(*ts)
+    return L.adamw4_step_noalloc(ctypes.byref(_cfg()), arr, len(ts) if n is None else n,
+                                 ctypes.byref(sb), 1, ctypes.c_float(1e-3), 0, None)
+
+
+
+
+def _no_gpu():
+    """These checks hand the library fake device addresses: on a machine with
+    a GPU a descriptor list that passed validation would be launched on
+    them, so they run only where no GPU is visible."""
+    try:
+        import torch
+        return not torch.cuda.is_available()
+    except Exception:
+        return True
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="host-validation check with fake device addresses")
+def test_noalloc_rejects_missing_state_buffers(L):
+    """The allocation-free step refuses, on the host and before any CUDA call,
+    a NULL state buffer that its tensor list needs: the codes and scales for a
+    4-bit tensor, the fp32 moments for an fp32-state tensor."""
+    q = B.adamw4_tensor(P0, P0 + (1 << 20), 8192, 1, 0, 0.0)          # 4-bit state
+    f = B.adamw4_tensor(P0 + (2 << 20), P0 + (3 << 20), 1000, 2, 0, 0.0)   # fp32 state
+    S = P0 + (8 << 20)
+    full = [S, S + 4096, S + 8192, S + 12288, S + 16384, S + 20480]
+    for missing in range(4):                       # any of the four 4-bit buffers
+        bufs = list(full)
+        bufs[missing] = 0
+        assert _noalloc(L, [q], B.adamw4_state_buffers(*bufs)) == -1
+    for missing in (4, 5):                         # either fp32 moment buffer
+        bufs = list(full)
+        bufs[missing] = 0
+        assert _noalloc(L, [f], B.adamw4_state_buffers(*bufs)) == -1
+    # the buffers a list does not use may be NULL: validation passes, and the
+    # call then fails only on the missing GPU (a CUDA error, not EINVAL)
+    assert _noalloc(L, [q], B.adamw4_state_buffers(S, S + 4096, S + 8192, S + 12288, 0, 0)) == -4
+    assert _noalloc(L, [f], B.adamw4_state_buffers(0, 0, 0, 0, S + 16384, S + 20480)) == -4
+
+
+def test_tensor_state_kind_follows_the_documented_rule(L):
+    """adamw4_tensor_state_kind (which the binding's is_fp32_state asks) gives
+    the classification the header documents: fp32 for NORM / FP32_STATE, 4-bit
+    for QUANT_STATE, else fp32 below 4096 elements; invalid descriptors are
+    refused."""
+    N, F, Q, H = (B.ADAMW4_T_NORM, B.ADAMW4_T_FP32_STATE, B.ADAMW4_T_QUANT_STATE,
+                  B.ADAMW4_T_LM_HEAD)
+    cases = [(1, 0, 1), (100, 0, 1), (4095, 0, 1), (4096, 0, 0), (8192, 0, 0), (8192, N, 1),
+             (8192, F, 1), (100, Q, 0), (4095, Q, 0), (4096, H, 0), (4000, H, 1),
+             (1 << 33, 0, 0), (1 << 33, N, 1), (4096, B.ADAMW4_T_BF16_PARAM, 0)]
+    for numel, flags, want in cases:
+        assert B.adamw4_tensor_state_kind(numel, flags) == want, (numel, flags)
+        assert B.is_fp32_state(numel, flags) == bool(want)
+    for numel, flags, off in [(0, 0, 0), (-5, 0, 0), (4096, 1 << 9, 0), (4096, Q | N, 0),
+                              (4096, 0, 100), (4096, 0, 1 << 39)]:
+        with pytest.raises(B.AdamW4Error):
+            B.adamw4_tensor_state_kind(numel, flags, off)

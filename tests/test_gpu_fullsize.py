@@ -69,3 +69,22 @@ def test_tensor_past_2_31_elements():
     including the two around element 2^31."""
     n = sampled_parity("huge-2g", vcode=0, steps=2, t0=8, total_steps=10, what="huge-2g")
     assert n > 100
+
+
+@pytest.mark.parametrize("vcode", [0, 1])
+def test_gpt_2p7b_step_100_teacher_forced(vcode):
+    """The benchmark's run length: 99 steps of the 2.7B list on the GPU (one
+    seeded grad set reused, as the benchmark times it), then step 100
+    teacher-forced -- the oracle starts from the GPU's state and weights after
+    step 99 and computes step 100 on sampled blocks and every fp32-state
+    tensor.  By then v has settled, and for ZIP-SR a large share of the
+    codes sit at 0, the cell next to zero where the draw's resolution
+    matters ("ZIP-SR 4-bit AdamW -- Preconditioner-space stochastic
+    rounding", worked example paragraph)."""
+    from gpu_common import teacher_forced_parity
+    n, zero_share = teacher_forced_parity("gpt-2.7b", vcode, 100, what=f"gpt-2.7b v{vcode} t100")
+    assert n > 1500
+    print(f"v{vcode}: {n} blocks checked at step 100; v codes at 0 after step 99: "
+          f"{100 * zero_share:.1f}%")
+    if vcode == 0:
+        assert zero_share > 0.2

@@ -1,8 +1,8 @@
 """The allocation-free step, for callers that must not allocate device memory
-(code inside CUDA graph capture, programs whose memory belongs to a pooling
-allocator or a fixed arena, loops where cudaMalloc's device synchronisation is
-not acceptable).  It keeps the step kernel's scratch -- the descriptor table
-and the status word -- in a static device array instead of allocating it.
+(programs whose memory belongs to a pooling allocator or a fixed arena, loops
+where cudaMalloc's device synchronisation is not acceptable).  It keeps the
+step kernel's scratch -- the descriptor table and the status word -- in a
+static device array instead of allocating it.
 
 Checked through the C ABI against the handle-based step: two calls in a row on
 the same inputs must give the same weights and packed state, within the
@@ -121,7 +121,7 @@ def test_noalloc_rejects_too_many_tensors():
     cfg = B.adamw4_config(1e-3, 0.9, 0.999, 1e-8, 0, 0, 0)
     with pytest.raises(B.AdamW4Error) as err:
         B.adamw4_step_noalloc(cfg, descs, sb, 1, 1e-3, 0, None)
-    assert err.value.code == -6
+    assert err.value.code == B.ADAMW4_ERANGE
 
 
 def test_noalloc_bf16_weights_and_pieces():
@@ -190,3 +190,77 @@ def test_noalloc_bf16_weights_and_pieces():
         assert r["mscale"].tobytes() == ms[b4:b4 + nb].tobytes()
         assert r["vscale"].tobytes() == vs[b4:b4 + nb].tobytes()
         b4 += nb
+
+
+def _small_noalloc_case(B, dev, vcode=0):
+    """One 4-bit tensor and one fp32-state tensor on caller-owned buffers."""
+    import torch
+    ts = [dict(numel=128 * 64, tensor_id=1, flags=0, weight_decay=0.1),
+          dict(numel=900, tensor_id=2, flags=0, weight_decay=0.0)]
+    rng = np.random.default_rng(11)
+    params = [torch.from_numpy((rng.standard_normal(t["numel"]) * 0.02).astype(np.float32)).to(dev)
+              for t in ts]
+    grads = [torch.from_numpy(workloads.bf16_bits((rng.standard_normal(t["numel"]) * 1e-3)
+                                                  .astype(np.float32)).view(np.int16)).to(dev)
+             .view(torch.bfloat16) for t in ts]
+    nb4, n32 = _layout(ts)
+    bufs = [torch.zeros(nb4 * 64, dtype=torch.uint8, device=dev),
+            torch.zeros(nb4 * 64, dtype=torch.uint8, device=dev),
+            torch.zeros(nb4, dtype=torch.float32, device=dev),
+            torch.zeros(nb4, dtype=torch.float32, device=dev),
+            torch.zeros(n32, dtype=torch.float32, device=dev),
+            torch.zeros(n32, dtype=torch.float32, device=dev)]
+    sb = B.adamw4_state_buffers(*[b.data_ptr() for b in bufs])
+    cfg = B.adamw4_config(1e-3, 0.9, 0.999, 1e-8, vcode, 9, 0)
+    descs = [B.adamw4_tensor(p.data_ptr(), g.data_ptr(), t["numel"], t["tensor_id"], t["flags"],
+                             t["weight_decay"]) for p, g, t in zip(params, grads, ts)]
+    return params, grads, bufs, sb, cfg, descs
+
+
+def _clear_status(B, stream):
+    """Reads and clears the status word (earlier calls may have set it)."""
+    try:
+        B.adamw4_noalloc_sync(0, stream)
+    except B.AdamW4Error:
+        pass
+
+
+def test_noalloc_status_reports_timeout_and_nonfinite_weights():
+    """The device status word of the allocation-free step, read through
+    adamw4_noalloc_sync: a stage stall armed on the host for one call (the
+    kernel's bounded waits run out after about a second each; nothing faults)
+    gives ADAMW4_ETIMEOUT; a NaN grad written on the host gives
+    ADAMW4_ENONFINITE; each is reported once, and a clean call then reads
+    ADAMW4_OK.  The context stays usable throughout."""
+    import torch
+    B = binding()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream().cuda_stream
+    params, grads, bufs, sb, cfg, descs = _small_noalloc_case(B, dev)
+    B.adamw4_step_noalloc(cfg, descs, sb, 1, 1e-3, 0, stream)
+    _clear_status(B, stream)
+    B.adamw4_step_noalloc(cfg, descs, sb, 2, 1e-3, 0, stream)
+    B.adamw4_noalloc_sync(0, stream)                          # clean: OK
+
+    B.adamw4_inject_fault(None, B.ADAMW4_FAULT_STALL_PIPELINE)
+    B.adamw4_step_noalloc(cfg, descs, sb, 3, 1e-3, 0, stream)
+    with pytest.raises(B.AdamW4Error) as err:
+        B.adamw4_noalloc_sync(0, stream)
+    assert err.value.code == B.ADAMW4_ETIMEOUT
+    B.adamw4_noalloc_sync(0, stream)                          # cleared
+
+    grads[0][100] = float("nan")
+    B.adamw4_step_noalloc(cfg, descs, sb, 4, 1e-3, 0, stream)
+    with pytest.raises(B.AdamW4Error) as err:
+        B.adamw4_noalloc_sync(0, stream)
+    assert err.value.code == B.ADAMW4_ENONFINITE
+    B.adamw4_noalloc_sync(0, stream)                          # cleared
+    # the context is still usable: a small device computation works
+    assert float(torch.ones(4, device=dev).sum()) == 4.0
+
+
+def test_noalloc_status_needs_a_used_device():
+    B = binding()
+    with pytest.raises(B.AdamW4Error) as err:
+        B.adamw4_noalloc_sync(63, None)
+    assert err.value.code == -1
