@@ -99,6 +99,15 @@ struct DeviceGuard {
   }
 };
 
+// The NF4 nearest-level bucket of x (the kernel's nf4_rtn_bucket reads the
+// same one from the bits of fma(x, 256, 1.5 * 2^23 + 256)).
+int nf4_bucket(float x) {
+  const float y = std::fma(x, 256.0f, 12583168.0f);
+  int32_t bits;
+  std::memcpy(&bits, &y, 4);
+  return std::min(std::max(bits - 0x4B400000, 0), 512) >> 3;
+}
+
 void build_tables(CodeTables* T) {
   for (int j = 0; j < 16; ++j) T->nf4[j] = kNF4Levels[j];
   for (int j = 0; j < 15; ++j) T->nf4_gap[j] = kNF4Levels[j + 1] - kNF4Levels[j];
@@ -115,16 +124,12 @@ void build_tables(CodeTables* T) {
   float mid[15];
   for (int j = 0; j < 15; ++j)
     mid[j] = (float)(((double)kNF4Levels[j] + (double)kNF4Levels[j + 1]) * 0.5);
-  // Bucket b of x is round(32 x + 32), in [0, 64] for |x| <= 1 + 2^-23 and
-  // monotone in x.  A bucket holds at most one midpoint, so the nearest level
-  // is the count of midpoints in lower buckets plus one comparison.
+  // Bucket b of x is floor(round(256 x + 256) / 8), in [0, 64] for
+  // |x| <= 1 + 2^-23 and monotone in x.  A bucket holds at most one midpoint,
+  // so the nearest level is the count of midpoints in lower buckets plus one
+  // comparison.
   int bucket_of[15];
-  for (int j = 0; j < 15; ++j) {
-    const float y = std::fma(mid[j], 32.0f, 12582944.0f);
-    int32_t bits;
-    std::memcpy(&bits, &y, 4);
-    bucket_of[j] = std::min(std::max(bits - 0x4B400000, 0), 64);
-  }
+  for (int j = 0; j < 15; ++j) bucket_of[j] = nf4_bucket(mid[j]);
   // Indices 65..127 never occur for |x| <= 1 + 2^-23; they hold "above all".
   for (int b = 0; b < 128; ++b) {
     int base = 0;
@@ -186,10 +191,7 @@ bool tables_ok(const CodeTables& T) {
   int seen[65] = {0};
   for (int j = 0; j < 15; ++j) {
     const float mid = (float)(((double)T.nf4[j] + (double)T.nf4[j + 1]) * 0.5);
-    const float y = std::fma(mid, 32.0f, 12582944.0f);
-    int32_t bits;
-    std::memcpy(&bits, &y, 4);
-    if (++seen[std::min(std::max(bits - 0x4B400000, 0), 64)] > 1) return false;
+    if (++seen[nf4_bucket(mid)] > 1) return false;
   }
   return true;
 }
@@ -223,6 +225,28 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.v_hi = 0x1p64f;
   const bool fast_ok = a.eps >= 0x1p-60f && a.eps <= 0x1p10f && a.rs_bc2 <= 0x1p20f;
   a.m_hi = fast_ok ? std::min(std::ldexp(a.eps, 100), 0x1p100f) : -1.0f;
+  auto pair = [](float x) { return make_float2(x, x); };
+  a.p_b1 = pair(a.b1);
+  a.p_omb1 = pair(a.omb1);
+  a.p_nb2 = pair(a.nb2);
+  a.p_nomb2 = pair(a.nomb2);
+  a.p_rs = pair(a.rs_bc2);
+  a.p_eps = pair(a.eps);
+  a.p_neps = pair(a.neps);
+  a.p_nstep = pair(a.nstep);
+  a.k_half = pair(0.5f);
+  a.k_one = pair(1.0f);
+  a.k_zero = pair(0.0f);
+  a.k_m1 = pair(-1.0f);
+  a.k_15 = pair(15.0f);
+  a.k_16 = pair(16.0f);
+  a.k_256 = pair(256.0f);
+  a.k_magic = pair(kMagic);
+  a.k_nmagic = pair(-kMagic);
+  a.k_magic256 = pair(kMagic + 256.0f);
+  a.k_magicm1 = pair(kMagic - 1.0f);
+  a.k_1_16 = pair(0.0625f);
+  a.k_2m32 = pair(0x1p-32f);
   // Philox round keys: round r uses the seed words plus r times the Weyl
   // constants (mod 2^32).
   for (int r = 0; r < 10; ++r) {

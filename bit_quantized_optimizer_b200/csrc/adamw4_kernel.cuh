@@ -63,15 +63,16 @@ constexpr int kProducerWarp = kConsumerThreads / 32;
 constexpr int kStages = 3;                        // tiles in flight per CTA
 // A tile is kHalves consecutive units; stage layout (CTA-wide):
 //   16 unit headers (64 B each) | w 16 x 512 B | g 16 x 256 B |
-//   m codes 16 x 64 B | v codes 16 x 64 B | m scales 16 x 4 B | v scales 16 x 4 B
+//   m codes 16 x 64 B | v codes 16 x 64 B | m scales 16 x 8 B | v scales 16 x 8 B
+// (each scale twice, as the pair the f32x2 decode multiplies by)
 constexpr int kOffHdr = 0;
 constexpr int kOffW = kOffHdr + kHalves * 64;
 constexpr int kOffG = kOffW + kHalves * 512;
 constexpr int kOffMC = kOffG + kHalves * 256;
 constexpr int kOffVC = kOffMC + kHalves * 64;
 constexpr int kOffMS = kOffVC + kHalves * 64;
-constexpr int kOffVS = kOffMS + kHalves * 4;
-constexpr int kStageBytes = kOffVS + kHalves * 4; // 15,488 B, a 16-byte multiple
+constexpr int kOffVS = kOffMS + kHalves * 8;
+constexpr int kStageBytes = kOffVS + kHalves * 8; // 15,616 B, a 16-byte multiple
 constexpr uint32_t kUnitTx = 896;                 // bulk-copied bytes of one whole block
 constexpr int kSmemStages = kStages * kStageBytes;
 static_assert(kStageBytes % 16 == 0, "stage alignment");
@@ -124,6 +125,12 @@ struct StepArgs {
   // in [v_lo, v_hi]; otherwise it uses the IEEE operations.  m_hi < 0
   // switches the fast path off (eps or rs_bc2 outside the range it needs).
   float m_lo, m_hi, v_lo, v_hi;
+  // The broadcast operands of the f32x2 instructions, duplicated into pairs
+  // here so that the instructions read them from the kernel parameters
+  // instead of rebuilding a register pair for each use.
+  float2 p_b1, p_omb1, p_nb2, p_nomb2, p_rs, p_eps, p_neps, p_nstep;
+  float2 k_half, k_one, k_zero, k_m1, k_15, k_16, k_256, k_magic, k_nmagic, k_magic256,
+      k_magicm1, k_1_16, k_2m32;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
   int lm_sr_active;      // final-10% LM-head phase
@@ -141,7 +148,8 @@ struct CodeTables {
   float vz[16];         // ZIP-SR code points k/15
   float vz_sqrt[16];    // sqrt(k/15)
   float vz_mid[16];     // nearest-point thresholds of the k/15 code (15 used)
-  float2 rtn[128];      // NF4 nearest-level buckets: .x threshold, .y base code (int bits)
+  float2 rtn[128];      // NF4 nearest-level buckets (floor(round(256x + 256)/8)):
+                        // .x threshold, .y base code (int bits)
 };
 
 struct StateArena {
@@ -358,20 +366,36 @@ __device__ __forceinline__ float absmin8(const float2 (&x)[4]) {
 
 // The ZIP-SR uniforms of two draw words: each word rounded to the nearest
 // binary32 (ties to even) and scaled by 2^-32, exactly.
-__device__ __forceinline__ float2 uniform32x2(uint32_t w0, uint32_t w1) {
-  return __fmul2_rn(make_float2(__uint2float_rn(w0), __uint2float_rn(w1)), f2(0x1p-32f));
+__device__ __forceinline__ float2 uniform32x2(uint32_t w0, uint32_t w1, float2 k2m32) {
+  return __fmul2_rn(make_float2(__uint2float_rn(w0), __uint2float_rn(w1)), k2m32);
 }
+
+// Collectives over a half-warp.  FULLW: both half-warps of the warp execute
+// the call together, so it runs with the constant full-warp mask (no
+// convergence bookkeeping around it); else with the half-warp's own mask.
+constexpr unsigned kFullMask = 0xFFFFFFFFu;
 
 // Max of non-negative binary32 values over a half-warp: their bit patterns
 // order like the values, so an integer reduction gives the exact maximum.
-__device__ __forceinline__ float hmax16_nonneg(float v, unsigned mask) {
-  return __uint_as_float(__reduce_max_sync(mask, __float_as_uint(v)));
+// Full-warp form: one reduction per half, the other half contributing 0.
+template <bool FULLW>
+__device__ __forceinline__ float hmax16(float v, unsigned hmask) {
+  const uint32_t b = __float_as_uint(v);
+  if (FULLW) {
+    const bool hi = (threadIdx.x & 16) != 0;
+    const uint32_t mlo = __reduce_max_sync(kFullMask, hi ? 0u : b);
+    const uint32_t mhi = __reduce_max_sync(kFullMask, hi ? b : 0u);
+    return __uint_as_float(hi ? mhi : mlo);
+  }
+  return __uint_as_float(__reduce_max_sync(hmask, b));
 }
 
 // Balanced pairwise sum of (x, y) pairs over the half-warp: partner offsets 1,
 // 2, 4, 8 join adjacent 8-value groups in index order (IEEE addition is
 // commutative, so both partners hold the same bits).
-__device__ __forceinline__ float2 hsum16_tree2(float2 v, unsigned mask) {
+template <bool FULLW>
+__device__ __forceinline__ float2 hsum16_tree2(float2 v, unsigned hmask) {
+  const unsigned mask = FULLW ? kFullMask : hmask;
 #pragma unroll
   for (int off = 1; off < 16; off <<= 1) {
     const float2 o = make_float2(__shfl_xor_sync(mask, v.x, off), __shfl_xor_sync(mask, v.y, off));
@@ -380,10 +404,15 @@ __device__ __forceinline__ float2 hsum16_tree2(float2 v, unsigned mask) {
   return v;
 }
 
-// NF4 nearest level: #{j : x > mid[j]}.  Bucket round(32 x + 32) holds at most
-// one threshold; the table has 128 entries so any 7-bit index stays inside.
+// NF4 nearest level: #{j : x > mid[j]}.  bucket_sum = fma(x, 256, kMagic +
+// 256) has the bit pattern of kMagic plus r = round(256 x + 256), r in
+// [0, 512] for |x| <= 1 + 2^-23, so r & 0x3F8 = 8 floor(r/8) is directly the
+// byte offset of bucket floor(r/8) in a table of 8-byte entries.  A bucket is
+// 1/32 wide in x and holds at most one threshold; the table has 128 entries,
+// so any 10-bit offset stays inside (entries past 64 read "above all").
 __device__ __forceinline__ uint32_t nf4_rtn_bucket(float x, float bucket_sum, const float2* rtn) {
-  const float2 e = rtn[__float_as_uint(bucket_sum) & 127u];
+  const float2 e = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(rtn) +
+                                                    (__float_as_uint(bucket_sum) & 0x3F8u));
   return (uint32_t)(__float_as_int(e.y) + (x > e.x ? 1 : 0));
 }
 
@@ -429,16 +458,30 @@ static __device__ __align__(16) SmemTables g_code_tables[2];
 template <bool FULL, bool FLAT, bool U32>
 __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
                                                  const float2 (&nv)[kPerLane / 2],
-                                                 const float2 (&ndv)[kPerLane / 2],
-                                                 const uint32_t (&rw)[kPerLane], float ninv,
-                                                 float R, int myn) {
+                                                 const float2 (&ndv)[kPerLane / 2], uint64_t quad,
+                                                 uint32_t c3, float ninv, float R, int myn) {
   // two values at a time; from the last pair to the first, so that element i
-  // ends in bits 4i..4i+3
+  // ends in bits 4i..4i+3.  The draws of values 4..7 come from the second
+  // Philox call (counter quad + 1), of 0..3 from the first, each made just
+  // before its pairs so that only four words are live.
   uint32_t vco = 0;
+  uint32_t rw[kPerLane];
+  if (U32) {   // (the binary64 decision keeps all eight words: fewer live doubles)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const uint4 r = philox4x32_10(quad + c, c3, a);
+      rw[4 * c + 0] = r.x; rw[4 * c + 1] = r.y; rw[4 * c + 2] = r.z; rw[4 * c + 3] = r.w;
+    }
+  }
 #pragma unroll
   for (int j = kPerLane / 2 - 1; j >= 0; --j) {
+    if (!U32 && (j == 3 || j == 1)) {
+      const uint4 r = philox4x32_10(quad + (j >> 1), c3, a);
+      rw[4 * (j >> 1) + 0] = r.x; rw[4 * (j >> 1) + 1] = r.y;
+      rw[4 * (j >> 1) + 2] = r.z; rw[4 * (j >> 1) + 3] = r.w;
+    }
     const float2 x2 = __fmul2_rn(nv[j], f2(ninv));                  // v1 / s
-    const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
+    const float2 t2 = __ffma2_rn(x2, a.k_15, a.k_magic);
     // k0, the nearest integer to 15x, is the bracket or one above it (the top
     // entry's threshold is +inf: its bracket is always 14)
     const uint32_t k0a = __float_as_uint(t2.x) & 15u, k0b = __float_as_uint(t2.y) & 15u;
@@ -447,10 +490,10 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
     // square roots of the lower and upper code points of each value
     const float2 sa = make_float2(deca ? ea.y : ea.z, decb ? eb.y : eb.z);
     const float2 sb = make_float2(deca ? ea.z : ea.w, decb ? eb.z : eb.w);
-    const float2 da = __ffma2_rn(sa, f2(R), f2(a.eps));
-    const float2 db = __ffma2_rn(sb, f2(R), f2(a.eps));
+    const float2 da = __ffma2_rn(sa, f2(R), a.p_eps);
+    const float2 db = __ffma2_rn(sb, f2(R), a.p_eps);
     // fma(y, -1, x) rounds like x - y; nB = -(db - da) dv, rhs = (db - dv) da
-    const float2 nB = __fmul2_rn(__ffma2_rn(da, f2(-1.0f), db), ndv[j]);
+    const float2 nB = __fmul2_rn(__ffma2_rn(da, a.k_m1, db), ndv[j]);
     const float2 rhs = __fmul2_rn(__fadd2_rn(db, ndv[j]), da);
     bool lowa, lowb;
     if (U32) {
@@ -459,7 +502,7 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
       lowb = __dmul_rn((double)rw[2 * j + 1], -(double)nB.y * 0x1p-32) < (double)rhs.y;
     } else {
       // u * B < rhs, with -(u * B) = u * nB rounded once
-      const float2 nlhs = __fmul2_rn(uniform32x2(rw[2 * j], rw[2 * j + 1]), nB);
+      const float2 nlhs = __fmul2_rn(uniform32x2(rw[2 * j], rw[2 * j + 1], a.k_2m32), nB);
       lowa = -nlhs.x < rhs.x;
       lowb = -nlhs.y < rhs.y;
     }
@@ -491,8 +534,8 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
 // binary32 integers in [1, 16]: cm + (kMagic - 1) is exact, and its bit
 // pattern is kMagic's (low byte 0) plus k.  The low byte of the result holds
 // k of the first value in bits 0-3 and of the second in bits 4-7.
-__device__ __forceinline__ uint32_t ze_code_pair(float2 cm) {
-  const float2 kb = __fadd2_rn(cm, f2(kMagic - 1.0f));
+__device__ __forceinline__ uint32_t ze_code_pair(float2 cm, float2 magic_m1) {
+  const float2 kb = __fadd2_rn(cm, magic_m1);                // magic_m1 = kMagic - 1
   return __float_as_uint(kb.x) + 16u * __float_as_uint(kb.y);
 }
 
@@ -518,27 +561,40 @@ __device__ __forceinline__ float block_rcp(float d) {
   return __fdiv_rn(1.0f, d);
 }
 
+// ZIP-SR's R = sqrt(s) rs_bc2 of a block scale s >= FLT_MIN.
+__device__ __forceinline__ float zipsr_block_R(const StepArgs& a, float av) {
+  const float rs = (av >= exact::kSqrtLo && av <= exact::kSqrtHi) ? exact::sqrt_rn(av)
+                                                                   : __fsqrt_rn(av);
+  return __fmul_rn(rs, a.rs_bc2);
+}
+// Whether R rules out two code points of a cell sharing one d value.
+__device__ __forceinline__ bool zipsr_not_flat(const StepArgs& a, float R) {
+  return R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN;
+}
+
 // Requantises one block held by a half-warp: m1 and nv = -v1 in pairs, ndv =
-// -d(v1) (ZIP-SR), lam / lav = the lane's largest |m1| and v1 (over its valid
-// values).  Writes this lane's code words and, from lane 0, the two scales.
-template <int VCODE, bool FULL>
+// -d(v1) (ZIP-SR), am / av = the block's largest |m1| and v1.  Writes this
+// lane's code words and, from lane 0, the two scales.
+// FAST: the caller has established that am and av lie inside the fast
+// sequences' ranges (every |m1| and v1 of the block passed the lanes' range
+// checks), that the LM head's stochastic phase does not apply, and for ZIP-SR
+// that R = sqrt(av) rs_bc2 (given) rules out flat cells; the code then has no
+// branches.  Otherwise each of those is tested here.
+template <int VCODE, bool FULL, bool FULLW, bool FAST>
 __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTables& S,
                                               uint32_t tensor_id, uint32_t flags, uint64_t e0,
                                               int lane, int myn, unsigned hmask,
                                               const float2 (&m1)[kPerLane / 2],
                                               const float2 (&nv)[kPerLane / 2],
-                                              const float2 (&ndv)[kPerLane / 2], float lam,
-                                              float lav, uint32_t* mcw, uint32_t* vcw, float* msp,
-                                              float* vsp) {
-  const float am = hmax16_nonneg(lam, hmask);
-  const float av = hmax16_nonneg(lav, hmask);
-
+                                              const float2 (&ndv)[kPerLane / 2], float am,
+                                              float av, float R_fast, uint32_t* mcw, uint32_t* vcw,
+                                              float* msp, float* vsp) {
   // ---- first moment: absmax scale, NF4 codes ----
   uint32_t mco = 0;
   float mso = 0.0f;
-  if (am >= FLT_MIN) {
-    const float inv = block_rcp(am);
-    if ((flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
+  if (FAST || am >= FLT_MIN) {
+    const float inv = FAST ? exact::rcp_rn(am) : block_rcp(am);
+    if (!FAST && (flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
       uint32_t rw[kPerLane];
       words8(a, tensor_id, kStreamM, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
 #pragma unroll
@@ -549,7 +605,7 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
 #pragma unroll
       for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
         const float2 x = __fmul2_rn(m1[j], f2(inv));
-        const float2 b = __ffma2_rn(x, f2(32.0f), f2(kMagic + 32.0f));
+        const float2 b = __ffma2_rn(x, a.k_256, a.k_magic256);
         const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? nf4_rtn_bucket(x.y, b.y, S.rtn) : 0u;
         const uint32_t c0 = (FULL || 2 * j < myn) ? nf4_rtn_bucket(x.x, b.x, S.rtn) : 0u;
         mco = (mco * 16u + c1) * 16u + c0;
@@ -561,24 +617,65 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   // ---- second moment ----
   uint32_t vco = 0;
   float vso = 0.0f;
-  if (av >= FLT_MIN) {
+  if (VCODE == kVZe) {
+    // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
+    // code point, scale times ||x||^2 / max(<x,Q(x)>, 1e-12 s^2) on x = v/s.
+    // The codes and sums are formed for every block, so that the sums'
+    // shuffles run with both half-warps together; an all-zero block (s below
+    // FLT_MIN) then stores zeros.
+    const bool von = FAST || av >= FLT_MIN;
     // -1/s: x = v1/s is then nv * ninv, the same binary32 product
-    const float ninv = -block_rcp(av);
+    const float ninv = FAST ? -exact::rcp_rn(av) : (von ? -block_rcp(av) : 0.0f);
+    float2 l1[kPerLane / 2];
+    uint32_t P[kPerLane / 2];
+#pragma unroll
+    for (int j = 0; j < kPerLane / 2; ++j) {
+      const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
+      const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
+      const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
+      const float2 cm = make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f));   // k + 1
+      const float2 q2 = __fmul2_rn(cm, a.k_1_16);                // (k+1)/16
+      P[j] = ze_code_pair(cm, a.k_magicm1);
+      float2 xx = __fmul2_rn(x2, x2);
+      float2 xq = __fmul2_rn(x2, q2);
+      if (!FULL) {
+        if (2 * j >= myn) { xx.x = 0.0f; xq.x = 0.0f; }
+        if (2 * j + 1 >= myn) { xx.y = 0.0f; xq.y = 0.0f; }
+      }
+      // first tree level: (x0^2 + x1^2, x0 q0 + x1 q1), two scalar adds whose
+      // results form the pair (cheaper than regrouping the operands)
+      l1[j] = make_float2(__fadd_rn(xx.x, xx.y), __fadd_rn(xq.x, xq.y));
+    }
+    const float2 l2a = __fadd2_rn(l1[0], l1[1]);
+    const float2 l2b = __fadd2_rn(l1[2], l1[3]);
+    const float2 s = hsum16_tree2<FULLW>(__fadd2_rn(l2a, l2b), hmask);   // (sum x^2, sum x q)
+    if (von) {
+      vco = pack_code_pairs(P, FULL ? kPerLane : myn);
+      const float den = fmaxf(s.y, 1e-12f);
+      // s.x >= 1 - 2^-22 (the block's largest x rounds to 1) and den <= 129:
+      // the fast quotient's range holds unless the inputs were not finite
+      // (then both forms give a NaN scale)
+      const float c = (FAST || (s.x >= 0x1p-60f && s.x <= 0x1p60f && den <= 0x1p60f))
+                          ? exact::div_rn(s.x, den)
+                          : __fdiv_rn(s.x, den);
+      vso = __fmul_rn(av, c);
+    }
+  } else if (FAST || av >= FLT_MIN) {
+    // -1/s: x = v1/s is then nv * ninv, the same binary32 product
+    const float ninv = FAST ? -exact::rcp_rn(av) : -block_rcp(av);
     if (VCODE == kVZip || VCODE == kVZip32) {
       // ZIP-SR ("ZIP-SR / ZE-EDEN", Core equation): keep the lower code point
       // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
       // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
-      const float rs = (av >= exact::kSqrtLo && av <= exact::kSqrtHi) ? exact::sqrt_rn(av)
-                                                                       : __fsqrt_rn(av);
-      const float R = __fmul_rn(rs, a.rs_bc2);
-      uint32_t rw[kPerLane];
-      words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
+      const float R = FAST ? R_fast : zipsr_block_R(a, av);
+      const uint64_t quad = (e0 + (uint64_t)(lane * kPerLane)) >> 2;   // Philox counter
+      const uint32_t c3 = tensor_id * 2u + kStreamV;
       // d(a) == d(b) needs (sqrt(k+1/15) - sqrt(k/15)) R below two ulps of
       // R + eps; the smallest gap is 0.0339, so R > 1e-5 eps rules it out.
-      if (R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN)
-        vco = zipsr_codes8<FULL, false, VCODE == kVZip32>(a, S, nv, ndv, rw, ninv, R, myn);
+      if (FAST || zipsr_not_flat(a, R))
+        vco = zipsr_codes8<FULL, false, VCODE == kVZip32>(a, S, nv, ndv, quad, c3, ninv, R, myn);
       else
-        vco = zipsr_codes8<FULL, true, VCODE == kVZip32>(a, S, nv, ndv, rw, ninv, R, myn);
+        vco = zipsr_codes8<FULL, true, VCODE == kVZip32>(a, S, nv, ndv, quad, c3, ninv, R, myn);
       vso = av;
     } else if (VCODE == kVZiRtn || VCODE == kVZiSr) {
       // State-space rules on the zero-inclusive code: nearest code point, or
@@ -588,7 +685,7 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
 #pragma unroll
       for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
         const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
-        const float2 t2 = __ffma2_rn(x2, f2(15.0f), f2(kMagic));
+        const float2 t2 = __ffma2_rn(x2, a.k_15, a.k_magic);
 #pragma unroll
         for (int h = 1; h >= 0; --h) {
           const int i = 2 * j + h;
@@ -613,45 +710,12 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
 #pragma unroll
       for (int j = 0; j < kPerLane / 2; ++j) {
         const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
-        const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
-        const float2 c2 = __fadd2_rn(t2, f2(-kMagic));             // rint(16x), exact
-        P[j] = ze_code_pair(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)));
+        const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
+        const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
+        P[j] = ze_code_pair(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)), a.k_magicm1);
       }
       vco = pack_code_pairs(P, FULL ? kPerLane : myn);
       vso = av;
-    } else {
-      // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
-      // code point, scale times ||x||^2 / max(<x,Q(x)>, 1e-12 s^2) on x = v/s.
-      float2 l1[kPerLane / 2];
-      uint32_t P[kPerLane / 2];
-#pragma unroll
-      for (int j = 0; j < kPerLane / 2; ++j) {
-        const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
-        const float2 t2 = __ffma2_rn(x2, f2(16.0f), f2(kMagic));   // kMagic + rint(16x)
-        const float2 c2 = __fadd2_rn(t2, f2(-kMagic));             // rint(16x), exact
-        const float2 cm = make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f));   // k + 1
-        const float2 q2 = __fmul2_rn(cm, f2(0.0625f));             // (k+1)/16
-        P[j] = ze_code_pair(cm);
-        float2 xx = __fmul2_rn(x2, x2);
-        float2 xq = __fmul2_rn(x2, q2);
-        if (!FULL) {
-          if (2 * j >= myn) { xx.x = 0.0f; xq.x = 0.0f; }
-          if (2 * j + 1 >= myn) { xx.y = 0.0f; xq.y = 0.0f; }
-        }
-        // first tree level: (x0^2 + x1^2, x0 q0 + x1 q1)
-        l1[j] = __fadd2_rn(make_float2(xx.x, xq.x), make_float2(xx.y, xq.y));
-      }
-      vco = pack_code_pairs(P, FULL ? kPerLane : myn);
-      const float2 l2a = __fadd2_rn(l1[0], l1[1]);
-      const float2 l2b = __fadd2_rn(l1[2], l1[3]);
-      const float2 s = hsum16_tree2(__fadd2_rn(l2a, l2b), hmask);    // (sum x^2, sum x q)
-      const float den = fmaxf(s.y, 1e-12f);
-      // s.x >= 1 - 2^-22 (the block's largest x rounds to 1) and den <= 129:
-      // the fast quotient's range holds unless the inputs were not finite
-      const float c = (s.x >= 0x1p-60f && s.x <= 0x1p60f && den <= 0x1p60f)
-                          ? exact::div_rn(s.x, den)
-                          : __fdiv_rn(s.x, den);
-      vso = __fmul_rn(av, c);
     }
   }
 
@@ -663,38 +727,99 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   }
 }
 
-// Decode + moment update + weight update for 8 values of a 4-bit block
-// ("ZIP-SR / ZE-EDEN", Method flowchart: decode the prior moments, update
-// them, update the weights -- with the unquantised moments, Core equation).
-// Out: m1 and nv = -v1 in pairs, ndv = -d(v1) = -(sqrt(v1) rs_bc2 + eps) in
-// pairs (KEEP_DV), lam / lav = the lane's largest |m1| and v1 over its valid
-// values, and nfacc += 0 * w (NaN once an updated weight is not finite).
-// A lane whose |m1| and v1 all lie in the fast ranges takes the square root
-// and the division from exact_math.cuh (the IEEE results, without branches);
-// any other lane, and every ragged block (FULL false: `myn` valid values),
-// calls the IEEE operations per value.
-template <bool FULL, bool KEEP_DV>
-__device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, float decay,
-                                        float (&w)[kPerLane], const float (&g)[kPerLane],
-                                        uint32_t mc, uint32_t vc, float sm, float sv, int myn,
-                                        float2 (&m1)[kPerLane / 2], float2 (&nv)[kPerLane / 2],
-                                        float2 (&ndv)[kPerLane / 2], float& lam, float& lav,
-                                        float2& nfacc) {
+// Decode and moment update for 8 values of a 4-bit block ("ZIP-SR / ZE-EDEN",
+// Method flowchart: decode the prior moments, update them).  Out: m1 and
+// nv = -v1 in pairs.
+__device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
+                                         const float (&g)[kPerLane], uint32_t mc, uint32_t vc,
+                                         float2 sm, float2 sv, float2 (&m1)[kPerLane / 2],
+                                         float2 (&nv)[kPerLane / 2]) {
 #pragma unroll
   for (int j = 0; j < kPerLane / 2; ++j) {
     // one byte holds the codes of values 2j (low nibble) and 2j+1 (high nibble)
-    const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], f2(sm));
-    const float2 v0 = __fmul2_rn(S.vpair[__byte_perm(vc, 0, 0x4440 + j)], f2(sv));
+    const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], sm);
+    const float2 v0 = __fmul2_rn(S.vpair[__byte_perm(vc, 0, 0x4440 + j)], sv);
     const float2 gg = make_float2(g[2 * j], g[2 * j + 1]);
-    m1[j] = __ffma2_rn(f2(a.b1), m0, __fmul2_rn(f2(a.omb1), gg));
+    m1[j] = __ffma2_rn(a.p_b1, m0, __fmul2_rn(a.p_omb1, gg));
     // -v1 = fma(-b2, v0, -(1-b2) g^2), the negation of the canonical v1 exactly
-    nv[j] = __ffma2_rn(f2(a.nb2), v0, __fmul2_rn(f2(a.nomb2), __fmul2_rn(gg, gg)));
+    nv[j] = __ffma2_rn(a.p_nb2, v0, __fmul2_rn(a.p_nomb2, __fmul2_rn(gg, gg)));
   }
-  bool fast;
+}
+
+// Whether a lane's eight |m1| and v1 all lie in the fast sequences' ranges
+// (also true of the block scales then: am in [2^-60, 2^100], av in
+// [2^-100, 2^64]).  lam / lav: the lane's largest |m1| and v1.
+__device__ __forceinline__ bool lane_in_range(const StepArgs& a, const float2 (&m1)[kPerLane / 2],
+                                              const float2 (&nv)[kPerLane / 2], float lam,
+                                              float lav) {
+  return absmin8(m1) >= a.m_lo && lam <= a.m_hi && absmin8(nv) >= a.v_lo && lav <= a.v_hi;
+}
+
+// Weight update of 8 values from their working moments ("ZIP-SR / ZE-EDEN",
+// Core equation: the weights use the unquantised moments): the square root
+// and the division from exact_math.cuh (operands in range), in pairs.
+// Out: ndv = -d(v1) (KEEP_DV), nfacc += 0 * w.
+template <bool KEEP_DV>
+__device__ __forceinline__ void weights8_fast(const StepArgs& a, float decay, float (&w)[kPerLane],
+                                              const float2 (&m1)[kPerLane / 2],
+                                              const float2 (&nv)[kPerLane / 2],
+                                              float2 (&ndv)[kPerLane / 2], float2& nfacc) {
+#pragma unroll
+  for (int j = 0; j < kPerLane / 2; ++j) {
+    const float2 ns = exact::neg_sqrt2_rn(nv[j], a.k_half);         // -sqrt(v1)
+    const float2 nd = __ffma2_rn(ns, a.p_rs, a.p_neps);             // -(sqrt(v1) rs + eps)
+    const float2 q = exact::div2_rn_neg(m1[j], nd, a.k_one);        // m1 / den
+    const float2 ww = __ffma2_rn(a.p_nstep, q,
+                                 __fmul2_rn(make_float2(w[2 * j], w[2 * j + 1]), f2(decay)));
+    if (KEEP_DV) ndv[j] = nd;
+    w[2 * j] = ww.x;
+    w[2 * j + 1] = ww.y;
+    nfacc = __ffma2_rn(ww, a.k_zero, nfacc);
+  }
+}
+
+// The same with the IEEE operations, value by value (FULL false: the first
+// `myn` values only).
+template <bool FULL, bool KEEP_DV>
+__device__ __forceinline__ void weights8_ieee(const StepArgs& a, float decay, float (&w)[kPerLane],
+                                              const float2 (&m1)[kPerLane / 2],
+                                              const float2 (&nv)[kPerLane / 2],
+                                              float2 (&ndv)[kPerLane / 2], int myn,
+                                              float2& nfacc) {
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    if (FULL || i < myn) {
+      const float v1 = -el(nv, i);
+      const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
+      const float wi = __fmaf_rn(a.nstep, __fdiv_rn(el(m1, i), den), __fmul_rn(w[i], decay));
+      w[i] = wi;
+      if (KEEP_DV) {
+        if (i & 1) ndv[i >> 1].y = -den;
+        else ndv[i >> 1].x = -den;
+      }
+      nfacc.x = __fmaf_rn(wi, 0.0f, nfacc.x);
+    }
+  }
+}
+
+// Decode + moment update + weight update for 8 values of a 4-bit block, each
+// lane choosing the fast sequences when its values are in range (see
+// weights8_fast).  Out: m1, nv, ndv as above, lam / lav = the lane's largest
+// |m1| and v1 over its valid values.  Ragged blocks (FULL false: `myn` valid
+// values) take the IEEE operations.
+template <bool FULL, bool KEEP_DV>
+__device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, float decay,
+                                        float (&w)[kPerLane], const float (&g)[kPerLane],
+                                        uint32_t mc, uint32_t vc, float2 sm, float2 sv, int myn,
+                                        float2 (&m1)[kPerLane / 2], float2 (&nv)[kPerLane / 2],
+                                        float2 (&ndv)[kPerLane / 2], float& lam, float& lav,
+                                        float2& nfacc) {
+  moments8(a, S, g, mc, vc, sm, sv, m1, nv);
   if (FULL) {
     lam = absmax8(m1);
     lav = absmax8(nv);
-    fast = absmin8(m1) >= a.m_lo && lam <= a.m_hi && absmin8(nv) >= a.v_lo && lav <= a.v_hi;
+    if (lane_in_range(a, m1, nv, lam, lav)) weights8_fast<KEEP_DV>(a, decay, w, m1, nv, ndv, nfacc);
+    else weights8_ieee<true, KEEP_DV>(a, decay, w, m1, nv, ndv, kPerLane, nfacc);
   } else {
     lam = 0.0f;
     lav = 0.0f;
@@ -707,36 +832,7 @@ __device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, 
         lav = fmaxf(lav, fabsf(el(nv, i)));
       }
     }
-    fast = false;
-  }
-  if (fast) {
-#pragma unroll
-    for (int j = 0; j < kPerLane / 2; ++j) {
-      const float2 ns = exact::neg_sqrt2_rn(nv[j]);                   // -sqrt(v1)
-      const float2 nd = __ffma2_rn(ns, f2(a.rs_bc2), f2(a.neps));     // -(sqrt(v1) rs + eps)
-      const float2 q = exact::div2_rn_neg(m1[j], nd);                 // m1 / den
-      const float2 ww = __ffma2_rn(f2(a.nstep), q,
-                                   __fmul2_rn(make_float2(w[2 * j], w[2 * j + 1]), f2(decay)));
-      if (KEEP_DV) ndv[j] = nd;
-      w[2 * j] = ww.x;
-      w[2 * j + 1] = ww.y;
-      nfacc = __ffma2_rn(ww, f2(0.0f), nfacc);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i) {
-      if (FULL || i < myn) {
-        const float v1 = -el(nv, i);
-        const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
-        const float wi = __fmaf_rn(a.nstep, __fdiv_rn(el(m1, i), den), __fmul_rn(w[i], decay));
-        w[i] = wi;
-        if (KEEP_DV) {
-          if (i & 1) ndv[i >> 1].y = -den;
-          else ndv[i >> 1].x = -den;
-        }
-        nfacc.x = __fmaf_rn(wi, 0.0f, nfacc.x);
-      }
-    }
+    weights8_ieee<false, KEEP_DV>(a, decay, w, m1, nv, ndv, myn, nfacc);
   }
 }
 
@@ -798,13 +894,15 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
   constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
   float2 m1[kPerLane / 2], nv[kPerLane / 2], ndv[kPerLane / 2];
   float lam, lav;
-  update8<false, kKeepDv>(a, S, decay, w, g, *mcw, *vcw, *msp, *vsp, myn, m1, nv, ndv, lam, lav,
-                          nfacc);
+  update8<false, kKeepDv>(a, S, decay, w, g, *mcw, *vcw, f2(*msp), f2(*vsp), myn, m1, nv, ndv, lam,
+                          lav, nfacc);
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i)
     if (i < myn) store_w<BF16W>(wp, wp16, wbf, i, w[i]);
-  requant_store<VCODE, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask, m1, nv,
-                              ndv, lam, lav, mcw, vcw, msp, vsp);
+  const float am = hmax16<false>(lam, hmask);
+  const float av = hmax16<false>(lav, hmask);
+  requant_store<VCODE, false, false, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask,
+                                            m1, nv, ndv, am, av, 0.0f, mcw, vcw, msp, vsp);
 }
 
 // ---------------------------------------------------------------------------
@@ -941,8 +1039,10 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     }
     if (staged && !a.fault_stall) {
       const int64_t blk = t_soff + ub;
-      cp_async4(dst + kOffMS + lane * 4, st.mscale + blk);
-      cp_async4(dst + kOffVS + lane * 4, st.vscale + blk);
+      cp_async4(dst + kOffMS + lane * 8, st.mscale + blk);
+      cp_async4(dst + kOffMS + lane * 8 + 4, st.mscale + blk);
+      cp_async4(dst + kOffVS + lane * 8, st.vscale + blk);
+      cp_async4(dst + kOffVS + lane * 8 + 4, st.vscale + blk);
     }
     cp_async_arrive_noinc(full);            // one arrival per lane, when its copies land
     // (test hook: with the stall armed no bulk copy is issued, so the expected
@@ -953,6 +1053,94 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     }
   }
   cp_async_wait_all();
+}
+
+// Stores a lane's eight updated weights of a whole block (16-byte stores):
+// fp32, or (wbf) bf16 rounded to nearest even.
+template <bool BF16W>
+__device__ __forceinline__ void store_w8(float* w0, bool wbf, int lane, const float (&w)[kPerLane]) {
+  if (BF16W && wbf) {
+    uint16_t* wp = reinterpret_cast<uint16_t*>(w0) + lane * kPerLane;
+    *reinterpret_cast<uint4*>(wp) = make_uint4(bf16x2_rn(w[0], w[1]), bf16x2_rn(w[2], w[3]),
+                                               bf16x2_rn(w[4], w[5]), bf16x2_rn(w[6], w[7]));
+  } else {
+    float* wp = w0 + lane * kPerLane;
+    *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// A whole 4-bit block whose data is in the stage, held by half-warp `half`.
+// FULLW: both half-warps of the warp take this path together (see hmax16).
+// Then, when every lane of both blocks has its moments inside the fast
+// ranges (and neither block is an LM head in its stochastic phase, nor, for
+// ZIP-SR, flat), the two blocks run one branch-free sequence; a warp that
+// does not qualify takes the general sequence, with its per-lane and
+// per-block range tests.
+template <int VCODE, bool BF16W, bool FULLW>
+__device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTables& S,
+                                               const StateArena& st, const uint8_t* sp,
+                                               const UnitHeader* hdp, uint32_t flags, int half,
+                                               int lane, unsigned hmask, float2& nfacc) {
+  constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
+  constexpr bool kZip = (VCODE == kVZip || VCODE == kVZip32);
+  float w[kPerLane], g[kPerLane];
+  const bool wbf = BF16W && (flags & kBf16W);
+  {
+    const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
+    if (wbf) {
+      const uint4 wr = *reinterpret_cast<const uint4*>(sp + (hdp->nv_soff >> 8) + lane * 16);
+      w[0] = bf16lo(wr.x); w[1] = bf16hi(wr.x); w[2] = bf16lo(wr.y); w[3] = bf16hi(wr.y);
+      w[4] = bf16lo(wr.z); w[5] = bf16hi(wr.z); w[6] = bf16lo(wr.w); w[7] = bf16hi(wr.w);
+    } else {
+      const uint8_t* wsrc = sp + kOffW + half * 512 + lane * 32;
+      const float4 wa = *reinterpret_cast<const float4*>(wsrc);
+      const float4 wb = *reinterpret_cast<const float4*>(wsrc + 16);
+      w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
+      w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
+    }
+    g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
+    g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
+  }
+  const uint32_t mc = *reinterpret_cast<const uint32_t*>(sp + kOffMC + half * 64 + lane * 4);
+  const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + half * 64 + lane * 4);
+  const float2 sm = *reinterpret_cast<const float2*>(sp + kOffMS + half * 8);
+  const float2 sv = *reinterpret_cast<const float2*>(sp + kOffVS + half * 8);
+  const float decay = hdp->decay;
+
+  float2 m1[kPerLane / 2], nv[kPerLane / 2], ndv[kPerLane / 2];
+  moments8(a, S, g, mc, vc, sm, sv, m1, nv);
+  const float lam = absmax8(m1);
+  const float lav = absmax8(nv);
+  const float am = hmax16<FULLW>(lam, hmask);
+  const float av = hmax16<FULLW>(lav, hmask);
+  const bool lane_fast = lane_in_range(a, m1, nv, lam, lav);
+  bool warp_fast = false;
+  float R = 0.0f;
+  if (FULLW) {
+    bool ok = lane_fast && !((flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active);
+    if (kZip) {
+      R = __fmul_rn(exact::sqrt_rn(av), a.rs_bc2);   // av in range whenever `ok` holds
+      ok = ok && zipsr_not_flat(a, R);
+    }
+    warp_fast = __all_sync(kFullMask, ok);
+  }
+  float* msp = hdp->ms;
+  if (warp_fast) {
+    weights8_fast<kKeepDv>(a, decay, w, m1, nv, ndv, nfacc);
+    store_w8<BF16W>(hdp->w, wbf, lane, w);
+    requant_store<VCODE, true, FULLW, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, kPerLane,
+                                            hmask, m1, nv, ndv, am, av, R, hdp->mc + lane,
+                                            hdp->vc + lane, msp, msp + st.vs_minus_ms);
+  } else {
+    if (lane_fast) weights8_fast<kKeepDv>(a, decay, w, m1, nv, ndv, nfacc);
+    else weights8_ieee<true, kKeepDv>(a, decay, w, m1, nv, ndv, kPerLane, nfacc);
+    store_w8<BF16W>(hdp->w, wbf, lane, w);
+    requant_store<VCODE, true, FULLW, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane,
+                                             kPerLane, hmask, m1, nv, ndv, am, av, 0.0f,
+                                             hdp->mc + lane, hdp->vc + lane, msp,
+                                             msp + st.vs_minus_ms);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -999,68 +1187,32 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
   const int half = threadIdx.x >> 4;
   const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
   const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
-  constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
   int s = 0;
   uint32_t parity = 0;
   float2 nfacc = make_float2(0.0f, 0.0f);   // NaN once an updated weight is not finite
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const uint32_t full = full0 + 8u * s;
     const uint32_t empty = empty0 + 8u * s;
-    if (!__all_sync(hmask, wait_phase(full, parity, kWaitLimitNs))) {
-      if (lane == 0) atomicOr(a.status, 1u);
+    if (!__all_sync(kFullMask, wait_phase(full, parity, kWaitLimitNs))) {
+      if ((threadIdx.x & 31) == 0) atomicOr(a.status, 1u);
       return;
     }
     const uint8_t* sp = s_stage + s * kStageBytes;
     const UnitHeader* hdp = reinterpret_cast<const UnitHeader*>(sp + kOffHdr) + half;
     const uint32_t flags = hdp->flags;
-    if (flags & kStaged) {
-      float w[kPerLane], g[kPerLane];
-      const bool wbf = BF16W && (flags & kBf16W);
-      {
-        const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
-        if (wbf) {
-          const uint4 wr = *reinterpret_cast<const uint4*>(sp + (hdp->nv_soff >> 8) + lane * 16);
-          w[0] = bf16lo(wr.x); w[1] = bf16hi(wr.x); w[2] = bf16lo(wr.y); w[3] = bf16hi(wr.y);
-          w[4] = bf16lo(wr.z); w[5] = bf16hi(wr.z); w[6] = bf16lo(wr.w); w[7] = bf16hi(wr.w);
-        } else {
-          const uint8_t* wsrc = sp + kOffW + half * 512 + lane * 32;
-          const float4 wa = *reinterpret_cast<const float4*>(wsrc);
-          const float4 wb = *reinterpret_cast<const float4*>(wsrc + 16);
-          w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
-          w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
-        }
-        g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
-        g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
-      }
-      const uint32_t mc = *reinterpret_cast<const uint32_t*>(sp + kOffMC + half * 64 + lane * 4);
-      const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + half * 64 + lane * 4);
-      const float sm = *reinterpret_cast<const float*>(sp + kOffMS + half * 4);
-      const float sv = *reinterpret_cast<const float*>(sp + kOffVS + half * 4);
-
-      float2 m1[kPerLane / 2], nv[kPerLane / 2], ndv[kPerLane / 2];
-      float lam, lav;
-      update8<true, kKeepDv>(a, S, hdp->decay, w, g, mc, vc, sm, sv, kPerLane, m1, nv, ndv, lam,
-                             lav, nfacc);
-      if (wbf) {
-        uint16_t* wp = reinterpret_cast<uint16_t*>(hdp->w) + lane * kPerLane;
-        *reinterpret_cast<uint4*>(wp) = make_uint4(bf16x2_rn(w[0], w[1]), bf16x2_rn(w[2], w[3]),
-                                                   bf16x2_rn(w[4], w[5]), bf16x2_rn(w[6], w[7]));
-      } else {
-        float* wp = hdp->w + lane * kPerLane;
-        *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
-      }
-      float* msp = hdp->ms;
-      requant_store<VCODE, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, kPerLane, hmask, m1,
-                                 nv, ndv, lam, lav, hdp->mc + lane, hdp->vc + lane, msp,
-                                 msp + st.vs_minus_ms);
+    const bool staged = (flags & kStaged) != 0;
+    if (__all_sync(kFullMask, staged)) {          // both half-warps hold whole blocks
+      process_staged<VCODE, BF16W, true>(a, S, st, sp, hdp, flags, half, lane, hmask, nfacc);
+    } else if (staged) {
+      process_staged<VCODE, BF16W, false>(a, S, st, sp, hdp, flags, half, lane, hmask, nfacc);
     } else if (!(flags & kNoUnit)) {
       process_direct<VCODE, BF16W>(a, S, st, hdp, lane, hmask, nfacc);
     }
-    // every read of the stage (header included) is done: hand it back
+    // every read of the stage (header included) is done: hand it back, one
+    // arrival per half-warp (both of the warp's, from its lane 0)
     fence_proxy_async_smem();
-    __syncwarp(hmask);
-    if (lane == 0) mbar_arrive(empty, 1);
+    __syncwarp(kFullMask);
+    if ((threadIdx.x & 31) == 0) mbar_arrive(empty, 2);
     if (++s == kStages) {
       s = 0;
       parity ^= 1u;
