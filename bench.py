@@ -624,9 +624,36 @@ def run_sweep(args):
     torch.cuda.set_device(0)
     B.lib()
     names = [args.vcode] if args.no_companion else ["zipsr", "zeeden"]
+    sweep_floor(args)
     for name in names:
         sweep_one(args, B, name)
     return 0
+
+
+def sweep_floor(args):
+    """The timing floor of the sweep's method: the same flush and event
+    bracket around a one-element fill (one tiny library kernel), so that the
+    step's fixed cost per launch can be read as the part above this."""
+    import torch
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
+    tiny = torch.empty(1, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        tiny.fill_(0.0)
+    times = []
+    for _ in range(max(args.steps // 10, 5)):
+        flush.fill_(1.0)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        tiny.fill_(2.0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    print(json.dumps({"sweep": "floor", "what": "one-element fill, same flush and event bracket",
+                      "us": float(np.median(times)) * 1e3,
+                      "us_p10": float(np.percentile(times, 10)) * 1e3,
+                      "us_p90": float(np.percentile(times, 90)) * 1e3}), flush=True)
 
 
 def sweep_one(args, B, name):

@@ -435,7 +435,7 @@ void launch_vcode(int vcode, bool bf16w, int grid, cudaStream_t s, const DevTens
 // One launch over units [u0, u1) of the handle's list.
 int launch(adamw4_handle* h, StepArgs a, cudaStream_t s, int64_t u0, int64_t u1) {
   if (u1 <= u0) return ADAMW4_OK;
-  const int64_t need = (u1 - u0 + kHalves - 1) / kHalves;
+  const int64_t need = (u1 - u0 + kTileUnits - 1) / kTileUnits;
   const int grid = (int)std::min<int64_t>(h->grid, need);
   a.status = h->d_status;
   a.fault_stall = h->fault_stall;
@@ -929,7 +929,7 @@ extern "C" int adamw4_tensor_state_kind(const adamw4_tensor* t) {
 
 extern "C" int adamw4_launch_info(const adamw4_handle* h, int* grid, int* block, int64_t* units) {
   if (!live(h)) return fail(nullptr, ADAMW4_EINVAL, "unknown or destroyed handle");
-  const int64_t need = (h->nunits + kHalves - 1) / kHalves;
+  const int64_t need = (h->nunits + kTileUnits - 1) / kTileUnits;
   if (grid) *grid = (int)std::min<int64_t>(h->grid, need);
   if (block) *block = kCtaThreads;
   if (units) *units = h->nunits;
@@ -1080,7 +1080,7 @@ extern "C" int adamw4_step_noalloc(const adamw4_config* cfg, const adamw4_tensor
   st.nblocks4 = blocks4;
   st.n32 = elems32;
   st.vs_minus_ms = st.vscale - st.mscale;
-  const int64_t need = (unit + kHalves - 1) / kHalves;
+  const int64_t need = (unit + kTileUnits - 1) / kTileUnits;
   launch_vcode(cfg->vcode, bf16w, (int)std::min<int64_t>(nd.grid[cfg->vcode][bf16w], need), s,
                table, 0, unit, a, st);
   return cudaGetLastError() == cudaSuccess ? ADAMW4_OK : ADAMW4_ECUDA;

@@ -6,23 +6,25 @@
 // One kernel launch covers a range of units of a flat unit list: each block
 // of a 4-bit tensor is one unit, and each fp32-state tensor is cut into
 // 128-element chunks.  The grid is persistent (SM count x resident CTAs) and
-// tiles of 16 consecutive units are dealt out round-robin, so all SMs stream
+// tiles of 28 consecutive units are dealt out round-robin, so all SMs stream
 // one contiguous window of HBM.
 //
-// A CTA has one producer warp and eight consumer warps (sixteen half-warps),
-// and a ring of kStages CTA-wide stages, one tile each.  For every unit of a
-// tile, producer lane i writes a 64-byte header (addresses, block index, tensor
-// id, flags, decay) into the stage; for runs of whole 4-bit blocks of one
-// tensor the first lane of the run fills the stage with TMA bulk copies
-// (cp.async.bulk: the run's fp32 or bf16 weights, bf16 grads and codes) and
-// every lane copies its two block scales with 4-byte cp.async, all completing
-// on the stage's "full" mbarrier.  Consumer half-warp i waits on it, computes
-// unit i from the stage, stores the results straight to global memory and
-// hands the stage back on its "empty" mbarrier.  Units that are not whole
-// 4-bit blocks (a ragged last block, fp32-state chunks) carry only the header
-// and are read from global memory by their half-warp.  Every wait is bounded
-// by a timer; on expiry the kernel records the failure in a status word and
-// the waiting warp leaves (the producer after draining its copies).
+// A CTA has one producer warp and seven consumer warps, and a ring of kStages
+// CTA-wide stages, one tile each.  Eight lanes take one unit, sixteen values
+// per lane (two groups of eight, 64 values apart), so a warp takes four units
+// and the CTA's 28 slots one tile.  For every unit of a tile, producer lane i
+// writes a 64-byte header (addresses, block index, tensor id, flags, decay)
+// into the stage; for runs of whole 4-bit blocks of one tensor the first lane
+// of the run fills the stage with TMA bulk copies (cp.async.bulk: the run's
+// fp32 or bf16 weights, bf16 grads and codes) and every lane copies its two
+// block scales with 4-byte cp.async, all completing on the stage's "full"
+// mbarrier.  The consumer lanes of slot i wait on it, compute unit i from the
+// stage, store the results straight to global memory and hand the stage back
+// on its "empty" mbarrier.  Units that are not whole 4-bit blocks (a ragged
+// last block, fp32-state chunks) carry only the header and are read from
+// global memory by their lanes.  Every wait is bounded by a timer; on expiry
+// the kernel records the failure in a status word and the waiting warp
+// leaves (the producer after draining its copies).
 //
 // Per unit, following the method flowchart of "ZIP-SR / ZE-EDEN: 4-bit AdamW
 // state quantization" (daiwk.github.io, Method): decode the prior moments,
@@ -54,25 +56,39 @@
 namespace {
 
 constexpr int kBlock = ADAMW4_BLOCK;              // values per quantisation block
-constexpr int kLanesPerUnit = 16;                 // a half-warp per block
-constexpr int kPerLane = kBlock / kLanesPerUnit;  // 8 values per lane
-constexpr int kConsumerThreads = 256;             // eight consumer warps
+// A lane holds kSub groups of kGroup consecutive values of one block, the
+// groups kBlock / kSub values apart: lane l of a block's kLanesPerUnit lanes
+// takes values [64 s + 8 l, 64 s + 8 l + 8) for s = 0, 1.  A group is one
+// 32-bit code word and two Philox calls.
+constexpr int kGroup = 8;
+constexpr int kSub = 2;
+constexpr int kLanesPerUnit = kBlock / (kGroup * kSub);   // 8 lanes per block
+constexpr int kUnitsPerWarp = 32 / kLanesPerUnit;         // 4 blocks per warp
+constexpr int kConsumerWarps = 7;
+constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kCtaThreads = kConsumerThreads + 32;  // plus the producer warp
-constexpr int kHalves = kConsumerThreads / kLanesPerUnit;  // consumer half-warps per CTA
-constexpr int kProducerWarp = kConsumerThreads / 32;
+constexpr int kTileUnits = kConsumerThreads / kLanesPerUnit;  // units per tile: 28
+constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kStages = 3;                        // tiles in flight per CTA
-// A tile is kHalves consecutive units; stage layout (CTA-wide):
-//   16 unit headers (64 B each) | w 16 x 512 B | g 16 x 256 B |
-//   m codes 16 x 64 B | v codes 16 x 64 B | m scales 16 x 8 B | v scales 16 x 8 B
+// Two CTAs of eight warps per SM: four warps per SM sub-partition, whose
+// 16,384-register file then gives each thread up to 128 registers.
+constexpr int kMinCtasPerSm = 2;
+static_assert(kGroup * kSub * kLanesPerUnit == kBlock, "lane layout");
+static_assert(kTileUnits <= 32, "one producer lane per unit");
+// Value offset of group s of lane l within its block.
+__host__ __device__ constexpr int group_off(int s, int l) { return s * (kBlock / kSub) + l * kGroup; }
+// A tile is kTileUnits consecutive units; stage layout (CTA-wide):
+//   unit headers (64 B each) | w 512 B each | g 256 B each |
+//   m codes 64 B each | v codes 64 B each | m scales 8 B each | v scales 8 B each
 // (each scale twice, as the pair the f32x2 decode multiplies by)
 constexpr int kOffHdr = 0;
-constexpr int kOffW = kOffHdr + kHalves * 64;
-constexpr int kOffG = kOffW + kHalves * 512;
-constexpr int kOffMC = kOffG + kHalves * 256;
-constexpr int kOffVC = kOffMC + kHalves * 64;
-constexpr int kOffMS = kOffVC + kHalves * 64;
-constexpr int kOffVS = kOffMS + kHalves * 8;
-constexpr int kStageBytes = kOffVS + kHalves * 8; // 15,616 B, a 16-byte multiple
+constexpr int kOffW = kOffHdr + kTileUnits * 64;
+constexpr int kOffG = kOffW + kTileUnits * 512;
+constexpr int kOffMC = kOffG + kTileUnits * 256;
+constexpr int kOffVC = kOffMC + kTileUnits * 64;
+constexpr int kOffMS = kOffVC + kTileUnits * 64;
+constexpr int kOffVS = kOffMS + kTileUnits * 8;
+constexpr int kStageBytes = kOffVS + kTileUnits * 8; // 27,328 B, a 16-byte multiple
 constexpr uint32_t kUnitTx = 896;                 // bulk-copied bytes of one whole block
 constexpr int kSmemStages = kStages * kStageBytes;
 static_assert(kStageBytes % 16 == 0, "stage alignment");
@@ -166,7 +182,7 @@ struct StateArena {
 
 // What the producer tells the consumer about one unit (64 bytes).
 // The addresses are formed by the producer (one lane per unit) so that the
-// consumers' sixteen lanes do not each recompute them.
+// consumers' eight lanes do not each recompute them.
 struct __align__(16) UnitHeader {
   float* w;              // the unit's first weight (fp32, or bf16 bit patterns)
   uint32_t* mc;          // 4-bit: the block's m code words; fp32 state: its first m
@@ -352,16 +368,22 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
   asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
-// Largest and smallest |x| over a lane's eight values (four pairs).
-__device__ __forceinline__ float absmax8(const float2 (&x)[4]) {
-  const float r = max3f(fabsf(x[0].x), fabsf(x[0].y), fabsf(x[1].x));
-  const float q = max3f(r, fabsf(x[1].y), fabsf(x[2].x));
-  return max3f(q, fabsf(x[2].y), fmaxf(fabsf(x[3].x), fabsf(x[3].y)));
+// Largest and smallest |x| over a lane's values (kSub groups of four pairs).
+__device__ __forceinline__ float absmax_lane(const float2 (&x)[kSub][4]) {
+  float r = fmaxf(fabsf(x[0][0].x), fabsf(x[0][0].y));
+#pragma unroll
+  for (int s = 0; s < kSub; ++s)
+#pragma unroll
+    for (int j = (s == 0 ? 1 : 0); j < 4; ++j) r = max3f(r, fabsf(x[s][j].x), fabsf(x[s][j].y));
+  return r;
 }
-__device__ __forceinline__ float absmin8(const float2 (&x)[4]) {
-  const float r = min3f(fabsf(x[0].x), fabsf(x[0].y), fabsf(x[1].x));
-  const float q = min3f(r, fabsf(x[1].y), fabsf(x[2].x));
-  return min3f(q, fabsf(x[2].y), fminf(fabsf(x[3].x), fabsf(x[3].y)));
+__device__ __forceinline__ float absmin_lane(const float2 (&x)[kSub][4]) {
+  float r = fminf(fabsf(x[0][0].x), fabsf(x[0][0].y));
+#pragma unroll
+  for (int s = 0; s < kSub; ++s)
+#pragma unroll
+    for (int j = (s == 0 ? 1 : 0); j < 4; ++j) r = min3f(r, fabsf(x[s][j].x), fabsf(x[s][j].y));
+  return r;
 }
 
 // The ZIP-SR uniforms of two draw words: each word rounded to the nearest
@@ -370,38 +392,47 @@ __device__ __forceinline__ float2 uniform32x2(uint32_t w0, uint32_t w1, float2 k
   return __fmul2_rn(make_float2(__uint2float_rn(w0), __uint2float_rn(w1)), k2m32);
 }
 
-// Collectives over a half-warp.  FULLW: both half-warps of the warp execute
-// the call together, so it runs with the constant full-warp mask (no
-// convergence bookkeeping around it); else with the half-warp's own mask.
+// Collectives over the kLanesPerUnit lanes of one block.  FULLW: all lanes
+// of the warp execute the call together (every block of the warp takes the
+// same path), so it runs with the constant full-warp mask and no convergence
+// bookkeeping around it; else with the block's own lane mask `gmask`.
 constexpr unsigned kFullMask = 0xFFFFFFFFu;
 
-// Max of non-negative binary32 values over a half-warp: their bit patterns
-// order like the values, so an integer reduction gives the exact maximum.
-// Full-warp form: one reduction per half, the other half contributing 0.
+// Max of non-negative binary32 values over a block's lanes: their bit
+// patterns order like the values, so an integer maximum is the exact one.
 template <bool FULLW>
-__device__ __forceinline__ float hmax16(float v, unsigned hmask) {
-  const uint32_t b = __float_as_uint(v);
+__device__ __forceinline__ float unit_max(float v, unsigned gmask) {
+  uint32_t b = __float_as_uint(v);
   if (FULLW) {
-    const bool hi = (threadIdx.x & 16) != 0;
-    const uint32_t mlo = __reduce_max_sync(kFullMask, hi ? 0u : b);
-    const uint32_t mhi = __reduce_max_sync(kFullMask, hi ? b : 0u);
-    return __uint_as_float(hi ? mhi : mlo);
+#pragma unroll
+    for (int off = 1; off < kLanesPerUnit; off <<= 1) b = max(b, __shfl_xor_sync(kFullMask, b, off));
+    return __uint_as_float(b);
   }
-  return __uint_as_float(__reduce_max_sync(hmask, b));
+  return __uint_as_float(__reduce_max_sync(gmask, b));
 }
 
-// Balanced pairwise sum of (x, y) pairs over the half-warp: partner offsets 1,
-// 2, 4, 8 join adjacent 8-value groups in index order (IEEE addition is
-// commutative, so both partners hold the same bits).
+// Balanced pairwise sum of (x, y) pairs over a block, from each lane's
+// per-group sums: partner offsets 1, 2, 4 join adjacent groups in index order
+// within each half of the block, and the two halves (a lane's two groups)
+// are joined last.  IEEE addition is commutative, so partners hold the same
+// bits.
 template <bool FULLW>
-__device__ __forceinline__ float2 hsum16_tree2(float2 v, unsigned hmask) {
-  const unsigned mask = FULLW ? kFullMask : hmask;
+__device__ __forceinline__ float2 unit_sum_tree2(const float2 (&v)[kSub], unsigned gmask) {
+  const unsigned mask = FULLW ? kFullMask : gmask;
+  float2 t[kSub];
 #pragma unroll
-  for (int off = 1; off < 16; off <<= 1) {
-    const float2 o = make_float2(__shfl_xor_sync(mask, v.x, off), __shfl_xor_sync(mask, v.y, off));
-    v = __fadd2_rn(v, o);
+  for (int s = 0; s < kSub; ++s) t[s] = v[s];
+#pragma unroll
+  for (int off = 1; off < kLanesPerUnit; off <<= 1) {
+#pragma unroll
+    for (int s = 0; s < kSub; ++s) {
+      const float2 o = make_float2(__shfl_xor_sync(mask, t[s].x, off),
+                                   __shfl_xor_sync(mask, t[s].y, off));
+      t[s] = __fadd2_rn(t[s], o);
+    }
   }
-  return v;
+  static_assert(kSub == 2, "the last level joins two halves");
+  return __fadd2_rn(t[0], t[1]);
 }
 
 // NF4 nearest level: #{j : x > mid[j]}.  bucket_sum = fma(x, 256, kMagic +
@@ -446,26 +477,28 @@ static_assert(sizeof(SmemTables) % 16 == 0, "tables are copied in 16-byte pieces
 static __device__ __align__(16) SmemTables g_code_tables[2];
 
 // ---------------------------------------------------------------------------
-// Requantisation of one 4-bit block held by a half-warp (8 values per lane).
-// FULL: all 128 values valid.  Otherwise `myn` values of this lane are valid.
+// Requantisation of one 4-bit block held by kLanesPerUnit lanes (kSub groups
+// of 8 values per lane).  FULL: all 128 values valid.  Otherwise myn[s]
+// values of group s of this lane are valid.
 // ---------------------------------------------------------------------------
 
-// ZIP-SR codes of 8 values, from nv = -v1 and ndv = -d(v1) (d = 1/h, the
-// update's denominator) in pairs, and ninv = -1/s of the block.  FLAT: also
-// test for d(a) == d(b), which needs the state-space fallback; callers skip
-// it when the block's R makes that impossible.  U32: the binary64 decision of
-// v code 5; else the binary32 one with the whole-word uniform.
+// ZIP-SR codes of one group of 8 values, from nv = -v1 and ndv = -d(v1)
+// (d = 1/h, the update's denominator) in pairs, and ninv = -1/s of the block.
+// FLAT: also test for d(a) == d(b), which needs the state-space fallback;
+// callers skip it when the block's R makes that impossible.  U32: the
+// binary64 decision of v code 5; else the binary32 one with the whole-word
+// uniform.
 template <bool FULL, bool FLAT, bool U32>
 __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
-                                                 const float2 (&nv)[kPerLane / 2],
-                                                 const float2 (&ndv)[kPerLane / 2], uint64_t quad,
-                                                 uint32_t c3, float ninv, float R, int myn) {
+                                                 const float2 (&nv)[4], const float2 (&ndv)[4],
+                                                 uint64_t quad, uint32_t c3, float ninv, float R,
+                                                 int myn) {
   // two values at a time; from the last pair to the first, so that element i
   // ends in bits 4i..4i+3.  The draws of values 4..7 come from the second
   // Philox call (counter quad + 1), of 0..3 from the first, each made just
   // before its pairs so that only four words are live.
   uint32_t vco = 0;
-  uint32_t rw[kPerLane];
+  uint32_t rw[kGroup];
   if (U32) {   // (the binary64 decision keeps all eight words: fewer live doubles)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
@@ -474,7 +507,7 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
     }
   }
 #pragma unroll
-  for (int j = kPerLane / 2 - 1; j >= 0; --j) {
+  for (int j = kGroup / 2 - 1; j >= 0; --j) {
     if (!U32 && (j == 3 || j == 1)) {
       const uint4 r = philox4x32_10(quad + (j >> 1), c3, a);
       rw[4 * (j >> 1) + 0] = r.x; rw[4 * (j >> 1) + 1] = r.y;
@@ -542,20 +575,19 @@ __device__ __forceinline__ uint32_t ze_code_pair(float2 cm, float2 magic_m1) {
 // The low bytes of four code pairs as one 32-bit word of eight nibbles
 // (value i in bits 4i..4i+3), with the nibbles of values at or past `nvalid`
 // cleared.
-__device__ __forceinline__ uint32_t pack_code_pairs(const uint32_t (&P)[kPerLane / 2],
-                                                    int nvalid) {
+__device__ __forceinline__ uint32_t pack_code_pairs(const uint32_t (&P)[4], int nvalid) {
   const uint32_t w = __byte_perm(__byte_perm(P[0], P[1], 0x0040), __byte_perm(P[2], P[3], 0x0040),
                                  0x5410);
-  return nvalid >= kPerLane ? w : w & ((1u << (4 * nvalid)) - 1u);
+  return nvalid >= kGroup ? w : w & ((1u << (4 * nvalid)) - 1u);
 }
 
-// Value i of a lane's eight, held as four pairs.
-__device__ __forceinline__ float el(const float2 (&x)[kPerLane / 2], int i) {
+// Value i of a group of eight, held as four pairs.
+__device__ __forceinline__ float el(const float2 (&x)[4], int i) {
   return (i & 1) ? x[i >> 1].y : x[i >> 1].x;
 }
 
 // RN(1/d) for a block scale d >= FLT_MIN: the fast sequence inside its range,
-// else the IEEE division (the branch is uniform over the half-warp).
+// else the IEEE division (the branch is uniform over the block's lanes).
 __device__ __forceinline__ float block_rcp(float d) {
   if (d >= exact::kRcpLo && d <= exact::kRcpHi) return exact::rcp_rn(d);
   return __fdiv_rn(1.0f, d);
@@ -572,9 +604,10 @@ __device__ __forceinline__ bool zipsr_not_flat(const StepArgs& a, float R) {
   return R > __fmul_rn(1e-5f, a.eps) && a.eps >= FLT_MIN;
 }
 
-// Requantises one block held by a half-warp: m1 and nv = -v1 in pairs, ndv =
-// -d(v1) (ZIP-SR), am / av = the block's largest |m1| and v1.  Writes this
-// lane's code words and, from lane 0, the two scales.
+// Requantises one block: m1 and nv = -v1 in pairs, ndv = -d(v1) (ZIP-SR),
+// am / av = the block's largest |m1| and v1.  Writes this lane's code words
+// (group s: word s * kLanesPerUnit + lane of the block's sixteen, from mcb /
+// vcb) and, from lane 0, the two scales.
 // FAST: the caller has established that am and av lie inside the fast
 // sequences' ranges (every |m1| and v1 of the block passed the lanes' range
 // checks), that the LM head's stochastic phase does not apply, and for ZIP-SR
@@ -583,81 +616,96 @@ __device__ __forceinline__ bool zipsr_not_flat(const StepArgs& a, float R) {
 template <int VCODE, bool FULL, bool FULLW, bool FAST>
 __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTables& S,
                                               uint32_t tensor_id, uint32_t flags, uint64_t e0,
-                                              int lane, int myn, unsigned hmask,
-                                              const float2 (&m1)[kPerLane / 2],
-                                              const float2 (&nv)[kPerLane / 2],
-                                              const float2 (&ndv)[kPerLane / 2], float am,
-                                              float av, float R_fast, uint32_t* mcw, uint32_t* vcw,
+                                              int lane, const int (&myn)[kSub], unsigned gmask,
+                                              const float2 (&m1)[kSub][4],
+                                              const float2 (&nv)[kSub][4],
+                                              const float2 (&ndv)[kSub][4], float am, float av,
+                                              float R_fast, uint32_t* mcb, uint32_t* vcb,
                                               float* msp, float* vsp) {
   // ---- first moment: absmax scale, NF4 codes ----
-  uint32_t mco = 0;
+  uint32_t mco[kSub];
+#pragma unroll
+  for (int s = 0; s < kSub; ++s) mco[s] = 0;
   float mso = 0.0f;
   if (FAST || am >= FLT_MIN) {
     const float inv = FAST ? exact::rcp_rn(am) : block_rcp(am);
     if (!FAST && (flags & ADAMW4_T_LM_HEAD) && a.lm_sr_active) {
-      uint32_t rw[kPerLane];
-      words8(a, tensor_id, kStreamM, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
 #pragma unroll
-      for (int i = 0; i < kPerLane; ++i)
-        if (FULL || i < myn)
-          mco |= nf4_sr(__fmul_rn(el(m1, i), inv), uniform23(rw[i]), S.nf4, S.gap) << (4 * i);
+      for (int s = 0; s < kSub; ++s) {
+        uint32_t rw[kGroup];
+        words8(a, tensor_id, kStreamM, (e0 + (uint64_t)group_off(s, lane)) >> 2, rw);
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i)
+          if (FULL || i < myn[s])
+            mco[s] |= nf4_sr(__fmul_rn(el(m1[s], i), inv), uniform23(rw[i]), S.nf4, S.gap)
+                      << (4 * i);
+      }
     } else {
 #pragma unroll
-      for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
-        const float2 x = __fmul2_rn(m1[j], f2(inv));
-        const float2 b = __ffma2_rn(x, a.k_256, a.k_magic256);
-        const uint32_t c1 = (FULL || 2 * j + 1 < myn) ? nf4_rtn_bucket(x.y, b.y, S.rtn) : 0u;
-        const uint32_t c0 = (FULL || 2 * j < myn) ? nf4_rtn_bucket(x.x, b.x, S.rtn) : 0u;
-        mco = (mco * 16u + c1) * 16u + c0;
+      for (int s = 0; s < kSub; ++s) {
+#pragma unroll
+        for (int j = kGroup / 2 - 1; j >= 0; --j) {   // last element first
+          const float2 x = __fmul2_rn(m1[s][j], f2(inv));
+          const float2 b = __ffma2_rn(x, a.k_256, a.k_magic256);
+          const uint32_t c1 = (FULL || 2 * j + 1 < myn[s]) ? nf4_rtn_bucket(x.y, b.y, S.rtn) : 0u;
+          const uint32_t c0 = (FULL || 2 * j < myn[s]) ? nf4_rtn_bucket(x.x, b.x, S.rtn) : 0u;
+          mco[s] = (mco[s] * 16u + c1) * 16u + c0;
+        }
       }
     }
     mso = am;
   }
 
   // ---- second moment ----
-  uint32_t vco = 0;
+  uint32_t vco[kSub];
+#pragma unroll
+  for (int s = 0; s < kSub; ++s) vco[s] = 0;
   float vso = 0.0f;
   if (VCODE == kVZe) {
     // ZE-EDEN ("ZIP-SR / ZE-EDEN", Core equation): nearest zero-excluded
     // code point, scale times ||x||^2 / max(<x,Q(x)>, 1e-12 s^2) on x = v/s.
     // The codes and sums are formed for every block, so that the sums'
-    // shuffles run with both half-warps together; an all-zero block (s below
-    // FLT_MIN) then stores zeros.
+    // shuffles run with all the warp's blocks together; an all-zero block
+    // (s below FLT_MIN) then stores zeros.
     const bool von = FAST || av >= FLT_MIN;
     // -1/s: x = v1/s is then nv * ninv, the same binary32 product
     const float ninv = FAST ? -exact::rcp_rn(av) : (von ? -block_rcp(av) : 0.0f);
-    float2 l1[kPerLane / 2];
-    uint32_t P[kPerLane / 2];
+    uint32_t P[kSub][4];
+    float2 gsum[kSub];
 #pragma unroll
-    for (int j = 0; j < kPerLane / 2; ++j) {
-      const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
-      const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
-      const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
-      const float2 cm = make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f));   // k + 1
-      const float2 q2 = __fmul2_rn(cm, a.k_1_16);                // (k+1)/16
-      P[j] = ze_code_pair(cm, a.k_magicm1);
-      float2 xx = __fmul2_rn(x2, x2);
-      float2 xq = __fmul2_rn(x2, q2);
-      if (!FULL) {
-        if (2 * j >= myn) { xx.x = 0.0f; xq.x = 0.0f; }
-        if (2 * j + 1 >= myn) { xx.y = 0.0f; xq.y = 0.0f; }
+    for (int s = 0; s < kSub; ++s) {
+      float2 l1[4];
+#pragma unroll
+      for (int j = 0; j < kGroup / 2; ++j) {
+        const float2 x2 = __fmul2_rn(nv[s][j], f2(ninv));
+        const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
+        const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
+        const float2 cm = make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f));   // k + 1
+        const float2 q2 = __fmul2_rn(cm, a.k_1_16);                // (k+1)/16
+        P[s][j] = ze_code_pair(cm, a.k_magicm1);
+        float2 xx = __fmul2_rn(x2, x2);
+        float2 xq = __fmul2_rn(x2, q2);
+        if (!FULL) {
+          if (2 * j >= myn[s]) { xx.x = 0.0f; xq.x = 0.0f; }
+          if (2 * j + 1 >= myn[s]) { xx.y = 0.0f; xq.y = 0.0f; }
+        }
+        // first tree level: (x0^2 + x1^2, x0 q0 + x1 q1), two scalar adds whose
+        // results form the pair (cheaper than regrouping the operands)
+        l1[j] = make_float2(__fadd_rn(xx.x, xx.y), __fadd_rn(xq.x, xq.y));
       }
-      // first tree level: (x0^2 + x1^2, x0 q0 + x1 q1), two scalar adds whose
-      // results form the pair (cheaper than regrouping the operands)
-      l1[j] = make_float2(__fadd_rn(xx.x, xx.y), __fadd_rn(xq.x, xq.y));
+      gsum[s] = __fadd2_rn(__fadd2_rn(l1[0], l1[1]), __fadd2_rn(l1[2], l1[3]));
     }
-    const float2 l2a = __fadd2_rn(l1[0], l1[1]);
-    const float2 l2b = __fadd2_rn(l1[2], l1[3]);
-    const float2 s = hsum16_tree2<FULLW>(__fadd2_rn(l2a, l2b), hmask);   // (sum x^2, sum x q)
+    const float2 t = unit_sum_tree2<FULLW>(gsum, gmask);   // (sum x^2, sum x q)
     if (von) {
-      vco = pack_code_pairs(P, FULL ? kPerLane : myn);
-      const float den = fmaxf(s.y, 1e-12f);
-      // s.x >= 1 - 2^-22 (the block's largest x rounds to 1) and den <= 129:
+#pragma unroll
+      for (int s = 0; s < kSub; ++s) vco[s] = pack_code_pairs(P[s], FULL ? kGroup : myn[s]);
+      const float den = fmaxf(t.y, 1e-12f);
+      // t.x >= 1 - 2^-22 (the block's largest x rounds to 1) and den <= 129:
       // the fast quotient's range holds unless the inputs were not finite
       // (then both forms give a NaN scale)
-      const float c = (FAST || (s.x >= 0x1p-60f && s.x <= 0x1p60f && den <= 0x1p60f))
-                          ? exact::div_rn(s.x, den)
-                          : __fdiv_rn(s.x, den);
+      const float c = (FAST || (t.x >= 0x1p-60f && t.x <= 0x1p60f && den <= 0x1p60f))
+                          ? exact::div_rn(t.x, den)
+                          : __fdiv_rn(t.x, den);
       vso = __fmul_rn(av, c);
     }
   } else if (FAST || av >= FLT_MIN) {
@@ -668,74 +716,90 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       // with probability [h(v)-h(b)]/[h(a)-h(b)], evaluated division-free as
       // u*((db-da)*dv) < (db-dv)*da with d = 1/h.
       const float R = FAST ? R_fast : zipsr_block_R(a, av);
-      const uint64_t quad = (e0 + (uint64_t)(lane * kPerLane)) >> 2;   // Philox counter
       const uint32_t c3 = tensor_id * 2u + kStreamV;
       // d(a) == d(b) needs (sqrt(k+1/15) - sqrt(k/15)) R below two ulps of
       // R + eps; the smallest gap is 0.0339, so R > 1e-5 eps rules it out.
-      if (FAST || zipsr_not_flat(a, R))
-        vco = zipsr_codes8<FULL, false, VCODE == kVZip32>(a, S, nv, ndv, quad, c3, ninv, R, myn);
-      else
-        vco = zipsr_codes8<FULL, true, VCODE == kVZip32>(a, S, nv, ndv, quad, c3, ninv, R, myn);
+      if (FAST || zipsr_not_flat(a, R)) {
+#pragma unroll
+        for (int s = 0; s < kSub; ++s)
+          vco[s] = zipsr_codes8<FULL, false, VCODE == kVZip32>(
+              a, S, nv[s], ndv[s], (e0 + (uint64_t)group_off(s, lane)) >> 2, c3, ninv, R, myn[s]);
+      } else {
+#pragma unroll
+        for (int s = 0; s < kSub; ++s)
+          vco[s] = zipsr_codes8<FULL, true, VCODE == kVZip32>(
+              a, S, nv[s], ndv[s], (e0 + (uint64_t)group_off(s, lane)) >> 2, c3, ninv, R, myn[s]);
+      }
       vso = av;
     } else if (VCODE == kVZiRtn || VCODE == kVZiSr) {
       // State-space rules on the zero-inclusive code: nearest code point, or
       // the lower one with probability (b - x)/(b - a).
-      uint32_t rw[kPerLane];
-      if (VCODE == kVZiSr) words8(a, tensor_id, kStreamV, (e0 + (uint64_t)(lane * kPerLane)) >> 2, rw);
 #pragma unroll
-      for (int j = kPerLane / 2 - 1; j >= 0; --j) {   // last element first
-        const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
-        const float2 t2 = __ffma2_rn(x2, a.k_15, a.k_magic);
+      for (int s = 0; s < kSub; ++s) {
+        uint32_t rw[kGroup];
+        if (VCODE == kVZiSr)
+          words8(a, tensor_id, kStreamV, (e0 + (uint64_t)group_off(s, lane)) >> 2, rw);
 #pragma unroll
-        for (int h = 1; h >= 0; --h) {
-          const int i = 2 * j + h;
-          const float x = h ? x2.y : x2.x;
-          const uint32_t k0 = __float_as_uint(h ? t2.y : t2.x) & 15u;
-          const uint32_t k = k0 - ((x < S.zip[k0].x) ? 1u : 0u);   // the bracket
-          uint32_t c;
-          if (VCODE == kVZiRtn) {
-            c = k + ((x > S.vzmid[k]) ? 1u : 0u);
-          } else {
-            const float2 z = S.vzp[k];
-            const bool lower = __fmul_rn(uniform23(rw[i]), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
-            c = k + (lower ? 0u : 1u);
+        for (int j = kGroup / 2 - 1; j >= 0; --j) {   // last element first
+          const float2 x2 = __fmul2_rn(nv[s][j], f2(ninv));
+          const float2 t2 = __ffma2_rn(x2, a.k_15, a.k_magic);
+#pragma unroll
+          for (int h = 1; h >= 0; --h) {
+            const int i = 2 * j + h;
+            const float x = h ? x2.y : x2.x;
+            const uint32_t k0 = __float_as_uint(h ? t2.y : t2.x) & 15u;
+            const uint32_t k = k0 - ((x < S.zip[k0].x) ? 1u : 0u);   // the bracket
+            uint32_t c;
+            if (VCODE == kVZiRtn) {
+              c = k + ((x > S.vzmid[k]) ? 1u : 0u);
+            } else {
+              const float2 z = S.vzp[k];
+              const bool lower =
+                  __fmul_rn(uniform23(rw[i]), __fsub_rn(z.y, z.x)) < __fsub_rn(z.y, x);
+              c = k + (lower ? 0u : 1u);
+            }
+            vco[s] = vco[s] * 16u + ((FULL || i < myn[s]) ? c : 0u);
           }
-          vco = vco * 16u + ((FULL || i < myn) ? c : 0u);
         }
       }
       vso = av;
     } else if (VCODE == kVZeFloor) {
       // Zero-excluded code with a positive floor: nearest (k+1)/16, no rescale.
-      uint32_t P[kPerLane / 2];
 #pragma unroll
-      for (int j = 0; j < kPerLane / 2; ++j) {
-        const float2 x2 = __fmul2_rn(nv[j], f2(ninv));
-        const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
-        const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
-        P[j] = ze_code_pair(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)), a.k_magicm1);
+      for (int s = 0; s < kSub; ++s) {
+        uint32_t P[4];
+#pragma unroll
+        for (int j = 0; j < kGroup / 2; ++j) {
+          const float2 x2 = __fmul2_rn(nv[s][j], f2(ninv));
+          const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
+          const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
+          P[j] = ze_code_pair(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)), a.k_magicm1);
+        }
+        vco[s] = pack_code_pairs(P, FULL ? kGroup : myn[s]);
       }
-      vco = pack_code_pairs(P, FULL ? kPerLane : myn);
       vso = av;
     }
   }
 
-  *mcw = mco;
-  *vcw = vco;
+#pragma unroll
+  for (int s = 0; s < kSub; ++s) {
+    mcb[s * kLanesPerUnit + lane] = mco[s];
+    vcb[s * kLanesPerUnit + lane] = vco[s];
+  }
   if (lane == 0) {
     *msp = mso;
     *vsp = vso;
   }
 }
 
-// Decode and moment update for 8 values of a 4-bit block ("ZIP-SR / ZE-EDEN",
-// Method flowchart: decode the prior moments, update them).  Out: m1 and
-// nv = -v1 in pairs.
+// Decode and moment update for one group of 8 values of a 4-bit block
+// ("ZIP-SR / ZE-EDEN", Method flowchart: decode the prior moments, update
+// them).  Out: m1 and nv = -v1 in pairs.
 __device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
-                                         const float (&g)[kPerLane], uint32_t mc, uint32_t vc,
-                                         float2 sm, float2 sv, float2 (&m1)[kPerLane / 2],
-                                         float2 (&nv)[kPerLane / 2]) {
+                                         const float (&g)[kGroup], uint32_t mc, uint32_t vc,
+                                         float2 sm, float2 sv, float2 (&m1)[4], float2 (&nv)[4]) {
 #pragma unroll
-  for (int j = 0; j < kPerLane / 2; ++j) {
+  for (int j = 0; j < kGroup / 2; ++j) {
     // one byte holds the codes of values 2j (low nibble) and 2j+1 (high nibble)
     const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], sm);
     const float2 v0 = __fmul2_rn(S.vpair[__byte_perm(vc, 0, 0x4440 + j)], sv);
@@ -746,26 +810,25 @@ __device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
   }
 }
 
-// Whether a lane's eight |m1| and v1 all lie in the fast sequences' ranges
-// (also true of the block scales then: am in [2^-60, 2^100], av in
-// [2^-100, 2^64]).  lam / lav: the lane's largest |m1| and v1.
-__device__ __forceinline__ bool lane_in_range(const StepArgs& a, const float2 (&m1)[kPerLane / 2],
-                                              const float2 (&nv)[kPerLane / 2], float lam,
-                                              float lav) {
-  return absmin8(m1) >= a.m_lo && lam <= a.m_hi && absmin8(nv) >= a.v_lo && lav <= a.v_hi;
+// Whether all a lane's |m1| and v1 lie in the fast sequences' ranges (also
+// true of the block scales then: am in [2^-60, 2^100], av in [2^-100, 2^64]).
+// lam / lav: the lane's largest |m1| and v1.
+__device__ __forceinline__ bool lane_in_range(const StepArgs& a, const float2 (&m1)[kSub][4],
+                                              const float2 (&nv)[kSub][4], float lam, float lav) {
+  return absmin_lane(m1) >= a.m_lo && lam <= a.m_hi && absmin_lane(nv) >= a.v_lo &&
+         lav <= a.v_hi;
 }
 
-// Weight update of 8 values from their working moments ("ZIP-SR / ZE-EDEN",
-// Core equation: the weights use the unquantised moments): the square root
-// and the division from exact_math.cuh (operands in range), in pairs.
-// Out: ndv = -d(v1) (KEEP_DV), nfacc += 0 * w.
+// Weight update of a group of 8 values from their working moments ("ZIP-SR /
+// ZE-EDEN", Core equation: the weights use the unquantised moments): the
+// square root and the division from exact_math.cuh (operands in range), in
+// pairs.  Out: ndv = -d(v1) (KEEP_DV), nfacc += 0 * w.
 template <bool KEEP_DV>
-__device__ __forceinline__ void weights8_fast(const StepArgs& a, float decay, float (&w)[kPerLane],
-                                              const float2 (&m1)[kPerLane / 2],
-                                              const float2 (&nv)[kPerLane / 2],
-                                              float2 (&ndv)[kPerLane / 2], float2& nfacc) {
+__device__ __forceinline__ void weights8_fast(const StepArgs& a, float decay, float (&w)[kGroup],
+                                              const float2 (&m1)[4], const float2 (&nv)[4],
+                                              float2 (&ndv)[4], float2& nfacc) {
 #pragma unroll
-  for (int j = 0; j < kPerLane / 2; ++j) {
+  for (int j = 0; j < kGroup / 2; ++j) {
     const float2 ns = exact::neg_sqrt2_rn(nv[j], a.k_half);         // -sqrt(v1)
     const float2 nd = __ffma2_rn(ns, a.p_rs, a.p_neps);             // -(sqrt(v1) rs + eps)
     const float2 q = exact::div2_rn_neg(m1[j], nd, a.k_one);        // m1 / den
@@ -781,13 +844,11 @@ __device__ __forceinline__ void weights8_fast(const StepArgs& a, float decay, fl
 // The same with the IEEE operations, value by value (FULL false: the first
 // `myn` values only).
 template <bool FULL, bool KEEP_DV>
-__device__ __forceinline__ void weights8_ieee(const StepArgs& a, float decay, float (&w)[kPerLane],
-                                              const float2 (&m1)[kPerLane / 2],
-                                              const float2 (&nv)[kPerLane / 2],
-                                              float2 (&ndv)[kPerLane / 2], int myn,
-                                              float2& nfacc) {
+__device__ __forceinline__ void weights8_ieee(const StepArgs& a, float decay, float (&w)[kGroup],
+                                              const float2 (&m1)[4], const float2 (&nv)[4],
+                                              float2 (&ndv)[4], int myn, float2& nfacc) {
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
+  for (int i = 0; i < kGroup; ++i) {
     if (FULL || i < myn) {
       const float v1 = -el(nv, i);
       const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
@@ -802,41 +863,7 @@ __device__ __forceinline__ void weights8_ieee(const StepArgs& a, float decay, fl
   }
 }
 
-// Decode + moment update + weight update for 8 values of a 4-bit block, each
-// lane choosing the fast sequences when its values are in range (see
-// weights8_fast).  Out: m1, nv, ndv as above, lam / lav = the lane's largest
-// |m1| and v1 over its valid values.  Ragged blocks (FULL false: `myn` valid
-// values) take the IEEE operations.
-template <bool FULL, bool KEEP_DV>
-__device__ __forceinline__ void update8(const StepArgs& a, const SmemTables& S, float decay,
-                                        float (&w)[kPerLane], const float (&g)[kPerLane],
-                                        uint32_t mc, uint32_t vc, float2 sm, float2 sv, int myn,
-                                        float2 (&m1)[kPerLane / 2], float2 (&nv)[kPerLane / 2],
-                                        float2 (&ndv)[kPerLane / 2], float& lam, float& lav,
-                                        float2& nfacc) {
-  moments8(a, S, g, mc, vc, sm, sv, m1, nv);
-  if (FULL) {
-    lam = absmax8(m1);
-    lav = absmax8(nv);
-    if (lane_in_range(a, m1, nv, lam, lav)) weights8_fast<KEEP_DV>(a, decay, w, m1, nv, ndv, nfacc);
-    else weights8_ieee<true, KEEP_DV>(a, decay, w, m1, nv, ndv, kPerLane, nfacc);
-  } else {
-    lam = 0.0f;
-    lav = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kPerLane / 2; ++j) ndv[j] = f2(-1.0f);   // (slots past myn)
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i) {
-      if (i < myn) {
-        lam = fmaxf(lam, fabsf(el(m1, i)));
-        lav = fmaxf(lav, fabsf(el(nv, i)));
-      }
-    }
-    weights8_ieee<false, KEEP_DV>(a, decay, w, m1, nv, ndv, myn, nfacc);
-  }
-}
-
-// Weight i of a lane's run, fp32 or (BF16W and flagged) bf16.
+// Weight i of a group, fp32 or (BF16W and flagged) bf16.
 template <bool BF16W>
 __device__ __forceinline__ float load_w(const float* wp, const uint16_t* wp16, bool wbf, int i) {
   if (BF16W && wbf) return __uint_as_float((uint32_t)wp16[i] << 16);
@@ -849,74 +876,114 @@ __device__ __forceinline__ void store_w(float* wp, uint16_t* wp16, bool wbf, int
 }
 
 // A unit read straight from global memory: a ragged last 4-bit block or a
-// chunk of an fp32-state tensor.
+// chunk of an fp32-state tensor.  Both take the IEEE operations value by
+// value.
 template <int VCODE, bool BF16W>
 __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTables& S,
-                                            const StateArena& st, const UnitHeader* hdp,
-                                            int lane, unsigned hmask, float2& nfacc) {
-  const int my0 = lane * kPerLane;
-  const int myn = min(max((int)(hdp->nv_soff & 255u) - my0, 0), kPerLane);
+                                               const StateArena& st, const UnitHeader* hdp,
+                                               int lane, unsigned gmask, float2& nfacc) {
+  const int nval = (int)(hdp->nv_soff & 255u);
   const uint32_t flags = hdp->flags;
   const bool wbf = BF16W && (flags & kBf16W);
   const float decay = hdp->decay;
-  // the header's w is the unit's first weight, of either width
-  float* wp = wbf ? nullptr : hdp->w + my0;
-  uint16_t* wp16 = wbf ? reinterpret_cast<uint16_t*>(hdp->w) + my0 : nullptr;
-  const uint16_t* gp = hdp->g + my0;
-  float w[kPerLane], g[kPerLane];
+  int myn[kSub];
+  float w[kSub][kGroup], g[kSub][kGroup];
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    w[i] = (i < myn) ? load_w<BF16W>(wp, wp16, wbf, i) : 0.0f;
-    g[i] = (i < myn) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
+  for (int s = 0; s < kSub; ++s) {
+    const int o = group_off(s, lane);
+    myn[s] = min(max(nval - o, 0), kGroup);
+    // the header's w is the unit's first weight, of either width
+    const float* wp = wbf ? nullptr : hdp->w + o;
+    const uint16_t* wp16 = wbf ? reinterpret_cast<const uint16_t*>(hdp->w) + o : nullptr;
+    const uint16_t* gp = hdp->g + o;
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i) {
+      w[s][i] = (i < myn[s]) ? load_w<BF16W>(wp, wp16, wbf, i) : 0.0f;
+      g[s][i] = (i < myn[s]) ? __uint_as_float((uint32_t)gp[i] << 16) : 0.0f;
+    }
   }
   if (flags & kKindFp32) {
-    float* mp = reinterpret_cast<float*>(hdp->mc) + my0;
-    float* vp = reinterpret_cast<float*>(hdp->vc) + my0;
 #pragma unroll
-    for (int i = 0; i < kPerLane; ++i) {
-      if (i < myn) {
-        const float m1 = __fmaf_rn(a.b1, mp[i], __fmul_rn(a.omb1, g[i]));
-        const float v1 = __fmaf_rn(a.b2, vp[i], __fmul_rn(a.omb2, __fmul_rn(g[i], g[i])));
-        const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
-        const float wi = __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[i], decay));
-        store_w<BF16W>(wp, wp16, wbf, i, wi);
-        nfacc.x = __fmaf_rn(wi, 0.0f, nfacc.x);
-        mp[i] = m1;
-        vp[i] = v1;
+    for (int s = 0; s < kSub; ++s) {
+      const int o = group_off(s, lane);
+      float* wp = wbf ? nullptr : hdp->w + o;
+      uint16_t* wp16 = wbf ? reinterpret_cast<uint16_t*>(hdp->w) + o : nullptr;
+      float* mp = reinterpret_cast<float*>(hdp->mc) + o;
+      float* vp = reinterpret_cast<float*>(hdp->vc) + o;
+#pragma unroll
+      for (int i = 0; i < kGroup; ++i) {
+        if (i < myn[s]) {
+          const float gi = g[s][i];
+          const float m1 = __fmaf_rn(a.b1, mp[i], __fmul_rn(a.omb1, gi));
+          const float v1 = __fmaf_rn(a.b2, vp[i], __fmul_rn(a.omb2, __fmul_rn(gi, gi)));
+          const float den = __fmaf_rn(__fsqrt_rn(v1), a.rs_bc2, a.eps);
+          const float wi = __fmaf_rn(-a.step_size, __fdiv_rn(m1, den), __fmul_rn(w[s][i], decay));
+          store_w<BF16W>(wp, wp16, wbf, i, wi);
+          nfacc.x = __fmaf_rn(wi, 0.0f, nfacc.x);
+          mp[i] = m1;
+          vp[i] = v1;
+        }
       }
     }
     return;
   }
-  uint32_t* mcw = hdp->mc + lane;
-  uint32_t* vcw = hdp->vc + lane;
+  // a ragged last block of a 4-bit tensor
+  constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
   float* msp = hdp->ms;
   float* vsp = msp + st.vs_minus_ms;
-  constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
-  float2 m1[kPerLane / 2], nv[kPerLane / 2], ndv[kPerLane / 2];
-  float lam, lav;
-  update8<false, kKeepDv>(a, S, decay, w, g, *mcw, *vcw, f2(*msp), f2(*vsp), myn, m1, nv, ndv, lam,
-                          lav, nfacc);
+  const float2 sm = f2(*msp), sv = f2(*vsp);
+  float2 m1[kSub][4], nv[kSub][4], ndv[kSub][4];
+  float lam = 0.0f, lav = 0.0f;
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i)
-    if (i < myn) store_w<BF16W>(wp, wp16, wbf, i, w[i]);
-  const float am = hmax16<false>(lam, hmask);
-  const float av = hmax16<false>(lav, hmask);
-  requant_store<VCODE, false, false, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, hmask,
-                                            m1, nv, ndv, am, av, 0.0f, mcw, vcw, msp, vsp);
+  for (int s = 0; s < kSub; ++s) {
+    moments8(a, S, g[s], hdp->mc[s * kLanesPerUnit + lane], hdp->vc[s * kLanesPerUnit + lane], sm,
+             sv, m1[s], nv[s]);
+#pragma unroll
+    for (int j = 0; j < kGroup / 2; ++j) ndv[s][j] = f2(-1.0f);   // (slots past myn)
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i) {
+      if (i < myn[s]) {
+        lam = fmaxf(lam, fabsf(el(m1[s], i)));
+        lav = fmaxf(lav, fabsf(el(nv[s], i)));
+      }
+    }
+    weights8_ieee<false, kKeepDv>(a, decay, w[s], m1[s], nv[s], ndv[s], myn[s], nfacc);
+    const int o = group_off(s, lane);
+    float* wp = wbf ? nullptr : hdp->w + o;
+    uint16_t* wp16 = wbf ? reinterpret_cast<uint16_t*>(hdp->w) + o : nullptr;
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i)
+      if (i < myn[s]) store_w<BF16W>(wp, wp16, wbf, i, w[s][i]);
+  }
+  const float am = unit_max<false>(lam, gmask);
+  const float av = unit_max<false>(lav, gmask);
+  requant_store<VCODE, false, false, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, myn, gmask,
+                                            m1, nv, ndv, am, av, 0.0f, hdp->mc, hdp->vc, msp, vsp);
+}
+
+// A tensor descriptor read with four 16-byte loads.
+__device__ __forceinline__ DevTensor load_tensor(const DevTensor* p) {
+  DevTensor d;
+  const uint4* src = reinterpret_cast<const uint4*>(p);
+  uint4* dst = reinterpret_cast<uint4*>(&d);
+#pragma unroll
+  for (int i = 0; i < (int)(sizeof(DevTensor) / 16); ++i) dst[i] = __ldg(src + i);
+  return d;
 }
 
 // ---------------------------------------------------------------------------
-// Producer: fills CTA-wide stages, one tile of kHalves consecutive units each.
-// Lane i handles unit i of the tile (header, scales); the lane that starts a
-// run of whole 4-bit blocks of one tensor issues that run's bulk copies.
+// Producer: fills CTA-wide stages, one tile of kTileUnits consecutive units
+// each.  Lane i handles unit i of the tile (header, scales); the lane that
+// starts a run of whole 4-bit blocks of one tensor issues that run's bulk
+// copies.
 // ---------------------------------------------------------------------------
 template <bool BF16W>
 __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t u_begin,
                                         int64_t u_end, const StepArgs& a, const StateArena& st,
                                         uint8_t* stages, uint32_t full0, uint32_t empty0,
                                         int lane) {
-  constexpr unsigned kMask = (1u << kHalves) - 1u;
-  const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
+  constexpr unsigned kMask = kTileUnits == 32 ? kFullMask : (1u << kTileUnits) - 1u;
+  const int64_t ntiles = (u_end - u_begin + kTileUnits - 1) / kTileUnits;
   int ti = -1;
   int64_t t_begin = 0, t_end = 0, t_numel = 0, t_soff = 0, t_eoff = 0;
   float* t_param = nullptr;
@@ -942,23 +1009,23 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
       cp_async_wait_all();
       return;
     }
-    const int64_t u = u_begin + tile * kHalves + lane;
+    const int64_t u = u_begin + tile * kTileUnits + lane;
     bool has = u < u_end;
     if (has && u >= t_end) {
+      DevTensor d;
       do {
-        ++ti;
-        t_end = __ldg(&T[ti].unit_end);
-      } while (u >= t_end);
-      const DevTensor* d = &T[ti];
-      t_begin = __ldg(&d->unit_begin);
-      t_numel = __ldg(&d->numel);
-      t_soff = __ldg(&d->state_off);
-      t_eoff = (int64_t)__ldg(&d->block_offset) * kBlock;
-      t_param = d->param;
-      t_grad = d->grad;
-      t_id = __ldg(&d->tensor_id);
-      t_flags = __ldg(&d->flags);
-      t_decay = (float)(1.0 - (double)a.lr * (double)__ldg(&d->weight_decay));
+        d = load_tensor(&T[++ti]);    // the whole descriptor in one round trip
+      } while (u >= d.unit_end);
+      t_end = d.unit_end;
+      t_begin = d.unit_begin;
+      t_numel = d.numel;
+      t_soff = d.state_off;
+      t_eoff = (int64_t)d.block_offset * kBlock;
+      t_param = d.param;
+      t_grad = d.grad;
+      t_id = d.tensor_id;
+      t_flags = d.flags;
+      t_decay = (float)(1.0 - (double)a.lr * (double)d.weight_decay);
     }
     const int64_t ub = u - t_begin;
     const int64_t e0 = ub * kBlock;
@@ -1012,7 +1079,8 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     if (BF16W) {
       // A run's weights land packed at the start of its own units' 512-B w
       // slots: 512 B per unit for fp32, 256 B for bf16.  The run starts at the
-      // nearest lane at or below this one that does not continue a run.
+      // nearest lane at or below this one that does not continue a run
+      // ((2 << 31) - 1 wraps to the full mask).
       const int start = 31 - __clz(~cont_mask & ((2u << lane) - 1u));
       w_soff = (uint32_t)(kOffW + start * 512 + (lane - start) * (wbf ? 256 : 512));
     }
@@ -1024,8 +1092,8 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
     if (lane == 0) mbar_arrive_expect_tx(full, tx);
     if (staged && !cont && !a.fault_stall) {
       // this lane starts a run: it extends over the following lanes whose
-      // unit continues it
-      const unsigned rest = ~(cont_mask >> (lane + 1));
+      // unit continues it (the shift is done in 64 bits: lane + 1 may be 32)
+      const unsigned rest = ~(uint32_t)((uint64_t)cont_mask >> (lane + 1));
       const int len = __ffs(rest);          // 1 + number of continuing lanes
       const int64_t blk = t_soff + ub;
       if (wbf)
@@ -1055,65 +1123,71 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
   cp_async_wait_all();
 }
 
-// Stores a lane's eight updated weights of a whole block (16-byte stores):
-// fp32, or (wbf) bf16 rounded to nearest even.
+// Stores one group of a lane's updated weights (value offset `off` in the
+// block; 16-byte stores): fp32, or (wbf) bf16 rounded to nearest even.
 template <bool BF16W>
-__device__ __forceinline__ void store_w8(float* w0, bool wbf, int lane, const float (&w)[kPerLane]) {
+__device__ __forceinline__ void store_w8(float* w0, bool wbf, int off, const float (&w)[kGroup]) {
   if (BF16W && wbf) {
-    uint16_t* wp = reinterpret_cast<uint16_t*>(w0) + lane * kPerLane;
+    uint16_t* wp = reinterpret_cast<uint16_t*>(w0) + off;
     *reinterpret_cast<uint4*>(wp) = make_uint4(bf16x2_rn(w[0], w[1]), bf16x2_rn(w[2], w[3]),
                                                bf16x2_rn(w[4], w[5]), bf16x2_rn(w[6], w[7]));
   } else {
-    float* wp = w0 + lane * kPerLane;
+    float* wp = w0 + off;
     *reinterpret_cast<float4*>(wp) = make_float4(w[0], w[1], w[2], w[3]);
     *reinterpret_cast<float4*>(wp + 4) = make_float4(w[4], w[5], w[6], w[7]);
   }
 }
 
-// A whole 4-bit block whose data is in the stage, held by half-warp `half`.
-// FULLW: both half-warps of the warp take this path together (see hmax16).
-// Then, when every lane of both blocks has its moments inside the fast
-// ranges (and neither block is an LM head in its stochastic phase, nor, for
-// ZIP-SR, flat), the two blocks run one branch-free sequence; a warp that
-// does not qualify takes the general sequence, with its per-lane and
-// per-block range tests.
+// A whole 4-bit block whose data is in the stage, slot `unit` of the tile.
+// FULLW: all the warp's blocks take this path together (see unit_max).  Then,
+// when every lane of every such block has its moments inside the fast ranges
+// (and no block is an LM head in its stochastic phase, nor, for ZIP-SR,
+// flat), the blocks run one branch-free sequence; a warp that does not
+// qualify takes the general sequence, with its per-lane and per-block range
+// tests.
 template <int VCODE, bool BF16W, bool FULLW>
 __device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTables& S,
                                                const StateArena& st, const uint8_t* sp,
-                                               const UnitHeader* hdp, uint32_t flags, int half,
-                                               int lane, unsigned hmask, float2& nfacc) {
+                                               const UnitHeader* hdp, uint32_t flags, int unit,
+                                               int lane, unsigned gmask, float2& nfacc) {
   constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
   constexpr bool kZip = (VCODE == kVZip || VCODE == kVZip32);
-  float w[kPerLane], g[kPerLane];
+  float w[kSub][kGroup], g[kSub][kGroup];
+  uint32_t mc[kSub], vc[kSub];
   const bool wbf = BF16W && (flags & kBf16W);
-  {
-    const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + half * 256 + lane * 16);
+#pragma unroll
+  for (int s = 0; s < kSub; ++s) {
+    const int o = group_off(s, lane);
+    const uint4 gg = *reinterpret_cast<const uint4*>(sp + kOffG + unit * 256 + o * 2);
     if (wbf) {
-      const uint4 wr = *reinterpret_cast<const uint4*>(sp + (hdp->nv_soff >> 8) + lane * 16);
-      w[0] = bf16lo(wr.x); w[1] = bf16hi(wr.x); w[2] = bf16lo(wr.y); w[3] = bf16hi(wr.y);
-      w[4] = bf16lo(wr.z); w[5] = bf16hi(wr.z); w[6] = bf16lo(wr.w); w[7] = bf16hi(wr.w);
+      const uint4 wr = *reinterpret_cast<const uint4*>(sp + (hdp->nv_soff >> 8) + o * 2);
+      w[s][0] = bf16lo(wr.x); w[s][1] = bf16hi(wr.x); w[s][2] = bf16lo(wr.y);
+      w[s][3] = bf16hi(wr.y); w[s][4] = bf16lo(wr.z); w[s][5] = bf16hi(wr.z);
+      w[s][6] = bf16lo(wr.w); w[s][7] = bf16hi(wr.w);
     } else {
-      const uint8_t* wsrc = sp + kOffW + half * 512 + lane * 32;
+      const uint8_t* wsrc = sp + kOffW + unit * 512 + o * 4;
       const float4 wa = *reinterpret_cast<const float4*>(wsrc);
       const float4 wb = *reinterpret_cast<const float4*>(wsrc + 16);
-      w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
-      w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
+      w[s][0] = wa.x; w[s][1] = wa.y; w[s][2] = wa.z; w[s][3] = wa.w;
+      w[s][4] = wb.x; w[s][5] = wb.y; w[s][6] = wb.z; w[s][7] = wb.w;
     }
-    g[0] = bf16lo(gg.x); g[1] = bf16hi(gg.x); g[2] = bf16lo(gg.y); g[3] = bf16hi(gg.y);
-    g[4] = bf16lo(gg.z); g[5] = bf16hi(gg.z); g[6] = bf16lo(gg.w); g[7] = bf16hi(gg.w);
+    g[s][0] = bf16lo(gg.x); g[s][1] = bf16hi(gg.x); g[s][2] = bf16lo(gg.y);
+    g[s][3] = bf16hi(gg.y); g[s][4] = bf16lo(gg.z); g[s][5] = bf16hi(gg.z);
+    g[s][6] = bf16lo(gg.w); g[s][7] = bf16hi(gg.w);
+    mc[s] = *reinterpret_cast<const uint32_t*>(sp + kOffMC + unit * 64 + o / 2);
+    vc[s] = *reinterpret_cast<const uint32_t*>(sp + kOffVC + unit * 64 + o / 2);
   }
-  const uint32_t mc = *reinterpret_cast<const uint32_t*>(sp + kOffMC + half * 64 + lane * 4);
-  const uint32_t vc = *reinterpret_cast<const uint32_t*>(sp + kOffVC + half * 64 + lane * 4);
-  const float2 sm = *reinterpret_cast<const float2*>(sp + kOffMS + half * 8);
-  const float2 sv = *reinterpret_cast<const float2*>(sp + kOffVS + half * 8);
+  const float2 sm = *reinterpret_cast<const float2*>(sp + kOffMS + unit * 8);
+  const float2 sv = *reinterpret_cast<const float2*>(sp + kOffVS + unit * 8);
   const float decay = hdp->decay;
 
-  float2 m1[kPerLane / 2], nv[kPerLane / 2], ndv[kPerLane / 2];
-  moments8(a, S, g, mc, vc, sm, sv, m1, nv);
-  const float lam = absmax8(m1);
-  const float lav = absmax8(nv);
-  const float am = hmax16<FULLW>(lam, hmask);
-  const float av = hmax16<FULLW>(lav, hmask);
+  float2 m1[kSub][4], nv[kSub][4], ndv[kSub][4];
+#pragma unroll
+  for (int s = 0; s < kSub; ++s) moments8(a, S, g[s], mc[s], vc[s], sm, sv, m1[s], nv[s]);
+  const float lam = absmax_lane(m1);
+  const float lav = absmax_lane(nv);
+  const float am = unit_max<FULLW>(lam, gmask);
+  const float av = unit_max<FULLW>(lav, gmask);
   const bool lane_fast = lane_in_range(a, m1, nv, lam, lav);
   bool warp_fast = false;
   float R = 0.0f;
@@ -1125,21 +1199,29 @@ __device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTabl
     }
     warp_fast = __all_sync(kFullMask, ok);
   }
+  int nall[kSub];
+#pragma unroll
+  for (int s = 0; s < kSub; ++s) nall[s] = kGroup;
   float* msp = hdp->ms;
   if (warp_fast) {
-    weights8_fast<kKeepDv>(a, decay, w, m1, nv, ndv, nfacc);
-    store_w8<BF16W>(hdp->w, wbf, lane, w);
-    requant_store<VCODE, true, FULLW, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, kPerLane,
-                                            hmask, m1, nv, ndv, am, av, R, hdp->mc + lane,
-                                            hdp->vc + lane, msp, msp + st.vs_minus_ms);
+#pragma unroll
+    for (int s = 0; s < kSub; ++s) {
+      weights8_fast<kKeepDv>(a, decay, w[s], m1[s], nv[s], ndv[s], nfacc);
+      store_w8<BF16W>(hdp->w, wbf, group_off(s, lane), w[s]);
+    }
+    requant_store<VCODE, true, FULLW, true>(a, S, hdp->tensor_id, flags, hdp->e0, lane, nall,
+                                            gmask, m1, nv, ndv, am, av, R, hdp->mc, hdp->vc, msp,
+                                            msp + st.vs_minus_ms);
   } else {
-    if (lane_fast) weights8_fast<kKeepDv>(a, decay, w, m1, nv, ndv, nfacc);
-    else weights8_ieee<true, kKeepDv>(a, decay, w, m1, nv, ndv, kPerLane, nfacc);
-    store_w8<BF16W>(hdp->w, wbf, lane, w);
-    requant_store<VCODE, true, FULLW, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane,
-                                             kPerLane, hmask, m1, nv, ndv, am, av, 0.0f,
-                                             hdp->mc + lane, hdp->vc + lane, msp,
-                                             msp + st.vs_minus_ms);
+#pragma unroll
+    for (int s = 0; s < kSub; ++s) {
+      if (lane_fast) weights8_fast<kKeepDv>(a, decay, w[s], m1[s], nv[s], ndv[s], nfacc);
+      else weights8_ieee<true, kKeepDv>(a, decay, w[s], m1[s], nv[s], ndv[s], kGroup, nfacc);
+      store_w8<BF16W>(hdp->w, wbf, group_off(s, lane), w[s]);
+    }
+    requant_store<VCODE, true, FULLW, false>(a, S, hdp->tensor_id, flags, hdp->e0, lane, nall,
+                                             gmask, m1, nv, ndv, am, av, 0.0f, hdp->mc, hdp->vc,
+                                             msp, msp + st.vs_minus_ms);
   }
 }
 
@@ -1148,7 +1230,7 @@ __device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTabl
 // ---------------------------------------------------------------------------
 
 template <int VCODE, bool BF16W>
-__global__ void __launch_bounds__(kCtaThreads, 3)
+__global__ void __launch_bounds__(kCtaThreads, kMinCtasPerSm)
 adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_end, StepArgs a,
                    StateArena st) {
   extern __shared__ __align__(128) uint8_t s_stage[];
@@ -1156,19 +1238,11 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
   __shared__ __align__(8) uint64_t s_empty[kStages];
   __shared__ SmemTables S;
 
-  {
-    const int t = threadIdx.x;
-    constexpr int kFamily = (VCODE == kVZe || VCODE == kVZeFloor) ? 1 : 0;   // zero-excluded
-    const uint4* src = reinterpret_cast<const uint4*>(&g_code_tables[kFamily]);
-    uint4* dst = reinterpret_cast<uint4*>(&S);
-#pragma unroll 1
-    for (int i = t; i < (int)(sizeof(SmemTables) / 16); i += kCtaThreads) dst[i] = src[i];
-    if (t < kStages) {
-      // full: the producer's expect-tx arrive plus one cp.async arrive per
-      // producer lane; empty: one release per consumer half-warp
-      mbar_init(smem_addr(&s_full[t]), 1 + kHalves);
-      mbar_init(smem_addr(&s_empty[t]), kHalves);
-    }
+  if (threadIdx.x < kStages) {
+    // full: the producer's expect-tx arrive plus one cp.async arrive per
+    // producer lane; empty: one release per unit slot
+    mbar_init(smem_addr(&s_full[threadIdx.x]), 1 + kTileUnits);
+    mbar_init(smem_addr(&s_empty[threadIdx.x]), kTileUnits);
     fence_mbar_init();
   }
   __syncthreads();
@@ -1177,16 +1251,41 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
   const uint32_t empty0 = smem_addr(&s_empty[0]);
   const int warp = threadIdx.x >> 5;
   if (warp == kProducerWarp) {
+    // (starts on the first tile at once; the tables are the consumers' concern)
     const int lane = threadIdx.x & 31;
-    if (lane < kHalves) produce<BF16W>(T, u_begin, u_end, a, st, s_stage, full0, empty0, lane);
+    if (lane < kTileUnits) produce<BF16W>(T, u_begin, u_end, a, st, s_stage, full0, empty0, lane);
     return;
   }
 
-  // ---- consumers: half-warp `half` takes unit `half` of every tile ----
-  const int lane = threadIdx.x & 15;
-  const int half = threadIdx.x >> 4;
-  const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
-  const int64_t ntiles = (u_end - u_begin + kHalves - 1) / kHalves;
+  // The consumers copy their code family's tables into shared memory while
+  // the producer fetches the first tiles, then meet at barrier 1 (consumer
+  // threads only; barrier 0 is the CTA-wide one above).
+  {
+    constexpr int kFamily = (VCODE == kVZe || VCODE == kVZeFloor) ? 1 : 0;   // zero-excluded
+    constexpr int kChunks = (int)(sizeof(SmemTables) / 16);
+    constexpr int kPerThread = (kChunks + kConsumerThreads - 1) / kConsumerThreads;
+    const uint4* src = reinterpret_cast<const uint4*>(&g_code_tables[kFamily]);
+    uint4* dst = reinterpret_cast<uint4*>(&S);
+    uint4 r[kPerThread];   // every load issued before the first store: one round trip
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = threadIdx.x + k * kConsumerThreads;
+      if (i < kChunks) r[k] = __ldg(src + i);
+    }
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = threadIdx.x + k * kConsumerThreads;
+      if (i < kChunks) dst[i] = r[k];
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+  }
+
+  // ---- consumers: the kLanesPerUnit lanes of slot `unit` take unit `unit`
+  // of every tile ----
+  const int lane = threadIdx.x & (kLanesPerUnit - 1);
+  const int unit = threadIdx.x / kLanesPerUnit;
+  const unsigned gmask = ((1u << kLanesPerUnit) - 1u) << (threadIdx.x & 31 & ~(kLanesPerUnit - 1));
+  const int64_t ntiles = (u_end - u_begin + kTileUnits - 1) / kTileUnits;
   int s = 0;
   uint32_t parity = 0;
   float2 nfacc = make_float2(0.0f, 0.0f);   // NaN once an updated weight is not finite
@@ -1198,21 +1297,21 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
       return;
     }
     const uint8_t* sp = s_stage + s * kStageBytes;
-    const UnitHeader* hdp = reinterpret_cast<const UnitHeader*>(sp + kOffHdr) + half;
+    const UnitHeader* hdp = reinterpret_cast<const UnitHeader*>(sp + kOffHdr) + unit;
     const uint32_t flags = hdp->flags;
     const bool staged = (flags & kStaged) != 0;
-    if (__all_sync(kFullMask, staged)) {          // both half-warps hold whole blocks
-      process_staged<VCODE, BF16W, true>(a, S, st, sp, hdp, flags, half, lane, hmask, nfacc);
+    if (__all_sync(kFullMask, staged)) {          // every block of the warp is whole and staged
+      process_staged<VCODE, BF16W, true>(a, S, st, sp, hdp, flags, unit, lane, gmask, nfacc);
     } else if (staged) {
-      process_staged<VCODE, BF16W, false>(a, S, st, sp, hdp, flags, half, lane, hmask, nfacc);
+      process_staged<VCODE, BF16W, false>(a, S, st, sp, hdp, flags, unit, lane, gmask, nfacc);
     } else if (!(flags & kNoUnit)) {
-      process_direct<VCODE, BF16W>(a, S, st, hdp, lane, hmask, nfacc);
+      process_direct<VCODE, BF16W>(a, S, st, hdp, lane, gmask, nfacc);
     }
     // every read of the stage (header included) is done: hand it back, one
-    // arrival per half-warp (both of the warp's, from its lane 0)
+    // arrival per unit slot (all of the warp's, from its lane 0)
     fence_proxy_async_smem();
     __syncwarp(kFullMask);
-    if ((threadIdx.x & 31) == 0) mbar_arrive(empty, 2);
+    if ((threadIdx.x & 31) == 0) mbar_arrive(empty, kUnitsPerWarp);
     if (++s == kStages) {
       s = 0;
       parity ^= 1u;

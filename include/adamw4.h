@@ -207,7 +207,7 @@ int adamw4_step_host(adamw4_handle *h, float lr, const uint16_t *const *grads_ho
 /* Waits for `cuda_stream` and reports whether the steps enqueued on it so far
  * completed.  The step kernel bounds every wait on its shared-memory pipeline
  * (about one second); when a wait runs out, the kernel records it in a device
- * status word and its half-warp stops, leaving that step incomplete.  The
+ * status word and the waiting warp stops, leaving that step incomplete.  The
  * kernel also records an updated weight that is not finite (a NaN or infinite
  * grad or weight leads to one; the pages leave non-finite inputs undefined, so
  * the step itself goes on).  This call reads and clears the word:
