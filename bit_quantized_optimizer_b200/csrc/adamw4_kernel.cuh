@@ -255,18 +255,6 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for a barrier phase; false if `limit_ns` passed first.  The timer is
 // read once per 64 polls.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
@@ -280,16 +268,31 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// mbarrier.try_wait with a suspend-time hint: the thread sleeps in hardware
+// until the phase completes or about `ns` nanoseconds pass, issuing nothing
+// meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // The producer's wait for a stage to come back: the consumers take
-// microseconds per tile, so it naps between polls instead of taking issue
-// slots from them.  False if `limit_ns` passed first.
-__device__ __forceinline__ bool wait_phase_napping(uint32_t bar, uint32_t parity,
+// microseconds per tile, so it sleeps in the barrier wait (20 us per try)
+// instead of polling, which would take issue slots from the consumer warps
+// of its SM sub-partition.  False if `limit_ns` passed first.
+__device__ __forceinline__ bool wait_phase_suspended(uint32_t bar, uint32_t parity,
                                                    uint64_t limit_ns) {
-  if (mbar_test_wait(bar, parity)) return true;
+  if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
-    __nanosleep(1000);
-    if (mbar_test_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
     if (global_ns() - t0 > limit_ns) return false;
   }
 }
@@ -308,10 +311,12 @@ __device__ __forceinline__ void mulwide(uint32_t a, uint32_t b, uint32_t& hi, ui
   asm("{\n\t.reg .u64 t;\n\tmul.wide.u32 t, %2, %3;\n\tmov.b64 {%1, %0}, t;\n\t}"
       : "=r"(hi), "=r"(lo) : "r"(a), "r"(b));
 }
-__device__ __forceinline__ uint4 philox4x32_10(uint64_t quad, uint32_t c3, const StepArgs& a) {
+// The counter's first two words are the 64-bit quad index (qhi, qlo).
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t qlo, uint32_t qhi, uint32_t c3,
+                                               const StepArgs& a) {
   uint32_t h0, l0;
-  mulwide(kPhiloxM0, (uint32_t)quad, h0, l0);
-  uint4 c = make_uint4(a.r0_hi_k0 ^ (uint32_t)(quad >> 32), a.r0_lo, h0 ^ c3 ^ a.rk1[0], l0);
+  mulwide(kPhiloxM0, qlo, h0, l0);
+  uint4 c = make_uint4(a.r0_hi_k0 ^ qhi, a.r0_lo, h0 ^ c3 ^ a.rk1[0], l0);
 #pragma unroll
   for (int r = 1; r < 10; ++r) {
     uint32_t hi0, lo0, hi1, lo1;
@@ -330,12 +335,21 @@ __device__ __forceinline__ float one_plus_u(uint32_t w) {
 }
 __device__ __forceinline__ float uniform23(uint32_t w) { return __fsub_rn(one_plus_u(w), 1.0f); }
 
-// The eight draw words of one lane: elements 4*quad .. 4*quad + 7.
+// The quad index (e0 + off) / 4 of a group at value offset `off` of a block
+// starting at element e0, as (low, high) words.  e0 is a multiple of 128 and
+// off + 7 < 128, so (e0 / 4) has five zero low bits and adding off / 4 or
+// off / 4 + 1 never carries into the high word.
+__device__ __forceinline__ uint32_t quad_lo(uint64_t e0, int off) {
+  return (uint32_t)(e0 >> 2) + (uint32_t)(off >> 2);
+}
+__device__ __forceinline__ uint32_t quad_hi(uint64_t e0) { return (uint32_t)(e0 >> 34); }
+
+// The eight draw words of one group: elements 4*quad .. 4*quad + 7.
 __device__ __forceinline__ void words8(const StepArgs& a, uint32_t tensor_id, uint32_t stream,
-                                       uint64_t quad, uint32_t r[8]) {
+                                       uint32_t qlo, uint32_t qhi, uint32_t r[8]) {
   const uint32_t c3 = tensor_id * 2u + stream;
-  const uint4 r0 = philox4x32_10(quad, c3, a);
-  const uint4 r1 = philox4x32_10(quad + 1, c3, a);
+  const uint4 r0 = philox4x32_10(qlo, qhi, c3, a);
+  const uint4 r1 = philox4x32_10(qlo + 1u, qhi, c3, a);
   r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w;
   r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
 }
@@ -491,7 +505,8 @@ static __device__ __align__(16) SmemTables g_code_tables[2];
 template <bool FULL, bool FLAT, bool U32>
 __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTables& S,
                                                  const float2 (&nv)[4], const float2 (&ndv)[4],
-                                                 uint64_t quad, uint32_t c3, float ninv, float R,
+                                                 uint32_t qlo, uint32_t qhi, uint32_t c3,
+                                                 float ninv, float R,
                                                  int myn) {
   // two values at a time; from the last pair to the first, so that element i
   // ends in bits 4i..4i+3.  The draws of values 4..7 come from the second
@@ -502,14 +517,14 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
   if (U32) {   // (the binary64 decision keeps all eight words: fewer live doubles)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      const uint4 r = philox4x32_10(quad + c, c3, a);
+      const uint4 r = philox4x32_10(qlo + (uint32_t)c, qhi, c3, a);
       rw[4 * c + 0] = r.x; rw[4 * c + 1] = r.y; rw[4 * c + 2] = r.z; rw[4 * c + 3] = r.w;
     }
   }
 #pragma unroll
   for (int j = kGroup / 2 - 1; j >= 0; --j) {
     if (!U32 && (j == 3 || j == 1)) {
-      const uint4 r = philox4x32_10(quad + (j >> 1), c3, a);
+      const uint4 r = philox4x32_10(qlo + (uint32_t)(j >> 1), qhi, c3, a);
       rw[4 * (j >> 1) + 0] = r.x; rw[4 * (j >> 1) + 1] = r.y;
       rw[4 * (j >> 1) + 2] = r.z; rw[4 * (j >> 1) + 3] = r.w;
     }
@@ -633,7 +648,7 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
 #pragma unroll
       for (int s = 0; s < kSub; ++s) {
         uint32_t rw[kGroup];
-        words8(a, tensor_id, kStreamM, (e0 + (uint64_t)group_off(s, lane)) >> 2, rw);
+        words8(a, tensor_id, kStreamM, quad_lo(e0, group_off(s, lane)), quad_hi(e0), rw);
 #pragma unroll
         for (int i = 0; i < kGroup; ++i)
           if (FULL || i < myn[s])
@@ -723,12 +738,14 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
 #pragma unroll
         for (int s = 0; s < kSub; ++s)
           vco[s] = zipsr_codes8<FULL, false, VCODE == kVZip32>(
-              a, S, nv[s], ndv[s], (e0 + (uint64_t)group_off(s, lane)) >> 2, c3, ninv, R, myn[s]);
+              a, S, nv[s], ndv[s], quad_lo(e0, group_off(s, lane)), quad_hi(e0), c3, ninv, R,
+              myn[s]);
       } else {
 #pragma unroll
         for (int s = 0; s < kSub; ++s)
           vco[s] = zipsr_codes8<FULL, true, VCODE == kVZip32>(
-              a, S, nv[s], ndv[s], (e0 + (uint64_t)group_off(s, lane)) >> 2, c3, ninv, R, myn[s]);
+              a, S, nv[s], ndv[s], quad_lo(e0, group_off(s, lane)), quad_hi(e0), c3, ninv, R,
+              myn[s]);
       }
       vso = av;
     } else if (VCODE == kVZiRtn || VCODE == kVZiSr) {
@@ -738,7 +755,7 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       for (int s = 0; s < kSub; ++s) {
         uint32_t rw[kGroup];
         if (VCODE == kVZiSr)
-          words8(a, tensor_id, kStreamV, (e0 + (uint64_t)group_off(s, lane)) >> 2, rw);
+          words8(a, tensor_id, kStreamV, quad_lo(e0, group_off(s, lane)), quad_hi(e0), rw);
 #pragma unroll
         for (int j = kGroup / 2 - 1; j >= 0; --j) {   // last element first
           const float2 x2 = __fmul2_rn(nv[s][j], f2(ninv));
@@ -995,7 +1012,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
   uint32_t round = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const uint32_t full = full0 + 8u * s;
-    if (round > 0 && !__all_sync(kMask, wait_phase_napping(empty0 + 8u * s, (round - 1) & 1u,
+    if (round > 0 && !__all_sync(kMask, wait_phase_suspended(empty0 + 8u * s, (round - 1) & 1u,
                                                            kWaitLimitNs))) {
       // Leaving early: flag it, then wait (bounded) for the copies this warp
       // issued into stages not yet handed back.  Stage j was last filled in
@@ -1004,7 +1021,7 @@ __device__ __forceinline__ void produce(const DevTensor* __restrict__ T, int64_t
       if (lane == 0) atomicOr(a.status, 1u);
       for (int j = 0; j < kStages; ++j) {
         const uint32_t last = (j < s) ? round : round - 1;
-        wait_phase_napping(full0 + 8u * j, last & 1u, kDrainLimitNs);
+        wait_phase_suspended(full0 + 8u * j, last & 1u, kDrainLimitNs);
       }
       cp_async_wait_all();
       return;
