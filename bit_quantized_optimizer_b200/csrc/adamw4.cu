@@ -100,12 +100,12 @@ struct DeviceGuard {
 };
 
 // The NF4 nearest-level bucket of x (the kernel's nf4_rtn_bucket reads the
-// same one from the bits of fma(x, 256, 1.5 * 2^23 + 256)).
+// same one from the bits of fma(x, 4096, 1.5 * 2^23 + 4096)).
 int nf4_bucket(float x) {
-  const float y = std::fma(x, 256.0f, 12583168.0f);
+  const float y = std::fma(x, 4096.0f, 12587008.0f);
   int32_t bits;
   std::memcpy(&bits, &y, 4);
-  return std::min(std::max(bits - 0x4B400000, 0), 512) >> 3;
+  return std::min(std::max(bits - 0x4B400000, 0), 8192) >> 7;
 }
 
 void build_tables(CodeTables* T) {
@@ -124,7 +124,7 @@ void build_tables(CodeTables* T) {
   float mid[15];
   for (int j = 0; j < 15; ++j)
     mid[j] = (float)(((double)kNF4Levels[j] + (double)kNF4Levels[j + 1]) * 0.5);
-  // Bucket b of x is floor(round(256 x + 256) / 8), in [0, 64] for
+  // Bucket b of x is floor(round(4096 x + 4096) / 128), in [0, 64] for
   // |x| <= 1 + 2^-23 and monotone in x.  A bucket holds at most one midpoint,
   // so the nearest level is the count of midpoints in lower buckets plus one
   // comparison.
@@ -155,7 +155,6 @@ void fill_smem_tables(const CodeTables& T, bool zero_excluded, SmemTables* S) {
     const float hi = zero_excluded ? (float)((t >> 4) + 1) * 0.0625f : T.vz[t >> 4];
     S->vpair[t] = make_float2(lo, hi);
   }
-  for (int t = 0; t < 128; ++t) S->rtn[t] = T.rtn[t];
   for (int t = 0; t < 16; ++t) {
     S->nf4[t] = T.nf4[t];
     S->gap[t] = T.nf4_gap[t];
@@ -181,8 +180,14 @@ cudaError_t upload_tables(int device) {
   static SmemTables host[2];
   fill_smem_tables(T, false, &host[0]);
   fill_smem_tables(T, true, &host[1]);
-  const cudaError_t e = cudaMemcpyToSymbol(g_code_tables, host, sizeof host, 0,
-                                           cudaMemcpyHostToDevice);
+  cudaError_t e = cudaMemcpyToSymbol(g_code_tables, host, sizeof host, 0,
+                                     cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return e;
+  // The NF4 buckets, one copy per lane of a half-warp, interleaved by entry.
+  static NF4Buckets buckets;
+  for (int b = 0; b < 128; ++b)
+    for (int c = 0; c < 16; ++c) buckets.e[b][c] = T.rtn[b];
+  e = cudaMemcpyToSymbol(g_nf4_buckets, &buckets, sizeof buckets, 0, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) g_tables_ready[device] = true;
   return e;
 }
@@ -240,13 +245,14 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.k_m1 = pair(-1.0f);
   a.k_15 = pair(15.0f);
   a.k_16 = pair(16.0f);
-  a.k_256 = pair(256.0f);
+  a.k_4096 = pair(4096.0f);
   a.k_magic = pair(kMagic);
   a.k_nmagic = pair(-kMagic);
-  a.k_magic256 = pair(kMagic + 256.0f);
+  a.k_magic4096 = pair(kMagic + 4096.0f);
   a.k_magicm1 = pair(kMagic - 1.0f);
   a.k_1_16 = pair(0.0625f);
   a.k_2m32 = pair(0x1p-32f);
+  a.k_ze_scale = make_float2(0.0625f, 0.00390625f);   // (1/16, 1/256)
   // Philox round keys: round r uses the seed words plus r times the Weyl
   // constants (mod 2^32).
   for (int r = 0; r < 10; ++r) {

@@ -145,8 +145,8 @@ struct StepArgs {
   // here so that the instructions read them from the kernel parameters
   // instead of rebuilding a register pair for each use.
   float2 p_b1, p_omb1, p_nb2, p_nomb2, p_rs, p_eps, p_neps, p_nstep;
-  float2 k_half, k_one, k_zero, k_m1, k_15, k_16, k_256, k_magic, k_nmagic, k_magic256,
-      k_magicm1, k_1_16, k_2m32;
+  float2 k_half, k_one, k_zero, k_m1, k_15, k_16, k_4096, k_magic, k_nmagic, k_magic4096,
+      k_magicm1, k_1_16, k_2m32, k_ze_scale;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
   int lm_sr_active;      // final-10% LM-head phase
@@ -164,7 +164,7 @@ struct CodeTables {
   float vz[16];         // ZIP-SR code points k/15
   float vz_sqrt[16];    // sqrt(k/15)
   float vz_mid[16];     // nearest-point thresholds of the k/15 code (15 used)
-  float2 rtn[128];      // NF4 nearest-level buckets (floor(round(256x + 256)/8)):
+  float2 rtn[128];      // NF4 nearest-level buckets (floor(round(4096x + 4096)/128)):
                         // .x threshold, .y base code (int bits)
 };
 
@@ -449,15 +449,27 @@ __device__ __forceinline__ float2 unit_sum_tree2(const float2 (&v)[kSub], unsign
   return __fadd2_rn(t[0], t[1]);
 }
 
-// NF4 nearest level: #{j : x > mid[j]}.  bucket_sum = fma(x, 256, kMagic +
-// 256) has the bit pattern of kMagic plus r = round(256 x + 256), r in
-// [0, 512] for |x| <= 1 + 2^-23, so r & 0x3F8 = 8 floor(r/8) is directly the
-// byte offset of bucket floor(r/8) in a table of 8-byte entries.  A bucket is
-// 1/32 wide in x and holds at most one threshold; the table has 128 entries,
-// so any 10-bit offset stays inside (entries past 64 read "above all").
-__device__ __forceinline__ uint32_t nf4_rtn_bucket(float x, float bucket_sum, const float2* rtn) {
-  const float2 e = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(rtn) +
-                                                    (__float_as_uint(bucket_sum) & 0x3F8u));
+// NF4 nearest-level buckets in shared memory, sixteen interleaved copies:
+// entry (b, c) = {threshold, base code} of bucket b for lane c of a
+// half-warp, so that the sixteen lanes of a half-warp read sixteen different
+// bank pairs whatever buckets they ask for (one wavefront per half-warp).
+struct NF4Buckets {
+  float2 e[128][16];
+};
+static __device__ __align__(16) NF4Buckets g_nf4_buckets;   // written once per device
+__shared__ __align__(16) NF4Buckets s_nf4_buckets;          // each CTA's copy
+
+// NF4 nearest level: #{j : x > mid[j]}.  bucket_sum = fma(x, 4096, kMagic +
+// 4096) has the bit pattern of kMagic plus r = round(4096 x + 4096), r in
+// [0, 8192] for |x| <= 1 + 2^-23, so r & 0x3F80 = 128 floor(r/128) is the
+// byte offset of row floor(r/128) of the 128-byte rows, and or-ing in the
+// lane's 8-byte column gives the address in one logic operation.  A bucket is
+// 1/32 wide in x and holds at most one threshold; there are 128 rows, so any
+// masked offset stays inside (rows past 64 read "above all").
+__device__ __forceinline__ uint32_t nf4_rtn_bucket(float x, float bucket_sum) {
+  const uint32_t off = (__float_as_uint(bucket_sum) & 0x3F80u) | ((threadIdx.x & 15u) << 3);
+  const float2 e = *reinterpret_cast<const float2*>(
+      reinterpret_cast<const uint8_t*>(&s_nf4_buckets) + off);
   return (uint32_t)(__float_as_int(e.y) + (x > e.x ? 1 : 0));
 }
 
@@ -474,7 +486,6 @@ __device__ __forceinline__ uint32_t nf4_sr(float x, float u, const float* nf4, c
 struct SmemTables {
   float2 mpair[256];   // byte of two m codes -> their two NF4 levels
   float2 vpair[256];   // byte of two v codes -> their two code points
-  float2 rtn[128];
   float nf4[16];
   float gap[16];
   float vz[16];        // ZIP-SR code points k/15
@@ -661,9 +672,9 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
 #pragma unroll
         for (int j = kGroup / 2 - 1; j >= 0; --j) {   // last element first
           const float2 x = __fmul2_rn(m1[s][j], f2(inv));
-          const float2 b = __ffma2_rn(x, a.k_256, a.k_magic256);
-          const uint32_t c1 = (FULL || 2 * j + 1 < myn[s]) ? nf4_rtn_bucket(x.y, b.y, S.rtn) : 0u;
-          const uint32_t c0 = (FULL || 2 * j < myn[s]) ? nf4_rtn_bucket(x.x, b.x, S.rtn) : 0u;
+          const float2 b = __ffma2_rn(x, a.k_4096, a.k_magic4096);
+          const uint32_t c1 = (FULL || 2 * j + 1 < myn[s]) ? nf4_rtn_bucket(x.y, b.y) : 0u;
+          const uint32_t c0 = (FULL || 2 * j < myn[s]) ? nf4_rtn_bucket(x.x, b.x) : 0u;
           mco[s] = (mco[s] * 16u + c1) * 16u + c0;
         }
       }
@@ -809,9 +820,15 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   }
 }
 
+// Whether the zero-excluded v codes are decoded by arithmetic instead of the
+// pair table (their code points (k+1)/16 are exact binary32 values).
+constexpr bool kArithZeDecode = true;
+
 // Decode and moment update for one group of 8 values of a 4-bit block
 // ("ZIP-SR / ZE-EDEN", Method flowchart: decode the prior moments, update
-// them).  Out: m1 and nv = -v1 in pairs.
+// them).  Out: m1 and nv = -v1 in pairs.  ZE_ARITH: the v codes are
+// zero-excluded and decoded arithmetically.
+template <bool ZE_ARITH>
 __device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
                                          const float (&g)[kGroup], uint32_t mc, uint32_t vc,
                                          float2 sm, float2 sv, float2 (&m1)[4], float2 (&nv)[4]) {
@@ -819,7 +836,19 @@ __device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
   for (int j = 0; j < kGroup / 2; ++j) {
     // one byte holds the codes of values 2j (low nibble) and 2j+1 (high nibble)
     const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], sm);
-    const float2 v0 = __fmul2_rn(S.vpair[__byte_perm(vc, 0, 0x4440 + j)], sv);
+    float2 vq;
+    if (ZE_ARITH) {
+      // kMagic + k and kMagic + 16 k (exact), minus kMagic: (k_lo, 16 k_hi);
+      // then (k + 1)/16 = k * (1/16) + 1/16 and 16 k * (1/256) + 1/16, exact
+      const uint32_t byte = __byte_perm(vc, 0, 0x4440 + j);
+      const float2 kk = __fadd2_rn(make_float2(__uint_as_float((byte & 0x0Fu) | 0x4B400000u),
+                                               __uint_as_float((byte & 0xF0u) | 0x4B400000u)),
+                                   a.k_nmagic);
+      vq = __ffma2_rn(kk, a.k_ze_scale, a.k_1_16);
+    } else {
+      vq = S.vpair[__byte_perm(vc, 0, 0x4440 + j)];
+    }
+    const float2 v0 = __fmul2_rn(vq, sv);
     const float2 gg = make_float2(g[2 * j], g[2 * j + 1]);
     m1[j] = __ffma2_rn(a.p_b1, m0, __fmul2_rn(a.p_omb1, gg));
     // -v1 = fma(-b2, v0, -(1-b2) g^2), the negation of the canonical v1 exactly
@@ -946,6 +975,7 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
   }
   // a ragged last block of a 4-bit tensor
   constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
+  constexpr bool kZeArith = kArithZeDecode && (VCODE == kVZe || VCODE == kVZeFloor);
   float* msp = hdp->ms;
   float* vsp = msp + st.vs_minus_ms;
   const float2 sm = f2(*msp), sv = f2(*vsp);
@@ -953,7 +983,8 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
   float lam = 0.0f, lav = 0.0f;
 #pragma unroll
   for (int s = 0; s < kSub; ++s) {
-    moments8(a, S, g[s], hdp->mc[s * kLanesPerUnit + lane], hdp->vc[s * kLanesPerUnit + lane], sm,
+    moments8<kZeArith>(a, S, g[s], hdp->mc[s * kLanesPerUnit + lane],
+                       hdp->vc[s * kLanesPerUnit + lane], sm,
              sv, m1[s], nv[s]);
 #pragma unroll
     for (int j = 0; j < kGroup / 2; ++j) ndv[s][j] = f2(-1.0f);   // (slots past myn)
@@ -1169,6 +1200,7 @@ __device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTabl
                                                int lane, unsigned gmask, float2& nfacc) {
   constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
   constexpr bool kZip = (VCODE == kVZip || VCODE == kVZip32);
+  constexpr bool kZeArith = kArithZeDecode && (VCODE == kVZe || VCODE == kVZeFloor);
   float w[kSub][kGroup], g[kSub][kGroup];
   uint32_t mc[kSub], vc[kSub];
   const bool wbf = BF16W && (flags & kBf16W);
@@ -1200,7 +1232,7 @@ __device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTabl
 
   float2 m1[kSub][4], nv[kSub][4], ndv[kSub][4];
 #pragma unroll
-  for (int s = 0; s < kSub; ++s) moments8(a, S, g[s], mc[s], vc[s], sm, sv, m1[s], nv[s]);
+  for (int s = 0; s < kSub; ++s) moments8<kZeArith>(a, S, g[s], mc[s], vc[s], sm, sv, m1[s], nv[s]);
   const float lam = absmax_lane(m1);
   const float lav = absmax_lane(nv);
   const float am = unit_max<FULLW>(lam, gmask);
@@ -1274,25 +1306,29 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
     return;
   }
 
-  // The consumers copy their code family's tables into shared memory while
-  // the producer fetches the first tiles, then meet at barrier 1 (consumer
-  // threads only; barrier 0 is the CTA-wide one above).
+  // The consumers copy their code family's tables and the NF4 buckets into
+  // shared memory while the producer fetches the first tiles, then meet at
+  // barrier 1 (consumer threads only; barrier 0 is the CTA-wide one above).
   {
     constexpr int kFamily = (VCODE == kVZe || VCODE == kVZeFloor) ? 1 : 0;   // zero-excluded
-    constexpr int kChunks = (int)(sizeof(SmemTables) / 16);
-    constexpr int kPerThread = (kChunks + kConsumerThreads - 1) / kConsumerThreads;
-    const uint4* src = reinterpret_cast<const uint4*>(&g_code_tables[kFamily]);
-    uint4* dst = reinterpret_cast<uint4*>(&S);
+    constexpr int kT = (int)(sizeof(SmemTables) / 16);
+    constexpr int kAll = kT + (int)(sizeof(NF4Buckets) / 16);
+    constexpr int kPerThread = (kAll + kConsumerThreads - 1) / kConsumerThreads;
+    const uint4* srcT = reinterpret_cast<const uint4*>(&g_code_tables[kFamily]);
+    const uint4* srcB = reinterpret_cast<const uint4*>(&g_nf4_buckets);
+    uint4* dstT = reinterpret_cast<uint4*>(&S);
+    uint4* dstB = reinterpret_cast<uint4*>(&s_nf4_buckets);
     uint4 r[kPerThread];   // every load issued before the first store: one round trip
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k) {
       const int i = threadIdx.x + k * kConsumerThreads;
-      if (i < kChunks) r[k] = __ldg(src + i);
+      if (i < kAll) r[k] = __ldg(i < kT ? srcT + i : srcB + (i - kT));
     }
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k) {
       const int i = threadIdx.x + k * kConsumerThreads;
-      if (i < kChunks) dst[i] = r[k];
+      if (i < kT) dstT[i] = r[k];
+      else if (i < kAll) dstB[i - kT] = r[k];
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
   }
