@@ -183,11 +183,17 @@ cudaError_t upload_tables(int device) {
   cudaError_t e = cudaMemcpyToSymbol(g_code_tables, host, sizeof host, 0,
                                      cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return e;
-  // The NF4 buckets, one copy per lane of a half-warp, interleaved by entry.
-  static NF4Buckets buckets;
+  // The lane tables: each entry repeated across the columns of its row.
+  static LaneTables lt;
   for (int b = 0; b < 128; ++b)
-    for (int c = 0; c < 16; ++c) buckets.e[b][c] = T.rtn[b];
-  e = cudaMemcpyToSymbol(g_nf4_buckets, &buckets, sizeof buckets, 0, cudaMemcpyHostToDevice);
+    for (int c = 0; c < 16; ++c) lt.nf4b[b][c] = T.rtn[b];
+  for (int k = 0; k < 16; ++k) {
+    for (int c = 0; c < 32; ++c) {
+      lt.nf4[k][c] = T.nf4[k];
+      lt.vz[k][c] = T.vz[k];
+    }
+  }
+  e = cudaMemcpyToSymbol(g_lane_tables, &lt, sizeof lt, 0, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) g_tables_ready[device] = true;
   return e;
 }

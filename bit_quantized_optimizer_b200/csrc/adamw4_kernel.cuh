@@ -449,15 +449,33 @@ __device__ __forceinline__ float2 unit_sum_tree2(const float2 (&v)[kSub], unsign
   return __fadd2_rn(t[0], t[1]);
 }
 
-// NF4 nearest-level buckets in shared memory, sixteen interleaved copies:
-// entry (b, c) = {threshold, base code} of bucket b for lane c of a
-// half-warp, so that the sixteen lanes of a half-warp read sixteen different
-// bank pairs whatever buckets they ask for (one wavefront per half-warp).
-struct NF4Buckets {
-  float2 e[128][16];
+// Tables read with data-dependent indices, laid out so that the lanes of a
+// warp never meet in a shared-memory bank whatever entries they ask for:
+// entry k of each table is one row, and lane c reads its own copy in column
+// c of that row.
+//   nf4b: NF4 nearest-level buckets {threshold, base code}, one 8-byte copy
+//         per half-warp lane (sixteen lanes per wavefront of 8-byte loads);
+//   nf4:  NF4 levels, one 4-byte copy per lane;
+//   vz:   the zero-inclusive v code points k/15, one copy per lane.
+struct LaneTables {
+  float2 nf4b[128][16];
+  float nf4[16][32];
+  float vz[16][32];
 };
-static __device__ __align__(16) NF4Buckets g_nf4_buckets;   // written once per device
-__shared__ __align__(16) NF4Buckets s_nf4_buckets;          // each CTA's copy
+static __device__ __align__(16) LaneTables g_lane_tables;   // written once per device
+__shared__ __align__(16) LaneTables s_lane;                  // each CTA's copy
+
+// Byte offset of the lane's copy of entry (nibble i of `code`) in a table of
+// 128-byte rows with 4-byte columns (i is a constant after unrolling, so the
+// shift is one instruction and the mask-and-or another).
+__device__ __forceinline__ uint32_t nibble_row_off(uint32_t code, int i) {
+  const uint32_t t = (4 * i <= 7) ? (code << (7 - 4 * i)) : (code >> (4 * i - 7));
+  return (t & 0x780u) | ((threadIdx.x & 31u) << 2);
+}
+__device__ __forceinline__ float lane_lookup(const float (&tab)[16][32], uint32_t code, int i) {
+  return *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(&tab[0][0]) +
+                                         nibble_row_off(code, i));
+}
 
 // NF4 nearest level: #{j : x > mid[j]}.  bucket_sum = fma(x, 4096, kMagic +
 // 4096) has the bit pattern of kMagic plus r = round(4096 x + 4096), r in
@@ -469,7 +487,7 @@ __shared__ __align__(16) NF4Buckets s_nf4_buckets;          // each CTA's copy
 __device__ __forceinline__ uint32_t nf4_rtn_bucket(float x, float bucket_sum) {
   const uint32_t off = (__float_as_uint(bucket_sum) & 0x3F80u) | ((threadIdx.x & 15u) << 3);
   const float2 e = *reinterpret_cast<const float2*>(
-      reinterpret_cast<const uint8_t*>(&s_nf4_buckets) + off);
+      reinterpret_cast<const uint8_t*>(&s_lane.nf4b[0][0]) + off);
   return (uint32_t)(__float_as_int(e.y) + (x > e.x ? 1 : 0));
 }
 
@@ -820,24 +838,44 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
   }
 }
 
-// Whether the zero-excluded v codes are decoded by arithmetic instead of the
-// pair table (their code points (k+1)/16 are exact binary32 values).
-constexpr bool kArithZeDecode = true;
+// How a group's codes are decoded, chosen per v code by measurement.  The
+// lane tables (one 4-byte load per value, no bank conflicts, two more
+// instructions per value for the address) pay for the zero-inclusive codes;
+// the zero-excluded ones decode v by arithmetic and keep the pair table for
+// m (one 8-byte load per two values), which costs them fewer instructions.
+constexpr int kVDecPair = 0;      // v through the pair table
+constexpr int kVDecZeArith = 1;   // v = (k + 1)/16 by arithmetic (zero-excluded)
+constexpr int kVDecLaneVz = 2;    // v through the lane table of k/15 (zero-inclusive)
+template <int VCODE>
+__host__ __device__ constexpr bool zero_excluded() {
+  return VCODE == kVZe || VCODE == kVZeFloor;
+}
+template <int VCODE>
+__host__ __device__ constexpr int v_decode() {
+  return zero_excluded<VCODE>() ? kVDecZeArith : kVDecLaneVz;
+}
+template <int VCODE>
+__host__ __device__ constexpr bool m_lane_decode() {
+  return !zero_excluded<VCODE>();
+}
 
 // Decode and moment update for one group of 8 values of a 4-bit block
 // ("ZIP-SR / ZE-EDEN", Method flowchart: decode the prior moments, update
-// them).  Out: m1 and nv = -v1 in pairs.  ZE_ARITH: the v codes are
-// zero-excluded and decoded arithmetically.
-template <bool ZE_ARITH>
+// them).  Out: m1 and nv = -v1 in pairs.  VDEC: how the v codes are decoded;
+// MLANE: the m codes through the lane table.
+template <int VDEC, bool MLANE>
 __device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
                                          const float (&g)[kGroup], uint32_t mc, uint32_t vc,
                                          float2 sm, float2 sv, float2 (&m1)[4], float2 (&nv)[4]) {
 #pragma unroll
   for (int j = 0; j < kGroup / 2; ++j) {
     // one byte holds the codes of values 2j (low nibble) and 2j+1 (high nibble)
-    const float2 m0 = __fmul2_rn(S.mpair[__byte_perm(mc, 0, 0x4440 + j)], sm);
+    const float2 mq = MLANE ? make_float2(lane_lookup(s_lane.nf4, mc, 2 * j),
+                                                 lane_lookup(s_lane.nf4, mc, 2 * j + 1))
+                                   : S.mpair[__byte_perm(mc, 0, 0x4440 + j)];
+    const float2 m0 = __fmul2_rn(mq, sm);
     float2 vq;
-    if (ZE_ARITH) {
+    if (VDEC == kVDecZeArith) {
       // kMagic + k and kMagic + 16 k (exact), minus kMagic: (k_lo, 16 k_hi);
       // then (k + 1)/16 = k * (1/16) + 1/16 and 16 k * (1/256) + 1/16, exact
       const uint32_t byte = __byte_perm(vc, 0, 0x4440 + j);
@@ -845,6 +883,8 @@ __device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
                                                __uint_as_float((byte & 0xF0u) | 0x4B400000u)),
                                    a.k_nmagic);
       vq = __ffma2_rn(kk, a.k_ze_scale, a.k_1_16);
+    } else if (VDEC == kVDecLaneVz) {
+      vq = make_float2(lane_lookup(s_lane.vz, vc, 2 * j), lane_lookup(s_lane.vz, vc, 2 * j + 1));
     } else {
       vq = S.vpair[__byte_perm(vc, 0, 0x4440 + j)];
     }
@@ -975,7 +1015,6 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
   }
   // a ragged last block of a 4-bit tensor
   constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
-  constexpr bool kZeArith = kArithZeDecode && (VCODE == kVZe || VCODE == kVZeFloor);
   float* msp = hdp->ms;
   float* vsp = msp + st.vs_minus_ms;
   const float2 sm = f2(*msp), sv = f2(*vsp);
@@ -983,7 +1022,7 @@ __device__ __forceinline__ void process_direct(const StepArgs& a, const SmemTabl
   float lam = 0.0f, lav = 0.0f;
 #pragma unroll
   for (int s = 0; s < kSub; ++s) {
-    moments8<kZeArith>(a, S, g[s], hdp->mc[s * kLanesPerUnit + lane],
+    moments8<v_decode<VCODE>(), m_lane_decode<VCODE>()>(a, S, g[s], hdp->mc[s * kLanesPerUnit + lane],
                        hdp->vc[s * kLanesPerUnit + lane], sm,
              sv, m1[s], nv[s]);
 #pragma unroll
@@ -1200,7 +1239,6 @@ __device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTabl
                                                int lane, unsigned gmask, float2& nfacc) {
   constexpr bool kKeepDv = (VCODE == kVZip || VCODE == kVZip32);
   constexpr bool kZip = (VCODE == kVZip || VCODE == kVZip32);
-  constexpr bool kZeArith = kArithZeDecode && (VCODE == kVZe || VCODE == kVZeFloor);
   float w[kSub][kGroup], g[kSub][kGroup];
   uint32_t mc[kSub], vc[kSub];
   const bool wbf = BF16W && (flags & kBf16W);
@@ -1232,7 +1270,8 @@ __device__ __forceinline__ void process_staged(const StepArgs& a, const SmemTabl
 
   float2 m1[kSub][4], nv[kSub][4], ndv[kSub][4];
 #pragma unroll
-  for (int s = 0; s < kSub; ++s) moments8<kZeArith>(a, S, g[s], mc[s], vc[s], sm, sv, m1[s], nv[s]);
+  for (int s = 0; s < kSub; ++s)
+    moments8<v_decode<VCODE>(), m_lane_decode<VCODE>()>(a, S, g[s], mc[s], vc[s], sm, sv, m1[s], nv[s]);
   const float lam = absmax_lane(m1);
   const float lav = absmax_lane(nv);
   const float am = unit_max<FULLW>(lam, gmask);
@@ -1306,18 +1345,18 @@ adamw4_step_kernel(const DevTensor* __restrict__ T, int64_t u_begin, int64_t u_e
     return;
   }
 
-  // The consumers copy their code family's tables and the NF4 buckets into
+  // The consumers copy their code family's tables and the lane tables into
   // shared memory while the producer fetches the first tiles, then meet at
   // barrier 1 (consumer threads only; barrier 0 is the CTA-wide one above).
   {
     constexpr int kFamily = (VCODE == kVZe || VCODE == kVZeFloor) ? 1 : 0;   // zero-excluded
     constexpr int kT = (int)(sizeof(SmemTables) / 16);
-    constexpr int kAll = kT + (int)(sizeof(NF4Buckets) / 16);
+    constexpr int kAll = kT + (int)(sizeof(LaneTables) / 16);
     constexpr int kPerThread = (kAll + kConsumerThreads - 1) / kConsumerThreads;
     const uint4* srcT = reinterpret_cast<const uint4*>(&g_code_tables[kFamily]);
-    const uint4* srcB = reinterpret_cast<const uint4*>(&g_nf4_buckets);
+    const uint4* srcB = reinterpret_cast<const uint4*>(&g_lane_tables);
     uint4* dstT = reinterpret_cast<uint4*>(&S);
-    uint4* dstB = reinterpret_cast<uint4*>(&s_nf4_buckets);
+    uint4* dstB = reinterpret_cast<uint4*>(&s_lane);
     uint4 r[kPerThread];   // every load issued before the first store: one round trip
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k) {
