@@ -291,7 +291,8 @@ def teacher_forced_parity(name, vcode, steps, seed=0, what=""):
     after step `steps` - 1 are given to the oracle, which computes step
     `steps` on sampled blocks of every 4-bit tensor and on every fp32-state
     tensor; the GPU's own step `steps` must match it.  Returns (blocks
-    checked, share of the sampled v codes that are 0 after step `steps` - 1)."""
+    checked, shares of the sampled v codes that are 0 and 1 after step
+    `steps` - 1)."""
     import torch
     ts = workloads.tensor_list(name)
     params, grads = workloads.device_inputs(name, ts, seed=seed)
@@ -308,7 +309,7 @@ def teacher_forced_parity(name, vcode, steps, seed=0, what=""):
         ref = oracle_for(ts, vcode=vcode, seed=0)
         ref.t = steps - 1
         d_in = {}
-        zero_codes, n_codes = 0, 0
+        zero_codes, one_codes, n_codes = 0, 0, 0
         for i, blocks in sel.items():
             w, valid = _gather_blocks(params[i], ts[i]["numel"], blocks, np.float32)
             g, _ = _gather_blocks(grads[i], ts[i]["numel"], blocks, np.uint16)
@@ -316,6 +317,7 @@ def teacher_forced_parity(name, vcode, steps, seed=0, what=""):
             vc = np.concatenate([tb["vcodes"][b * 64:(b + 1) * 64] for b in blocks]).copy()
             nib = np.stack([vc & 15, vc >> 4], axis=1).reshape(-1)[:valid.size][valid]
             zero_codes += int((nib == 0).sum())
+            one_codes += int((nib == 1).sum())
             n_codes += nib.size
             d_in[i] = dict(blocks=blocks, w=w, w0=w.copy(), g=g, valid=valid,
                            mc=np.concatenate([tb["mcodes"][b * 64:(b + 1) * 64] for b in blocks]).copy(),
@@ -358,7 +360,7 @@ def teacher_forced_parity(name, vcode, steps, seed=0, what=""):
             assert_weights_close(params[i].cpu().numpy(), fp_w[i], old_fp[i], f"{what} fp32 {i}")
             np.testing.assert_allclose(after["tensors"][i]["m"], st.m, rtol=1e-6, atol=0)
             np.testing.assert_allclose(after["tensors"][i]["v"], st.v, rtol=1e-6, atol=0)
-        return checked, zero_codes / max(n_codes, 1)
+        return checked, zero_codes / max(n_codes, 1), one_codes / max(n_codes, 1)
     finally:
         opt.close()
         del params, grads

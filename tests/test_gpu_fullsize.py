@@ -82,11 +82,13 @@ def test_gpt_2p7b_step_100_teacher_forced(vcode):
     preconditioner-space rounding picks from the first cell only with
     probability about eps / sqrt(v_hat), v_hat = v / (1 - b2^t) ("ZIP-SR
     4-bit AdamW -- Preconditioner-space stochastic rounding", worked example
-    paragraph), so it stays rare while v is well above eps^2; for ZE-EDEN
-    code 0 is the lowest nonzero point 1/16."""
+    paragraph), so it stays rare while v is well above eps^2, and the values
+    of that cell land on code 1, its upper point (also reported); for
+    ZE-EDEN code 0 is the lowest nonzero point 1/16."""
     from gpu_common import teacher_forced_parity
-    n, zero_share = teacher_forced_parity("gpt-2.7b", vcode, 100, what=f"gpt-2.7b v{vcode} t100")
+    n, zero_share, one_share = teacher_forced_parity("gpt-2.7b", vcode, 100,
+                                                     what=f"gpt-2.7b v{vcode} t100")
     assert n > 1500
-    assert 0.0 <= zero_share <= 1.0
+    assert 0.0 <= zero_share <= 1.0 and 0.0 <= one_share <= 1.0
     print(f"v{vcode}: {n} blocks checked at step 100; v codes at 0 after step 99: "
-          f"{100 * zero_share:.3f}%")
+          f"{100 * zero_share:.3f}%, at 1: {100 * one_share:.3f}%")
