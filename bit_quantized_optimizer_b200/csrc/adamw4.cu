@@ -255,7 +255,7 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.k_magic = pair(kMagic);
   a.k_nmagic = pair(-kMagic);
   a.k_magic4096 = pair(kMagic + 4096.0f);
-  a.k_magicm1 = pair(kMagic - 1.0f);
+  a.k_nmagic_16 = pair(-kMagic / 16.0f);                 // exact
   a.k_1_16 = pair(0.0625f);
   a.k_2m32 = pair(0x1p-32f);
   a.k_ze_scale = make_float2(0.0625f, 0.00390625f);   // (1/16, 1/256)

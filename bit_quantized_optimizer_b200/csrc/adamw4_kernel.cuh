@@ -146,7 +146,7 @@ struct StepArgs {
   // instead of rebuilding a register pair for each use.
   float2 p_b1, p_omb1, p_nb2, p_nomb2, p_rs, p_eps, p_neps, p_nstep;
   float2 k_half, k_one, k_zero, k_m1, k_15, k_16, k_4096, k_magic, k_nmagic, k_magic4096,
-      k_magicm1, k_1_16, k_2m32, k_ze_scale;
+      k_nmagic_16, k_1_16, k_2m32, k_ze_scale;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
   int lm_sr_active;      // final-10% LM-head phase
@@ -607,13 +607,17 @@ __device__ __forceinline__ uint32_t zipsr_codes8(const StepArgs& a, const SmemTa
   return vco;
 }
 
-// The codes k of a pair of zero-excluded values from cm = (k + 1) as exact
-// binary32 integers in [1, 16]: cm + (kMagic - 1) is exact, and its bit
+// The codes k of a pair of zero-excluded values from tm = kMagic + (k + 1),
+// k in [0, 15] (exact binary32 integers): tm - 1 is exact, and its bit
 // pattern is kMagic's (low byte 0) plus k.  The low byte of the result holds
 // k of the first value in bits 0-3 and of the second in bits 4-7.
-__device__ __forceinline__ uint32_t ze_code_pair(float2 cm, float2 magic_m1) {
-  const float2 kb = __fadd2_rn(cm, magic_m1);                // magic_m1 = kMagic - 1
+__device__ __forceinline__ uint32_t ze_code_pair(float2 tm, float2 m1) {
+  const float2 kb = __fadd2_rn(tm, m1);                      // m1 = (-1, -1)
   return __float_as_uint(kb.x) + 16u * __float_as_uint(kb.y);
+}
+// kMagic + max(rint(16x), 1) from t2 = fma(x, 16, kMagic) = kMagic + rint(16x).
+__device__ __forceinline__ float2 ze_point(float2 t2) {
+  return make_float2(fmaxf(t2.x, kMagic + 1.0f), fmaxf(t2.y, kMagic + 1.0f));
 }
 
 // The low bytes of four code pairs as one 32-bit word of eight nibbles
@@ -723,10 +727,10 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
       for (int j = 0; j < kGroup / 2; ++j) {
         const float2 x2 = __fmul2_rn(nv[s][j], f2(ninv));
         const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
-        const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
-        const float2 cm = make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f));   // k + 1
-        const float2 q2 = __fmul2_rn(cm, a.k_1_16);                // (k+1)/16
-        P[s][j] = ze_code_pair(cm, a.k_magicm1);
+        const float2 tm = ze_point(t2);                            // kMagic + k + 1
+        // (k+1)/16 = tm/16 - kMagic/16: both terms and the result exact
+        const float2 q2 = __ffma2_rn(tm, a.k_1_16, a.k_nmagic_16);
+        P[s][j] = ze_code_pair(tm, a.k_m1);
         float2 xx = __fmul2_rn(x2, x2);
         float2 xq = __fmul2_rn(x2, q2);
         if (!FULL) {
@@ -818,8 +822,7 @@ __device__ __forceinline__ void requant_store(const StepArgs& a, const SmemTable
         for (int j = 0; j < kGroup / 2; ++j) {
           const float2 x2 = __fmul2_rn(nv[s][j], f2(ninv));
           const float2 t2 = __ffma2_rn(x2, a.k_16, a.k_magic);       // kMagic + rint(16x)
-          const float2 c2 = __fadd2_rn(t2, a.k_nmagic);              // rint(16x), exact
-          P[j] = ze_code_pair(make_float2(fmaxf(c2.x, 1.0f), fmaxf(c2.y, 1.0f)), a.k_magicm1);
+          P[j] = ze_code_pair(ze_point(t2), a.k_m1);
         }
         vco[s] = pack_code_pairs(P, FULL ? kGroup : myn[s]);
       }
