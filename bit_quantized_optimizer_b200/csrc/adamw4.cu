@@ -258,7 +258,13 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.k_nmagic_16 = pair(-kMagic / 16.0f);                 // exact
   a.k_1_16 = pair(0.0625f);
   a.k_2m32 = pair(0x1p-32f);
-  a.k_ze_scale = make_float2(0.0625f, 0.00390625f);   // (1/16, 1/256)
+  // the arithmetic decode of zero-excluded v codes: scales 2^-(p+4) and
+  // offsets 1/16 - kMagic 2^-(p+4) for nibbles at bit p = 0, 4 (byte 0) and
+  // 8, 12 (byte 1), all exact
+  a.k_ze_scale0 = make_float2(0x1p-4f, 0x1p-8f);
+  a.k_ze_off0 = make_float2(0.0625f - kMagic * 0x1p-4f, 0.0625f - kMagic * 0x1p-8f);
+  a.k_ze_scale1 = make_float2(0x1p-12f, 0x1p-16f);
+  a.k_ze_off1 = make_float2(0.0625f - kMagic * 0x1p-12f, 0.0625f - kMagic * 0x1p-16f);
   // Philox round keys: round r uses the seed words plus r times the Weyl
   // constants (mod 2^32).
   for (int r = 0; r < 10; ++r) {

@@ -146,7 +146,7 @@ struct StepArgs {
   // instead of rebuilding a register pair for each use.
   float2 p_b1, p_omb1, p_nb2, p_nomb2, p_rs, p_eps, p_neps, p_nstep;
   float2 k_half, k_one, k_zero, k_m1, k_15, k_16, k_4096, k_magic, k_nmagic, k_magic4096,
-      k_nmagic_16, k_1_16, k_2m32, k_ze_scale;
+      k_nmagic_16, k_1_16, k_2m32, k_ze_scale0, k_ze_off0, k_ze_scale1, k_ze_off1;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
   int lm_sr_active;      // final-10% LM-head phase
@@ -879,13 +879,17 @@ __device__ __forceinline__ void moments8(const StepArgs& a, const SmemTables& S,
     const float2 m0 = __fmul2_rn(mq, sm);
     float2 vq;
     if (VDEC == kVDecZeArith) {
-      // kMagic + k and kMagic + 16 k (exact), minus kMagic: (k_lo, 16 k_hi);
-      // then (k + 1)/16 = k * (1/16) + 1/16 and 16 k * (1/256) + 1/16, exact
-      const uint32_t byte = __byte_perm(vc, 0, 0x4440 + j);
-      const float2 kk = __fadd2_rn(make_float2(__uint_as_float((byte & 0x0Fu) | 0x4B400000u),
-                                               __uint_as_float((byte & 0xF0u) | 0x4B400000u)),
-                                   a.k_nmagic);
-      vq = __ffma2_rn(kk, a.k_ze_scale, a.k_1_16);
+      // The two nibbles of byte j, left in place in the low 16 bits of the
+      // word (bytes 2 and 3 shifted down first), or-ed into kMagic's
+      // mantissa: kMagic + k 2^p, exact, with p = 8 (j & 1) or 8 (j & 1) + 4.
+      // Then (k + 1)/16 = (kMagic + k 2^p) 2^-(p+4) + (1/16 - kMagic 2^-(p+4)),
+      // one fma whose product, addend and result are all exact.
+      const uint32_t w = (j < 2) ? vc : (vc >> 16);
+      const uint32_t lo = (w & (0x0Fu << (8 * (j & 1)))) | 0x4B400000u;
+      const uint32_t hi = (w & (0xF0u << (8 * (j & 1)))) | 0x4B400000u;
+      vq = __ffma2_rn(make_float2(__uint_as_float(lo), __uint_as_float(hi)),
+                      (j & 1) ? a.k_ze_scale1 : a.k_ze_scale0,
+                      (j & 1) ? a.k_ze_off1 : a.k_ze_off0);
     } else if (VDEC == kVDecLaneVz) {
       vq = make_float2(lane_lookup(s_lane.vz, vc, 2 * j), lane_lookup(s_lane.vz, vc, 2 * j + 1));
     } else {
