@@ -221,9 +221,6 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.omb2 = (float)(1.0 - (double)c.beta2);
   a.eps = c.eps;
   a.lr = lr;
-  a.nb2 = -a.b2;
-  a.nomb2 = -a.omb2;
-  a.neps = -a.eps;
   a.nstep = -a.step_size;
   // Ranges of the kernel's fast square root and division (exact_math.cuh):
   // v1 in [2^-100, 2^64] keeps sqrt(v1) rs_bc2 + eps within [eps, 2^53) when
@@ -239,11 +236,11 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   auto pair = [](float x) { return make_float2(x, x); };
   a.p_b1 = pair(a.b1);
   a.p_omb1 = pair(a.omb1);
-  a.p_nb2 = pair(a.nb2);
-  a.p_nomb2 = pair(a.nomb2);
+  a.p_nb2 = pair(-a.b2);
+  a.p_nomb2 = pair(-a.omb2);
   a.p_rs = pair(a.rs_bc2);
   a.p_eps = pair(a.eps);
-  a.p_neps = pair(a.neps);
+  a.p_neps = pair(-a.eps);
   a.p_nstep = pair(a.nstep);
   a.k_half = pair(0.5f);
   a.k_one = pair(1.0f);
@@ -253,7 +250,6 @@ StepArgs make_args(const adamw4_config& c, float lr, int64_t t) {
   a.k_16 = pair(16.0f);
   a.k_4096 = pair(4096.0f);
   a.k_magic = pair(kMagic);
-  a.k_nmagic = pair(-kMagic);
   a.k_magic4096 = pair(kMagic + 4096.0f);
   a.k_nmagic_16 = pair(-kMagic / 16.0f);                 // exact
   a.k_1_16 = pair(0.0625f);

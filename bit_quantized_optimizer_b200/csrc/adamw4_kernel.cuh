@@ -135,7 +135,7 @@ struct StepArgs {
   float step_size;   // lr / (1 - b1^t)
   float rs_bc2;      // 1 / sqrt(1 - b2^t)
   float b1, omb1, b2, omb2, eps, lr;
-  float nb2, nomb2, neps, nstep;  // -b2, -(1 - b2), -eps, -step_size
+  float nstep;                  // -step_size
   // Operand ranges of the fast division and square root (exact_math.cuh):
   // a lane takes them when all its |m1| lie in [m_lo, m_hi] and all its v1
   // in [v_lo, v_hi]; otherwise it uses the IEEE operations.  m_hi < 0
@@ -145,7 +145,7 @@ struct StepArgs {
   // here so that the instructions read them from the kernel parameters
   // instead of rebuilding a register pair for each use.
   float2 p_b1, p_omb1, p_nb2, p_nomb2, p_rs, p_eps, p_neps, p_nstep;
-  float2 k_half, k_one, k_zero, k_m1, k_15, k_16, k_4096, k_magic, k_nmagic, k_magic4096,
+  float2 k_half, k_one, k_zero, k_m1, k_15, k_16, k_4096, k_magic, k_magic4096,
       k_nmagic_16, k_1_16, k_2m32, k_ze_scale0, k_ze_off0, k_ze_scale1, k_ze_off1;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   uint32_t r0_hi_k0, r0_lo;   // round 0 with counter word 2 = t: hi(M1 t) ^ key0, lo(M1 t)
