@@ -6,13 +6,13 @@
 // One kernel launch covers a range of units of a flat unit list: each block
 // of a 4-bit tensor is one unit, and each fp32-state tensor is cut into
 // 128-element chunks.  The grid is persistent (SM count x resident CTAs) and
-// tiles of 28 consecutive units are dealt out round-robin, so all SMs stream
+// tiles of 16 consecutive units are dealt out round-robin, so all SMs stream
 // one contiguous window of HBM.
 //
-// A CTA has one producer warp and seven consumer warps, and a ring of kStages
+// A CTA has one producer warp and four consumer warps, and a ring of kStages
 // CTA-wide stages, one tile each.  Eight lanes take one unit, sixteen values
 // per lane (two groups of eight, 64 values apart), so a warp takes four units
-// and the CTA's 28 slots one tile.  For every unit of a tile, producer lane i
+// and the CTA's 16 slots one tile.  For every unit of a tile, producer lane i
 // writes a 64-byte header (addresses, block index, tensor id, flags, decay)
 // into the stage; for runs of whole 4-bit blocks of one tensor the first lane
 // of the run fills the stage with TMA bulk copies (cp.async.bulk: the run's
@@ -64,15 +64,15 @@ constexpr int kGroup = 8;
 constexpr int kSub = 2;
 constexpr int kLanesPerUnit = kBlock / (kGroup * kSub);   // 8 lanes per block
 constexpr int kUnitsPerWarp = 32 / kLanesPerUnit;         // 4 blocks per warp
-constexpr int kConsumerWarps = 7;
+constexpr int kConsumerWarps = 4;
 constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kCtaThreads = kConsumerThreads + 32;  // plus the producer warp
-constexpr int kTileUnits = kConsumerThreads / kLanesPerUnit;  // units per tile: 28
+constexpr int kTileUnits = kConsumerThreads / kLanesPerUnit;  // units per tile: 16
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kStages = 3;                        // tiles in flight per CTA
-// Two CTAs of eight warps per SM: four warps per SM sub-partition, whose
-// 16,384-register file then gives each thread up to 128 registers.
-constexpr int kMinCtasPerSm = 2;
+// Three CTAs of five warps per SM: at most four warps per SM sub-partition,
+// whose 16,384-register file then gives each thread up to 128 registers.
+constexpr int kMinCtasPerSm = 3;
 static_assert(kGroup * kSub * kLanesPerUnit == kBlock, "lane layout");
 static_assert(kTileUnits <= 32, "one producer lane per unit");
 // Value offset of group s of lane l within its block.
@@ -88,7 +88,7 @@ constexpr int kOffMC = kOffG + kTileUnits * 256;
 constexpr int kOffVC = kOffMC + kTileUnits * 64;
 constexpr int kOffMS = kOffVC + kTileUnits * 64;
 constexpr int kOffVS = kOffMS + kTileUnits * 8;
-constexpr int kStageBytes = kOffVS + kTileUnits * 8; // 27,328 B, a 16-byte multiple
+constexpr int kStageBytes = kOffVS + kTileUnits * 8; // 15,616 B, a 16-byte multiple
 constexpr uint32_t kUnitTx = 896;                 // bulk-copied bytes of one whole block
 constexpr int kSmemStages = kStages * kStageBytes;
 static_assert(kStageBytes % 16 == 0, "stage alignment");
