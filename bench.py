@@ -173,6 +173,9 @@ def dist_setup(n_gpus):
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
+        # one line per rank on stderr (stdout carries rank 0's JSON line only)
+        print(f"bench: rank {rank} of {ws} on cuda:{local} ({torch.cuda.get_device_name(local)}), "
+              f"process group {dist.get_backend()}", file=sys.stderr, flush=True)
     else:
         torch.cuda.set_device(0)
     return ws, rank, local
