@@ -284,7 +284,7 @@ def sampled_parity(name, vcode, steps, t0=0, total_steps=0, prewarm=False, seed=
         torch.cuda.empty_cache()
 
 
-def teacher_forced_parity(name, vcode, steps, seed=0, what=""):
+def teacher_forced_parity(name, vcode, steps, seed=0, what="", total_steps=0):
     """Runs the CUDA path for `steps` steps over a full-size list (device
     inputs, one seeded grad set reused every step, zero initial state), then
     checks the last step teacher-forced: the state and weights the GPU holds
@@ -292,21 +292,22 @@ def teacher_forced_parity(name, vcode, steps, seed=0, what=""):
     `steps` on sampled blocks of every 4-bit tensor and on every fp32-state
     tensor; the GPU's own step `steps` must match it.  Returns (blocks
     checked, shares of the sampled v codes that are 0 and 1 after step
-    `steps` - 1)."""
+    `steps` - 1).  total_steps: the run length that sets the LM head's
+    final-10% phase (0: never)."""
     import torch
     ts = workloads.tensor_list(name)
     params, grads = workloads.device_inputs(name, ts, seed=seed)
     sel = sampled_blocks(ts, seed=seed + 1)
     fp_idx = [i for i, t in enumerate(ts) if oracle.is_fp32_state(t["numel"], t["flags"])]
     B_ = binding()
-    opt = B_.AdamW4(params, grads, ts, lr=1e-3, vcode=vcode, seed=0)
+    opt = B_.AdamW4(params, grads, ts, lr=1e-3, vcode=vcode, seed=0, total_steps=total_steps)
     try:
         for _ in range(steps - 1):
             opt.step()
         torch.cuda.synchronize()
         before = parse_blob(opt.state_dict_blob())
         assert before["t"] == steps - 1
-        ref = oracle_for(ts, vcode=vcode, seed=0)
+        ref = oracle_for(ts, vcode=vcode, seed=0, total_steps=total_steps)
         ref.t = steps - 1
         d_in = {}
         zero_codes, one_codes, n_codes = 0, 0, 0

@@ -92,3 +92,19 @@ def test_gpt_2p7b_step_100_teacher_forced(vcode):
     assert 0.0 <= zero_share <= 1.0 and 0.0 <= one_share <= 1.0
     print(f"v{vcode}: {n} blocks checked at step 100; v codes at 0 after step 99: "
           f"{100 * zero_share:.3f}%, at 1: {100 * one_share:.3f}%")
+
+
+@pytest.mark.parametrize("vcode", [0, 1])
+def test_gpt_130m_step_1000_teacher_forced_lm_head_phase(vcode):
+    """A longer run on the 130M list: 999 GPU steps (one grad set reused), then
+    step 1000 teacher-forced against the oracle, with total_steps = 1000 so
+    that steps past 900 are in the LM head's final-10% phase ("ZIP-SR 4-bit
+    AdamW -- Preconditioner-space stochastic rounding", ZE-EDEN paragraph):
+    the tied embedding's m is then rounded stochastically on the NF4 grid,
+    and the oracle checks extra blocks of it."""
+    from gpu_common import teacher_forced_parity
+    n, zero_share, one_share = teacher_forced_parity(
+        "gpt-130m", vcode, 1000, what=f"gpt-130m v{vcode} t1000", total_steps=1000)
+    assert n > 300
+    print(f"v{vcode}: {n} blocks checked at step 1000; v codes at 0 after step 999: "
+          f"{100 * zero_share:.3f}%, at 1: {100 * one_share:.3f}%")
